@@ -1,0 +1,407 @@
+"""Pins of the fp64 oracle to facts the pages and the mathematics fix (CPU only).
+
+Each pin is chosen so that a plausible mistake in the oracle -- a dropped scale, a wrong
+sign, a transposed operand, an off-by-one in a mask bound, a wrong GQA head mapping, a
+log base, a merge weight -- fails at least one of them.  Library special cases use torch's
+CPU float64 SDPA with masks built here independently of the oracle's ``visible``.
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle import (MASK_CAUSAL, MASK_DOCUMENT_CAUSAL, MASK_NONE, MASK_SLIDING_CAUSAL,
+                    TILE_EMPTY, TILE_FULL, TILE_PARTIAL)
+import workloads
+from workloads import accounting
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _rows(name):
+    out = []
+    with open(os.path.join(GOLDEN, name), encoding="utf-8") as f:
+        for line in f:
+            line = line.strip()
+            if line and not line.startswith("#"):
+                out.append(line)
+    return out
+
+
+def _one_row(scores, scale=1.0):
+    """Attention of one query over keys whose scaled scores are ``scores``: q = [1],
+    k_j = [s_j], V = identity so that O is the probability row."""
+    s = np.asarray(scores, dtype=np.float64)
+    q = np.ones((1, 1, 1, 1))
+    k = (s / scale).reshape(1, 1, -1, 1)
+    v = np.eye(len(s)).reshape(1, 1, len(s), len(s))
+    O, lse = oracle.attention(q, k, v, scale=scale)
+    return O[0, 0, 0], lse[0, 0, 0]
+
+
+# --------------------------------------------------------------------- worked examples
+
+def test_worked_softmax_example_figure4():
+    for line in _rows("softmax_row_worked_example.txt"):
+        name, scores, qty, printed, tol = line.split()
+        scores = [float(x) for x in scores.split(",")]
+        printed, tol = float(printed), float(tol)
+        p, lse = _one_row(scores)
+        expsum = math.exp(lse)            # LSE is ln(sum exp(s)) when the max is 0
+        if qty == "p0":
+            got = p[0]
+        elif qty == "expsum":
+            got = expsum
+        elif qty == "exp2":
+            got = (expsum - 2.0) / 2.0    # the two keys of score 2 share the rest
+        else:
+            raise AssertionError(qty)
+        assert abs(got - printed) <= tol + 1e-12, (name, qty, got, printed)
+        assert abs(p.sum() - 1.0) < 1e-15
+
+
+def test_partial_softmax_is_not_the_row_softmax_but_merges_to_it():
+    # Figure 4: the first two keys alone give 0.5 each, not 0.25 / ~0.06.
+    p_part, lse_a = _one_row([0.0, 0.0])
+    p_full, lse_full = _one_row([0.0, 0.0, 2.0, 2.0])
+    assert p_part[0] == 0.5 and abs(p_full[0] - 1 / (2 + 2 * math.e ** 2)) < 1e-15
+    # the other half, then the rescaling merge of the two partial results
+    p_b, lse_b = _one_row([2.0, 2.0])
+    o_a = np.concatenate([p_part, [0, 0]])
+    o_b = np.concatenate([[0, 0], p_b])
+    O, lse = oracle.merge_partials(np.stack([o_a, o_b])[None], np.array([[lse_a, lse_b]]))
+    assert np.allclose(O[0], p_full, atol=1e-15, rtol=0)
+    assert abs(lse[0] - lse_full) < 1e-14
+
+
+def test_causal_tile_example_figure3():
+    T = 4
+    for line in _rows("causal_tile_example.txt"):
+        qi, keys = line.split()
+        want = sorted(int(x) for x in keys.split(","))
+        vis = oracle.visible(int(qi), np.arange(T), MASK_CAUSAL)
+        assert sorted(np.nonzero(vis)[0].tolist()) == want
+    # The tile (queries 2,3 x keys 0,1) is entirely visible, yet the rows' denominators
+    # need keys outside it: the tile alone gives a different probability.
+    rng = np.random.default_rng(0)
+    q = rng.standard_normal((1, 1, T, 8))
+    k = rng.standard_normal((1, 1, T, 8))
+    v = rng.standard_normal((1, 1, T, 8))
+    assert oracle.tile_map(1, T, T, MASK_CAUSAL, block_q=2, block_kv=2)[0, 1, 0] == TILE_FULL
+    _, lse_full = oracle.attention(q, k, v, mask_kind=MASK_CAUSAL)
+    _, lse_tile = oracle.attention_head(q[0, 0, 2:4], np.arange(2, 4), k[0, 0, :2],
+                                        v[0, 0, :2], 1 / math.sqrt(8), MASK_CAUSAL)
+    assert np.all(lse_tile < lse_full[0, 0, 2:4])
+
+
+# --------------------------------------------------------------------------- invariants
+
+def _rand_qkv(B, Hq, Hkv, N, d, seed, std=1.0, Nk=None):
+    rng = np.random.default_rng(seed)
+    Nk = N if Nk is None else Nk
+    return (std * rng.standard_normal((B, Hq, N, d)), std * rng.standard_normal((B, Hkv, Nk, d)),
+            std * rng.standard_normal((B, Hkv, Nk, d)))
+
+
+DOCS_SMALL = np.array([0, 5, 6, 13, 20], dtype=np.int32)   # lengths 5, 1, 7, 7
+MASKS = [(MASK_NONE, 0, None), (MASK_CAUSAL, 0, None), (MASK_SLIDING_CAUSAL, 3, None),
+         (MASK_DOCUMENT_CAUSAL, 0, DOCS_SMALL)]
+
+
+@pytest.mark.parametrize("mask_kind,window,docs", MASKS)
+def test_rows_sum_to_one_and_masked_probabilities_are_zero(mask_kind, window, docs):
+    q, k, v = _rand_qkv(1, 1, 1, 20, 16, 1)
+    rows = np.arange(20)
+    _, _, P = oracle.attention_head(q[0, 0], rows, k[0, 0], v[0, 0], 0.25, mask_kind, window,
+                                    0.0, docs, return_probs=True)
+    assert np.all(np.abs(P.sum(axis=1) - 1.0) < 1e-12)
+    vis = oracle.visible(rows[:, None], rows[None, :], mask_kind, window, docs)
+    assert np.all(P[~vis] == 0.0)
+    assert np.all(P[vis] > 0.0)
+
+
+def _visible_counts_by_hand(N, mask_kind, window, docs):
+    """Number of keys each query row sees, by counting the definition's interval."""
+    out = []
+    for i in range(N):
+        if mask_kind == MASK_NONE:
+            out.append(N)
+        elif mask_kind == MASK_CAUSAL:
+            out.append(i + 1)
+        elif mask_kind == MASK_SLIDING_CAUSAL:
+            out.append(min(i, window) + 1)
+        else:
+            start = max(int(o) for o in docs if o <= i)
+            out.append(i - start + 1)
+    return out
+
+
+@pytest.mark.parametrize("mask_kind,window,docs", MASKS)
+def test_equal_scores_give_mean_of_visible_values(mask_kind, window, docs):
+    N, d = 20, 8
+    _, k, v = _rand_qkv(1, 1, 1, N, d, 2)
+    q = np.zeros((1, 1, N, d))                   # every score 0
+    O, lse = oracle.attention(q, k, v, mask_kind=mask_kind, window=window, doc_offsets=docs)
+    counts = _visible_counts_by_hand(N, mask_kind, window, docs)
+    for i in range(N):
+        if mask_kind == MASK_NONE:
+            lo, hi = 0, N
+        elif mask_kind == MASK_CAUSAL:
+            lo, hi = 0, i + 1
+        elif mask_kind == MASK_SLIDING_CAUSAL:
+            lo, hi = max(0, i - window), i + 1
+        else:
+            lo, hi = max(int(o) for o in docs if o <= i), i + 1
+        assert hi - lo == counts[i]
+        assert np.allclose(O[0, 0, i], v[0, 0, lo:hi].mean(axis=0), atol=1e-14, rtol=0)
+        assert abs(lse[0, 0, i] - math.log(counts[i])) < 1e-14
+
+
+def test_causal_row0_returns_v0_and_its_own_score():
+    q, k, v = _rand_qkv(2, 4, 2, 9, 16, 3)
+    scale = 0.3
+    O, lse = oracle.attention(q, k, v, scale=scale, mask_kind=MASK_CAUSAL)
+    for b in range(2):
+        for h in range(4):
+            hk = h // 2
+            assert np.array_equal(O[b, h, 0], v[b, hk, 0])
+            s00 = scale * float(np.dot(q[b, h, 0], k[b, hk, 0]))
+            assert abs(lse[b, h, 0] - s00) < 1e-13
+
+
+# ------------------------------------------------------------- library special cases
+
+def _torch_mask(N, mask_kind, window, docs):
+    m = torch.ones(N, N, dtype=torch.bool)
+    if mask_kind in (MASK_CAUSAL, MASK_SLIDING_CAUSAL, MASK_DOCUMENT_CAUSAL):
+        m = torch.tril(m)
+    if mask_kind == MASK_SLIDING_CAUSAL:
+        m = m & torch.triu(torch.ones(N, N, dtype=torch.bool), diagonal=-window)
+    if mask_kind == MASK_DOCUMENT_CAUSAL:
+        blk = torch.zeros(N, N, dtype=torch.bool)
+        for s, e in zip(docs[:-1], docs[1:]):
+            blk[s:e, s:e] = True
+        m = m & blk
+    return m
+
+
+@pytest.mark.parametrize("mask_kind,window,docs", MASKS)
+@pytest.mark.parametrize("Hq,Hkv", [(4, 4), (4, 2), (6, 1)])
+def test_matches_torch_sdpa_float64(mask_kind, window, docs, Hq, Hkv):
+    B, N, d = 2, 20, 16
+    q, k, v = _rand_qkv(B, Hq, Hkv, N, d, 4)
+    scale = 0.17
+    O, lse = oracle.attention(q, k, v, scale=scale, mask_kind=mask_kind, window=window,
+                              doc_offsets=docs)
+    tq, tk, tv = (torch.from_numpy(x) for x in (q, k, v))
+    G = Hq // Hkv
+    tk = tk.repeat_interleave(G, dim=1)
+    tv = tv.repeat_interleave(G, dim=1)
+    if mask_kind == MASK_CAUSAL:
+        ref = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, is_causal=True,
+                                                               scale=scale)
+    else:
+        ref = torch.nn.functional.scaled_dot_product_attention(
+            tq, tk, tv, attn_mask=_torch_mask(N, mask_kind, window, docs), scale=scale)
+    assert np.allclose(O, ref.numpy(), atol=1e-12, rtol=0)
+    S = torch.einsum("bhid,bhjd->bhij", tq, tk) * scale
+    S = S.masked_fill(~_torch_mask(N, mask_kind, window, docs), float("-inf"))
+    assert np.allclose(lse, torch.logsumexp(S, dim=-1).numpy(), atol=1e-12, rtol=0)
+
+
+def test_non_square_unmasked_and_default_scale():
+    q, k, v = _rand_qkv(1, 2, 2, 3, 32, 5, Nk=11)
+    O, lse = oracle.attention(q, k, v)            # scale None -> 1/sqrt(d)
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        *(torch.from_numpy(x) for x in (q, k, v)))
+    assert np.allclose(O, ref.numpy(), atol=1e-12, rtol=0)
+
+
+# ------------------------------------------------------------------------------ soft-cap
+
+def test_softcap_limits():
+    q, k, v = _rand_qkv(1, 2, 1, 16, 8, 6, std=3.0)
+    O0, l0 = oracle.attention(q, k, v, mask_kind=MASK_CAUSAL)
+    O1, l1 = oracle.attention(q, k, v, mask_kind=MASK_CAUSAL, softcap=1e9)
+    assert np.allclose(O0, O1, atol=1e-12) and np.allclose(l0, l1, atol=1e-12)
+    s = np.linspace(-500, 500, 101)
+    c = oracle.softcap_scores(s, 50.0)
+    assert np.all(np.abs(c) < 50.0) and np.allclose(c, -oracle.softcap_scores(-s, 50.0))
+    assert abs(oracle.softcap_scores(np.array([1e4]), 50.0)[0] - 50.0) < 1e-12
+    assert np.all(np.diff(c) > 0)
+
+
+def test_softcap_acts_on_the_scaled_score():
+    # one visible key: LSE equals the (capped) score itself.  q.k = 100, scale 0.5 ->
+    # scaled score 50; capped at c = 50: 50 * tanh(1) = 38.0797...
+    q = np.array([10.0]).reshape(1, 1, 1, 1)
+    k = np.array([10.0]).reshape(1, 1, 1, 1)
+    v = np.ones((1, 1, 1, 1))
+    _, lse = oracle.attention(q, k, v, scale=0.5, softcap=50.0)
+    assert abs(lse[0, 0, 0] - 38.07970779778824) < 1e-12
+
+
+# ---------------------------------------------------------------- tiled and split merges
+
+@pytest.mark.parametrize("mask_kind,window,docs", MASKS)
+@pytest.mark.parametrize("bq,bk", [(1, 1), (2, 3), (3, 7), (5, 2), (16, 16)])
+def test_tiled_online_softmax_equals_full(mask_kind, window, docs, bq, bk):
+    q, k, v = _rand_qkv(1, 2, 1, 20, 8, 7, std=2.0)
+    O, lse = oracle.attention(q, k, v, mask_kind=mask_kind, window=window, doc_offsets=docs,
+                              softcap=30.0)
+    Ot, lt = oracle.attention_tiled_online(q, k, v, block_q=bq, block_kv=bk,
+                                           mask_kind=mask_kind, window=window,
+                                           doc_offsets=docs, softcap=30.0)
+    assert np.allclose(O, Ot, atol=1e-12, rtol=0)
+    assert np.allclose(lse, lt, atol=1e-12, rtol=0)
+
+
+@pytest.mark.parametrize("splits", [1, 2, 3, 8, 37])
+def test_split_kv_merge_equals_unsplit(splits):
+    B, Hq, Hkv, T, d = 2, 8, 2, 37, 16
+    rng = np.random.default_rng(8)
+    q = rng.standard_normal((B, Hq, 1, d))
+    kc = rng.standard_normal((B, Hkv, T, d))
+    vc = rng.standard_normal((B, Hkv, T, d))
+    O, lse, _, _ = oracle.decode_splitkv(q, kc, vc, splits)
+    Ou, lu = oracle.attention(q, kc, vc)
+    assert np.allclose(O, Ou, atol=1e-12, rtol=0)
+    assert np.allclose(lse, lu, atol=1e-12, rtol=0)
+
+
+def test_merge_with_fully_masked_splits():
+    # document mask: the splits outside the query's document have LSE = -inf (weight 0)
+    N, d = 20, 8
+    q, k, v = _rand_qkv(1, 1, 1, N, d, 9)
+    O, lse = oracle.attention(q, k, v, mask_kind=MASK_DOCUMENT_CAUSAL, doc_offsets=DOCS_SMALL)
+    rows = np.arange(N)
+    parts_o, parts_l = [], []
+    for s0, s1 in oracle.split_bounds(N, 5):
+        cols = np.arange(s0, s1)
+        o, l = oracle.attention_head(q[0, 0], rows, k[0, 0, s0:s1], v[0, 0, s0:s1],
+                                     1 / math.sqrt(d), MASK_DOCUMENT_CAUSAL, 0, 0.0,
+                                     DOCS_SMALL, kv_idx=cols)
+        parts_o.append(o)
+        parts_l.append(l)
+    assert np.isneginf(np.stack(parts_l, axis=1)).any()
+    Om, lm = oracle.merge_partials(np.stack(parts_o, axis=1), np.stack(parts_l, axis=1))
+    assert np.allclose(Om, O[0, 0], atol=1e-12, rtol=0)
+    assert np.allclose(lm, lse[0, 0], atol=1e-12, rtol=0)
+
+
+def test_fully_masked_row_gives_zero_and_minus_inf():
+    # kv positions beyond the keys of a doc never seen: use a sliding window of -1 so no
+    # key is visible at all (window < 0 keeps nothing), the degenerate case of reading c6
+    q, k, v = _rand_qkv(1, 1, 1, 4, 8, 10)
+    O, lse = oracle.attention(q, k, v, mask_kind=MASK_SLIDING_CAUSAL, window=-1)
+    assert np.all(O == 0.0) and np.all(np.isneginf(lse))
+    Ot, lt = oracle.attention_tiled_online(q, k, v, mask_kind=MASK_SLIDING_CAUSAL, window=-1)
+    assert np.all(Ot == 0.0) and np.all(np.isneginf(lt))
+
+
+# ------------------------------------------------------------------ tile maps and counts
+
+def _tile_class_by_intervals(i, j, N, bq, bk, mask_kind, window, docs):
+    """Classify a tile from each row's visible key interval [lo(q), hi(q)]."""
+    q0, q1 = i * bq, min(N, (i + 1) * bq)
+    k0, k1 = j * bk, min(N, (j + 1) * bk)
+    full, any_ = True, False
+    for qq in range(q0, q1):
+        if mask_kind == MASK_NONE:
+            lo, hi = 0, N - 1
+        elif mask_kind == MASK_CAUSAL:
+            lo, hi = 0, qq
+        elif mask_kind == MASK_SLIDING_CAUSAL:
+            lo, hi = max(0, qq - window), qq
+        else:
+            lo, hi = max(int(o) for o in docs if o <= qq), qq
+        a, b = max(lo, k0), min(hi, k1 - 1)
+        if a <= b:
+            any_ = True
+        if not (lo <= k0 and k1 - 1 <= hi):
+            full = False
+    return TILE_FULL if full else (TILE_PARTIAL if any_ else TILE_EMPTY)
+
+
+@pytest.mark.parametrize("mask_kind,window,docs", MASKS)
+@pytest.mark.parametrize("bq,bk", [(4, 4), (3, 5), (8, 2)])
+def test_tile_map_small_against_intervals(mask_kind, window, docs, bq, bk):
+    N = 20
+    tm = oracle.tile_map(2, N, N, mask_kind, window, docs, bq, bk)
+    for i in range(tm.shape[1]):
+        for j in range(tm.shape[2]):
+            want = _tile_class_by_intervals(i, j, N, bq, bk, mask_kind, window, docs)
+            assert tm[0, i, j] == want and tm[1, i, j] == want
+
+
+def test_tile_map_causal_4096_counts():
+    tm = oracle.tile_map(1, 4096, 4096, MASK_CAUSAL)
+    assert (tm == TILE_FULL).sum() == 496 and (tm == TILE_PARTIAL).sum() == 32
+    assert np.all(np.diag(tm[0]) == TILE_PARTIAL)
+
+
+@pytest.mark.slow
+def test_tile_map_sliding_16384_w1024_counts():
+    # rows i >= 8 of 128-row tiles: 7 full tiles (i-7..i-1) and 2 partial (i-8, i);
+    # rows i < 8: i full tiles and the diagonal partial.
+    tm = oracle.tile_map(1, 16384, 16384, MASK_SLIDING_CAUSAL, window=1024)
+    full = sum(i for i in range(8)) + 120 * 7
+    part = 8 + 120 * 2
+    assert (tm == TILE_FULL).sum() == full == 868
+    assert (tm == TILE_PARTIAL).sum() == part == 248
+
+
+def test_visible_pair_closed_forms_match_element_counts():
+    docs = workloads.doc_offsets_for(3000, 100, 700, seed=3)
+    for (kind, w, dd) in [(MASK_NONE, 0, None), (MASK_CAUSAL, 0, None),
+                          (MASK_SLIDING_CAUSAL, 257, None), (MASK_SLIDING_CAUSAL, 5000, None),
+                          (MASK_DOCUMENT_CAUSAL, 0, docs)]:
+        assert accounting.visible_pairs(3000, 3000, kind, w, dd) == \
+            oracle.visible_pairs(3000, 3000, kind, w, dd)
+    assert accounting.visible_pairs(16384, 16384, MASK_SLIDING_CAUSAL, 1024) == 16268800
+
+
+def test_document_generator():
+    lens = workloads.doc_lengths(32768, 512, 4096, seed=0)
+    assert sum(lens) == 32768 and all(512 <= x <= 4096 for x in lens[:-1])
+    assert 1 <= lens[-1] <= 4096
+    offs = workloads.doc_offsets_for(32768)
+    assert offs[0] == 0 and offs[-1] == 32768 and np.all(np.diff(offs) > 0)
+    ids = oracle.document_ids(np.arange(32768), offs)
+    assert np.array_equal(np.bincount(ids), np.array(lens))
+
+
+# ------------------------------------------------------------- byte-accounting closed forms
+
+def test_score_matrix_sizes_printed_on_pages():
+    units = {"GB": 1e9, "MiB": 2 ** 20}
+    for line in _rows("memory_sizes.txt"):
+        _, B, H, N, eb, printed, unit, tol = [x.strip() for x in line.split("|")]
+        got = accounting.score_matrix_bytes(int(B), int(H), int(N), int(eb)) / units[unit]
+        assert abs(got - float(printed)) <= float(tol) + 5e-3, line
+    # FlexAttention page, section 1: 32k tokens -> more than a billion scores per head
+    assert 32768 * 32768 > 1e9
+
+
+def test_gqa_kv_cache_exercise():
+    # "3.7 어텐션 II", exercise 3: Hq=32, d=128, fp16, T=16384, B=1; K and V both.
+    mib = 2 ** 20
+    assert accounting.kv_cache_bytes(32, 16384, 128) == 256 * mib
+    assert accounting.kv_cache_bytes(8, 16384, 128) == 64 * mib
+    assert accounting.kv_cache_bytes(1, 16384, 128) == 8 * mib
+    # the decode workload's KV cache: 8 GiB per step
+    w = workloads.DECODE
+    assert accounting.decode_kv_bytes(w.B, w.Hkv, w.Nk, w.d) == 8 * 2 ** 30
+
+
+def test_useful_flops_of_the_prefill_workloads():
+    w = workloads.CAUSAL_MHA
+    f = accounting.prefill_useful_flops(w.B, w.Hq, w.Nq, w.Nk, w.d, w.mask_kind)
+    assert f == 4 * 128 * (4096 * 4097 // 2) * 8 * 32      # 1.0998 TFLOP
+    w = workloads.DOC_SOFTCAP
+    docs = workloads.workload_doc_offsets(w)
+    pairs = accounting.visible_pairs(w.Nq, w.Nk, w.mask_kind, 0, docs)
+    assert pairs == sum(L * (L + 1) // 2 for L in workloads.doc_lengths(32768))
