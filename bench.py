@@ -1,0 +1,450 @@
+#!/usr/bin/env python3
+"""Benchmark of the fused attention hot path on B200.
+
+Headline (``value``): useful prefill TFLOP/s of ``attn_fwd`` on the causal multi-head
+workload (B=8, H=32, N=4096, d=128, causal): 4*d flops per visible (query, key) pair.
+One step is one ``attn_fwd`` call, which performs every prefill row of the hot path in one
+kernel (tile classification, TMA loads, QK^T, mask, online softmax, PV, epilogue).
+The ``decode`` object reports the split-KV decode workload (B=64, Hq=32, Hkv=8, T=32768,
+d=128): KV-cache GB/s and tokens/s of one ``attn_decode_splitkv`` call (split + merge).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Multi-GPU: one process per GPU (torchrun); every rank runs the same workload on its own GPU
+(independent replicas of (batch, head) units, no collective on the data path); the value is
+all ranks' work divided by the slowest rank's device time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import workloads  # noqa: E402
+from workloads import accounting  # noqa: E402
+
+METRIC = "prefill useful TFLOPS & decode KV GB/s on 1 B200, as % of roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_BYTES = 126 * 2 ** 20
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except (OSError, ValueError):
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ---------------------------------------------------------------- clocks during timing
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ distributed plumbing
+def dist_setup(n_gpus: int):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(world, x: float) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------------- CPU baseline
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return len(os.sched_getaffinity(0))
+
+
+def oracle_prefill_sample(w: workloads.Workload, budget_s: float, max_heads: int = 256):
+    """Times the fp64 oracle on whole heads of the workload until ``budget_s`` is spent.
+    Returns (useful TFLOP/s, heads done, seconds)."""
+    import oracle
+    q, k, v = (x.float().numpy() for x in _cpu_head_inputs(w, 0))
+    docs = workloads.workload_doc_offsets(w)
+    pairs = accounting.visible_pairs(w.Nq, w.Nk, w.mask_kind, w.window, docs)
+    G = w.Hq // w.Hkv
+    rows = np.arange(w.Nq)
+    done, t0 = 0, time.perf_counter()
+    while done < max_heads:
+        h = done % w.Hq
+        for r0 in range(0, w.Nq, 256):
+            rr = rows[r0:r0 + 256]
+            oracle.attention_head(q[h, rr], rr, k[h // G], v[h // G], w.scale, w.mask_kind,
+                                  w.window, w.softcap, docs)
+        done += 1
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return 4 * w.d * pairs * done / dt / 1e12, done, dt
+
+
+def _cpu_head_inputs(w: workloads.Workload, b: int):
+    """q[b], k[b], v[b] of the workload, drawn on the CPU (same seeds as make_inputs)."""
+    q = workloads.randn_bf16((1, w.Hq, w.Nq, w.d), w.seed, 0, w.input_std)[0]
+    k = workloads.randn_bf16((1, w.Hkv, w.Nk, w.d), w.seed, 1, w.input_std)[0]
+    v = workloads.randn_bf16((1, w.Hkv, w.Nk, w.d), w.seed, 2, w.input_std)[0]
+    return q, k, v
+
+
+# ----------------------------------------------------------------- traffic from ncu
+def recorded_traffic(kernel_key: str):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on the current
+    kernel source (the summary stores a hash of the sources it measured)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f).get(kernel_key)
+    except (OSError, ValueError):
+        return None
+    if not rec:
+        return None
+    from io_aware_softmax_b200 import build as _b
+    import hashlib
+    h = hashlib.sha256()
+    for name in rec.get("sources", []):
+        with open(os.path.join(_b.CSRC, name), "rb") as f:
+            h.update(f.read())
+    return rec.get("bytes_per_launch") if h.hexdigest() == rec.get("sha256") else None
+
+
+# ----------------------------------------------------------------------------- our arm
+def time_launches(fn, steps: int, world: int):
+    import torch
+    stream = torch.cuda.current_stream()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    t_all0 = torch.cuda.Event(enable_timing=True)
+    t_all1 = torch.cuda.Event(enable_timing=True)
+    t_all0.record(stream)
+    for i in range(steps):
+        starts[i].record(stream)
+        fn()
+        ends[i].record(stream)
+    t_all1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    per = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    total_ms = t_all0.elapsed_time(t_all1)
+    return total_ms, per
+
+
+def run_ours(args, world, rank, local):
+    import torch
+    import io_aware_softmax_b200 as attn
+
+    peaks, peak_src = load_peaks()
+    w = workloads.CAUSAL_MHA
+    dev = torch.device("cuda", torch.cuda.current_device())
+    q, k, v = workloads.make_inputs(w, device=dev)
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.Hq, w.Nq), dtype=torch.float32, device=dev)
+    flops = accounting.prefill_useful_flops(w.B, w.Hq, w.Nq, w.Nk, w.d, w.mask_kind)
+
+    def step():
+        attn.attn_fwd(q, k, v, scale=w.scale, mask=w.mask_kind, out=o, lse=lse)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if attn.device_status() != 0:
+        raise RuntimeError("device status not ok after warm-up")
+    with ClockSampler(local) as clk:
+        total_ms, per = time_launches(step, args.steps, world)
+    if attn.device_status() != 0:
+        raise RuntimeError("device status not ok after timed steps")
+    ms_step = max_over_ranks(world, total_ms / args.steps)
+    kernel_ms = max_over_ranks(world, sum(per) / len(per))
+    value = flops * world / (ms_step * 1e-3) / 1e12
+    achieved = flops / (kernel_ms * 1e-3) / 1e12
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    out = {
+        "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.Nq, "d": w.d,
+                   "mask": "causal", "useful_tflop_per_step": round(flops / 1e12, 4),
+                   "l2": "inputs larger than L2 (q+k+v %.0f MB > 126 MB)" %
+                         (3 * q.numel() * 2 / 1e6),
+                   "parallelism": f"replicas x{world} (independent (batch, head) units)",
+                   "seed": w.seed},
+        "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak,
+                     "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                     "peak_source": f"bf16_tflops (burst, {peak_src})",
+                     "kernel": "attn_fwd_sm100_kernel<128>",
+                     "traffic": recorded_traffic("prefill_causal_mha")},
+        "gpu_launches": args.steps,
+    }
+    out["clocks"] = clk.summary()
+
+    if not args.no_e2e:
+        out["e2e"] = e2e_prefill(w, args, world, q, k, v)
+    if not args.no_decode:
+        del q, k, v, o, lse
+        torch.cuda.empty_cache()
+        out["decode"] = bench_decode(args, world, local, peaks, peak_src)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        tf, heads, dt = oracle_prefill_sample(w, args.cpu_budget)
+        out["cpu_baseline"] = {"value": round(tf, 5), "unit": "TFLOP/s",
+                               "cores": blas_threads(), "kind": "oracle",
+                               "sample": f"{heads} whole heads (4096 query rows each, all keys) "
+                                         f"of {w.name}, fp64, {dt:.1f} s"}
+    return out
+
+
+def e2e_prefill(w, args, world, q, k, v):
+    """Same metric through the public API with host buffers: every step copies q, k, v from
+    pinned host memory, runs attn_fwd and reads O and LSE back."""
+    import torch
+    import io_aware_softmax_b200 as attn
+    hq, hk, hv = (x.cpu().pin_memory() for x in (q, k, v))
+    ho = torch.empty(q.shape, dtype=torch.bfloat16).pin_memory()
+    hl = torch.empty((w.B, w.Hq, w.Nq), dtype=torch.float32).pin_memory()
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    do = torch.empty_like(q)
+    dl = torch.empty((w.B, w.Hq, w.Nq), dtype=torch.float32, device=q.device)
+
+    def step():
+        dq.copy_(hq, non_blocking=True)
+        dk.copy_(hk, non_blocking=True)
+        dv.copy_(hv, non_blocking=True)
+        attn.attn_fwd(dq, dk, dv, scale=w.scale, mask=w.mask_kind, out=do, lse=dl)
+        ho.copy_(do, non_blocking=True)
+        hl.copy_(dl, non_blocking=True)
+
+    steps = max(3, min(args.steps, 10))
+    for _ in range(2):
+        step()
+    total_ms, _ = time_launches(step, steps, world)
+    ms = max_over_ranks(world, total_ms / steps)
+    flops = accounting.prefill_useful_flops(w.B, w.Hq, w.Nq, w.Nk, w.d, w.mask_kind)
+    return {"value": round(flops * world / (ms * 1e-3) / 1e12, 3), "unit": "TFLOP/s",
+            "h2d_bytes_per_step": 3 * q.numel() * 2, "d2h_bytes_per_step": q.numel() * 2 +
+            w.B * w.Hq * w.Nq * 4, "steps": steps, "ms_per_step": round(ms, 3)}
+
+
+def bench_decode(args, world, local, peaks, peak_src):
+    import torch
+    import io_aware_softmax_b200 as attn
+    w = workloads.DECODE
+    dev = torch.device("cuda", torch.cuda.current_device())
+    q, kc, vc = workloads.make_inputs(w, device=dev)
+    S = attn.default_splits(w.B, w.Hkv, w.Nk, dev.index)
+    ws = torch.empty(attn.decode_workspace_bytes(w.B, w.Hq, w.d, S), dtype=torch.uint8,
+                     device=dev)
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.Hq, 1), dtype=torch.float32, device=dev)
+
+    def step():
+        attn.attn_decode(q, kc, vc, scale=w.scale, num_splits=S, workspace=ws, out=o, lse=lse)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        total_ms, per = time_launches(step, args.steps, world)
+    if attn.device_status() != 0:
+        raise RuntimeError("device status not ok after decode steps")
+    ms = max_over_ranks(world, total_ms / args.steps)
+    call_ms = max_over_ranks(world, sum(per) / len(per))
+    kv = accounting.decode_kv_bytes(w.B, w.Hkv, w.Nk, w.d)
+    io = accounting.decode_io_bytes(w.B, w.Hq, w.Hkv, w.Nk, w.d)
+    peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    gbs = kv * world / (ms * 1e-3) / 1e9
+    res = {"workload": w.name, "value": round(gbs, 1), "unit": "GB/s (KV cache)",
+           "tokens_per_s": round(w.B * world / (ms * 1e-3), 1), "ms_per_step": round(ms, 4),
+           "num_splits": S, "kv_bytes_per_step": kv,
+           "roofline": {"bound": "hbm", "achieved": round(io / (call_ms * 1e-3) / 1e9, 1),
+                        "peak": peak, "unit": "GB/s", "frac": round(io / (call_ms * 1e-3) / 1e9
+                                                                   / peak, 4),
+                        "peak_source": f"hbm_gbs ({peak_src})",
+                        "kernel": "attn_decode_split_kernel + attn_merge_kernel (one call)",
+                        "traffic": recorded_traffic("decode")},
+           "gpu_launches": 2 * args.steps, "clocks": clk.summary()}
+    if not args.no_e2e:
+        hk, hv = kc.cpu().pin_memory(), vc.cpu().pin_memory()
+        hq = q.cpu().pin_memory()
+        ho = torch.empty(q.shape, dtype=torch.bfloat16).pin_memory()
+        hl = torch.empty((w.B, w.Hq, 1), dtype=torch.float32).pin_memory()
+
+        def e2e_step():
+            q.copy_(hq, non_blocking=True)
+            kc.copy_(hk, non_blocking=True)
+            vc.copy_(hv, non_blocking=True)
+            attn.attn_decode(q, kc, vc, scale=w.scale, num_splits=S, workspace=ws, out=o,
+                             lse=lse)
+            ho.copy_(o, non_blocking=True)
+            hl.copy_(lse, non_blocking=True)
+
+        e2e_step()
+        total, _ = time_launches(e2e_step, 3, world)
+        ems = max_over_ranks(world, total / 3)
+        res["e2e"] = {"value": round(kv * world / (ems * 1e-3) / 1e9, 2), "unit": "GB/s",
+                      "h2d_bytes_per_step": kv + q.numel() * 2,
+                      "d2h_bytes_per_step": q.numel() * 2 + w.B * w.Hq * 4, "steps": 3}
+    return res
+
+
+# ------------------------------------------------------------------------ reference arm
+def run_reference(args, world, rank):
+    """The fp64 CPU oracle, as it stands, on the host cores: each step is one whole head of
+    the causal multi-head workload (a bounded sample of the same workload)."""
+    import oracle
+    w = workloads.CAUSAL_MHA
+    q, k, v = (x.float().numpy() for x in _cpu_head_inputs(w, 0))
+    pairs = accounting.visible_pairs(w.Nq, w.Nk, w.mask_kind)
+    rows = np.arange(w.Nq)
+
+    def step(h):
+        for r0 in range(0, w.Nq, 256):
+            rr = rows[r0:r0 + 256]
+            oracle.attention_head(q[h, rr], rr, k[h], v[h], w.scale, w.mask_kind)
+
+    for i in range(args.warmup):
+        step(i % w.Hq)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        step((args.warmup + i) % w.Hq)
+    dt = time.perf_counter() - t0
+    ms = dt * 1e3 / args.steps
+    value = 4 * w.d * pairs / (ms * 1e-3) / 1e12
+    cores = blas_threads()
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 5), "unit": "TFLOP/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(ms, 2), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.Nq, "d": w.d,
+                   "mask": "causal", "sample_per_step": "one whole head (b=0), 4096 rows"},
+        "cpu_baseline": {"value": round(value, 5), "unit": "TFLOP/s", "cores": cores,
+                         "kind": "oracle", "sample": "one whole head of the workload per step"},
+        "e2e": {"value": round(value, 5), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle time")
+    args = ap.parse_args(argv)
+    args.warmup = max(3, args.warmup)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args, world, rank)), flush=True)
+        return 0
+    world, rank, local = dist_setup(args.gpus)
+    out = run_ours(args, world, rank, local)
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,152 @@
+/*
+ * io_aware_softmax_b200 -- exact fused attention on NVIDIA B200 (sm_100a), C ABI.
+ *
+ * What is computed (the plain definition the kernels reproduce up to rounding):
+ *   O = softmax(scale * Q K^T + mask) V, and the row log-sum-exp LSE = ln sum_j exp(s_ij)
+ * ("PyTorch FlexAttention 도입 분석", section 1; "FlashAttention 논문 분석: IO-Aware Exact
+ * Attention", section "수학적 정의"; the row statistics m and l that the forward keeps for a
+ * recomputing backward, section "Recomputation 전략").  The score matrix S and the
+ * probabilities P never reach device memory: the softmax is taken tile by tile with the
+ * online rescaling of "Online Softmax와 블록 단위 누적" / "알고리즘 의사코드" on the same page.
+ *
+ * Conventions shared by every entry point:
+ *   - Tensors are caller-owned DEVICE memory, contiguous, row-major in the order given
+ *     ([B, H, N, d] as in PyTorch, "사례 2: 텐서 형태 불일치" on the FlashAttention page).
+ *     bf16 arrays are passed as void*.  Every pointer must be 16-byte aligned.
+ *   - Calls are asynchronous on `stream`; they never synchronise, never allocate and keep
+ *     no state across calls except a per-process cache of device attributes, so they may be
+ *     recorded into a CUDA graph with fixed shapes ("CUDA 그래프와의 호환성").
+ *   - Arguments are validated before anything is launched; an unsupported case returns
+ *     ATTN_ERR_UNSUPPORTED and nothing runs -- there is no fallback path ("3.7 어텐션 II",
+ *     section 3.7.3, on diagnosing silent fallbacks: here the failure is the diagnosis).
+ *   - Kernels never hang: every wait inside them is bounded.  A wait that runs out records
+ *     a device-side error and the kernel returns; attn_get_device_status() reports it.
+ */
+#ifndef IO_AWARE_SOFTMAX_B200_ATTN_H
+#define IO_AWARE_SOFTMAX_B200_ATTN_H
+
+#include <stddef.h>
+#include <cuda_runtime_api.h>
+
+#if defined(__GNUC__)
+#define ATTN_API __attribute__((visibility("default")))
+#else
+#define ATTN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Mask hooks ("PyTorch FlexAttention 도입 분석", section 2: score_mod / mask applied to each
+ * scalar score right after Q.K^T).  Every kind other than NONE needs Nq == Nk. */
+typedef enum {
+  ATTN_MASK_NONE = 0,             /* every key visible                                    */
+  ATTN_MASK_CAUSAL = 1,           /* kv <= q                                               */
+  ATTN_MASK_SLIDING_CAUSAL = 2,   /* 0 <= q - kv <= window (window + 1 keys incl. self)    */
+  ATTN_MASK_DOCUMENT_CAUSAL = 3   /* same packed document AND kv <= q                      */
+} attn_mask_kind;
+
+typedef enum {
+  ATTN_OK = 0,
+  ATTN_ERR_INVALID_ARG = -1,      /* null pointer, negative size, bad mask parameters       */
+  ATTN_ERR_UNSUPPORTED = -2,      /* valid request this library does not implement          */
+  ATTN_ERR_MISALIGNED = -3,       /* a pointer is not 16-byte aligned                       */
+  ATTN_ERR_CUDA = -4,             /* a CUDA runtime/driver call failed                      */
+  ATTN_ERR_DEVICE_TIMEOUT = -5,   /* a kernel's bounded wait ran out (see get_device_status)*/
+  ATTN_ERR_WORKSPACE = -6         /* workspace missing or too small                         */
+} attn_status;
+
+typedef enum { ATTN_TILE_EMPTY = 0, ATTN_TILE_PARTIAL = 1, ATTN_TILE_FULL = 2 } attn_tile_class;
+
+/*
+ * attn_fwd -- fused prefill attention forward.
+ * Defining passages: FlashAttention page, "알고리즘 의사코드" (tiled forward returning O, m, l);
+ * "3.7 어텐션 II", 3.7.5 (GQA/MQA: query-head groups share a KV head; sliding window;
+ * soft-cap as a kernel flag) and 3.7.6 (packed documents by cumulative boundaries).
+ *
+ *   q        bf16 [B, Hq,  Nq, d]     k, v  bf16 [B, Hkv, Nk, d]
+ *   o        bf16 [B, Hq,  Nq, d]     (written)   lse  fp32 [B, Hq, Nq] natural log (written)
+ *   d        64 or 128; Hq % Hkv == 0; query head h reads KV head h / (Hq / Hkv)
+ *   scale    multiplies q.k; <= 0 selects 1/sqrt(d)
+ *   mask_kind, window   see attn_mask_kind; window >= 0 for SLIDING_CAUSAL
+ *   softcap  > 0: score s (already scaled) becomes softcap * tanh(s / softcap); <= 0: off
+ *   doc_offsets, num_docs   DOCUMENT_CAUSAL only: device int32 [num_docs + 1], with
+ *            doc_offsets[0] = 0, non-decreasing, doc_offsets[num_docs] = Nk; the same
+ *            documents apply to every batch entry.  Ignored for other masks.
+ * A row with no visible key gets O = 0 and LSE = -inf.  Outputs are rounded to bf16 (RNE).
+ * Errors: INVALID_ARG, UNSUPPORTED (d not in {64,128}; Hq % Hkv != 0; a mask with
+ * Nq != Nk), MISALIGNED, CUDA.  Empty problems (B, Hq or Nq == 0) return ATTN_OK at once.
+ */
+ATTN_API int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+             int Hkv, int Nq, int Nk, int d, float scale, int mask_kind, int window,
+             float softcap, const int* doc_offsets, int num_docs, cudaStream_t stream);
+
+/*
+ * attn_blockmap -- 128x128 block-sparsity map of a mask ("PyTorch FlexAttention 도입 분석",
+ * section 2: BlockMask precomputed in 128 x 128 chunks so empty tiles are skipped).
+ *   map  device uint8 [B, ceil(Nq/128), ceil(Nk/128)] (written): ATTN_TILE_EMPTY when no
+ *        (q, kv) pair of the tile is visible, ATTN_TILE_FULL when all are, else PARTIAL.
+ *        Only pairs with q < Nq and kv < Nk count.
+ * Mask arguments and errors as attn_fwd.
+ */
+ATTN_API int attn_blockmap(int B, int Nq, int Nk, int mask_kind, int window, const int* doc_offsets,
+                  int num_docs, unsigned char* map, cudaStream_t stream);
+
+/*
+ * Split-KV decode ("3.7 어텐션 II", 3.7.4: one query token against the whole KV cache; the
+ * cache axis is split, every split produces partial (m, l, O), and the partials are merged
+ * by the rescaling recurrence).
+ *
+ * attn_decode_workspace_bytes: bytes of device workspace attn_decode_splitkv needs for
+ *   num_splits splits (fp32 partial O [B, Hq, S, d] and LSE [B, Hq, S]).
+ * attn_decode_default_splits: the split count that fills every SM of `device` with whole
+ *   waves of work items for B * Hkv KV heads and cache length T (>= 1).
+ * attn_decode_splitkv:
+ *   q        bf16 [B, Hq, 1, d]           k_cache, v_cache  bf16 [B, Hkv, T, d] contiguous
+ *   o        bf16 [B, Hq, 1, d] (written) lse fp32 [B, Hq, 1] natural log (written)
+ *   scale    <= 0 selects 1/sqrt(d); num_splits <= 0 selects attn_decode_default_splits
+ *   workspace, workspace_bytes  caller-owned device scratch, >= attn_decode_workspace_bytes,
+ *            16-byte aligned; its contents on return are the per-split partials.
+ *   No mask (every cached key is visible).  Hq / Hkv <= 16, d in {64, 128}.
+ * Errors: INVALID_ARG, UNSUPPORTED, MISALIGNED, WORKSPACE, CUDA.  T == 0 writes O = 0 and
+ * LSE = -inf.
+ */
+ATTN_API size_t attn_decode_workspace_bytes(int B, int Hq, int d, int num_splits);
+ATTN_API int attn_decode_default_splits(int B, int Hkv, int T, int device);
+ATTN_API int attn_decode_splitkv(const void* q, const void* k_cache, const void* v_cache, void* o,
+                        float* lse, int B, int Hq, int Hkv, int T, int d, float scale,
+                        int num_splits, void* workspace, size_t workspace_bytes,
+                        cudaStream_t stream);
+
+/*
+ * attn_decode_merge -- merge S partial results per row by the rescaling rule ("3.7 어텐션
+ * II", 3.7.4): L = max_s LSE_s, w_s = exp(LSE_s - L), O = sum_s w_s O_s / sum_s w_s,
+ * LSE = L + ln sum_s w_s.  Partials with LSE = -inf have weight 0.
+ *   o_part fp32 [rows, S, d] (each partial normalised by its own sum); lse_part fp32
+ *   [rows, S]; o bf16 [rows, d] (written); lse fp32 [rows] (written).  d in {64, 128}.
+ * Errors: INVALID_ARG, UNSUPPORTED, MISALIGNED, CUDA.
+ */
+ATTN_API int attn_decode_merge(const float* o_part, const float* lse_part, void* o, float* lse,
+                      long long rows, int num_splits, int d, cudaStream_t stream);
+
+/*
+ * attn_get_device_status -- synchronises `stream`, then returns and clears the device-side
+ * error word of the current device: ATTN_OK, ATTN_ERR_DEVICE_TIMEOUT (a bounded wait in a
+ * kernel ran out; attn_last_error_site() names which), or ATTN_ERR_CUDA if the
+ * synchronisation itself failed.
+ */
+ATTN_API int attn_get_device_status(cudaStream_t stream);
+ATTN_API int attn_last_error_site(void);
+
+/* Human-readable name of a status code (static storage). */
+ATTN_API const char* attn_status_string(int status);
+
+/* Library ABI version (major * 100 + minor). */
+ATTN_API int attn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* IO_AWARE_SOFTMAX_B200_ATTN_H */

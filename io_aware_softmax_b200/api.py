@@ -1,0 +1,166 @@
+"""Python binding of the C ABI: marshals torch tensors (device pointers, sizes, the current
+CUDA stream) into the ``libattn_b200`` entry points.  Every step of the computation runs
+in the library's CUDA kernels; nothing here computes attention.
+"""
+from __future__ import annotations
+
+from typing import Optional, Tuple
+
+import torch
+
+from . import _lib
+
+MASKS = {"none": 0, "causal": 1, "sliding_causal": 2, "document_causal": 3}
+
+ATTN_OK = 0
+
+
+class AttnError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        lib = _lib.load()
+        msg = lib.attn_status_string(status).decode()
+        super().__init__(f"{where}: status {status} ({msg})")
+        self.status = status
+
+
+def _check(status: int, where: str):
+    if status != ATTN_OK:
+        raise AttnError(status, where)
+
+
+def _mask_id(mask) -> int:
+    if isinstance(mask, str):
+        return MASKS[mask]
+    return int(mask)
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream(device: torch.device, stream=None) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return stream.cuda_stream
+
+
+def _need(t: torch.Tensor, name: str, dtype: torch.dtype, dims: int):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.device.type != "cuda":
+        raise ValueError(f"{name} must be on a CUDA device")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.dim() != dims:
+        raise ValueError(f"{name} must have {dims} dimensions")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, scale: Optional[float] = None,
+             mask="none", window: int = 0, softcap: float = 0.0,
+             doc_offsets: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
+             lse: Optional[torch.Tensor] = None, stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Fused prefill attention: q [B,Hq,Nq,d], k/v [B,Hkv,Nk,d] bf16 -> (O bf16, LSE fp32)."""
+    lib = _lib.load()
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, n, torch.bfloat16, 4)
+    B, Hq, Nq, d = q.shape
+    Hkv, Nk = k.shape[1], k.shape[2]
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
+    num_docs = 0
+    if doc_offsets is not None:
+        _need(doc_offsets, "doc_offsets", torch.int32, 1)
+        num_docs = doc_offsets.numel() - 1
+    st = lib.attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, Nq, Nk, d,
+                      float(scale or 0.0), _mask_id(mask), int(window), float(softcap or 0.0),
+                      _ptr(doc_offsets), num_docs, _stream(q.device, stream))
+    _check(st, "attn_fwd")
+    return out, lse
+
+
+def attn_blockmap(B: int, Nq: int, Nk: int, *, mask="none", window: int = 0,
+                  doc_offsets: Optional[torch.Tensor] = None, device=None,
+                  out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """128x128 tile classes (0 empty, 1 partial, 2 full) as uint8 [B, ceil(Nq/128), ceil(Nk/128)]."""
+    lib = _lib.load()
+    if device is None:
+        device = doc_offsets.device if doc_offsets is not None else torch.device("cuda")
+    device = torch.device(device)
+    if out is None:
+        out = torch.empty((B, -(-Nq // 128), -(-Nk // 128)), dtype=torch.uint8, device=device)
+    num_docs = 0
+    if doc_offsets is not None:
+        _need(doc_offsets, "doc_offsets", torch.int32, 1)
+        num_docs = doc_offsets.numel() - 1
+    st = lib.attn_blockmap(B, Nq, Nk, _mask_id(mask), int(window), _ptr(doc_offsets), num_docs,
+                           _ptr(out), _stream(device, stream))
+    _check(st, "attn_blockmap")
+    return out
+
+
+def decode_workspace_bytes(B: int, Hq: int, d: int, num_splits: int) -> int:
+    return int(_lib.load().attn_decode_workspace_bytes(B, Hq, d, num_splits))
+
+
+def default_splits(B: int, Hkv: int, T: int, device: int = 0) -> int:
+    return int(_lib.load().attn_decode_default_splits(B, Hkv, T, device))
+
+
+def attn_decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, *,
+                scale: Optional[float] = None, num_splits: Optional[int] = None,
+                workspace: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
+                lse: Optional[torch.Tensor] = None, stream=None
+                ) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Split-KV decode: q [B,Hq,1,d], caches [B,Hkv,T,d] bf16 -> (O [B,Hq,1,d], LSE [B,Hq,1])."""
+    lib = _lib.load()
+    for t, n in ((q, "q"), (k_cache, "k_cache"), (v_cache, "v_cache")):
+        _need(t, n, torch.bfloat16, 4)
+    B, Hq, nq, d = q.shape
+    if nq != 1:
+        raise ValueError("decode takes one query token per sequence")
+    Hkv, T = k_cache.shape[1], k_cache.shape[2]
+    dev_index = q.device.index if q.device.index is not None else torch.cuda.current_device()
+    S = int(num_splits) if num_splits else default_splits(B, Hkv, T, dev_index)
+    S = max(1, min(S, max(T, 1)))
+    need = decode_workspace_bytes(B, Hq, d, S)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq, 1), dtype=torch.float32, device=q.device)
+    st = lib.attn_decode_splitkv(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(out), _ptr(lse), B,
+                                 Hq, Hkv, T, d, float(scale or 0.0), S, _ptr(workspace),
+                                 workspace.numel() * workspace.element_size(),
+                                 _stream(q.device, stream))
+    _check(st, "attn_decode_splitkv")
+    return out, lse
+
+
+def attn_merge(o_part: torch.Tensor, lse_part: torch.Tensor, *, out: Optional[torch.Tensor] = None,
+               lse: Optional[torch.Tensor] = None, stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Merge partials o_part fp32 [rows, S, d], lse_part fp32 [rows, S] -> (O bf16, LSE fp32)."""
+    lib = _lib.load()
+    _need(o_part, "o_part", torch.float32, 3)
+    _need(lse_part, "lse_part", torch.float32, 2)
+    rows, S, d = o_part.shape
+    if out is None:
+        out = torch.empty((rows, d), dtype=torch.bfloat16, device=o_part.device)
+    if lse is None:
+        lse = torch.empty((rows,), dtype=torch.float32, device=o_part.device)
+    st = lib.attn_decode_merge(_ptr(o_part), _ptr(lse_part), _ptr(out), _ptr(lse), rows, S, d,
+                               _stream(o_part.device, stream))
+    _check(st, "attn_decode_merge")
+    return out, lse
+
+
+def device_status(stream=None, device=None) -> int:
+    """Synchronises the stream and returns (and clears) the library's device error status."""
+    lib = _lib.load()
+    dev = torch.device(device) if device is not None else torch.device("cuda",
+                                                                        torch.cuda.current_device())
+    return int(lib.attn_get_device_status(_stream(dev, stream)))

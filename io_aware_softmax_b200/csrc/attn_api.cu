@@ -1,0 +1,283 @@
+// C-ABI entry points: argument validation, TMA descriptor construction and launches.
+// Nothing here allocates device memory or synchronises (except attn_get_device_status).
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <algorithm>
+#include <cstdint>
+#include <mutex>
+
+#include "../../include/attn.h"
+#include "attn_internal.h"
+#include "sm100_ptx.cuh"
+
+namespace attn {
+
+__device__ uint32_t g_error_word = 0;
+__device__ uint32_t g_error_site = 0;
+
+namespace {
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+// 3-D bf16 tensor map over [z, rows, d] (d innermost) with a (64 x box_rows x 1) box and
+// 128-byte swizzle: one box fills `box_rows` rows of 128 bytes in shared memory.
+bool make_map_3d(CUtensorMap* map, const void* ptr, int d, long long rows, long long z,
+                 int box_rows) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)rows, (cuuint64_t)z};
+  cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)d * 2 * (cuuint64_t)rows};
+  cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+int check_mask(int mask_kind, int window, const int* doc_offsets, int num_docs, int Nq, int Nk) {
+  if (mask_kind < ATTN_MASK_NONE || mask_kind > ATTN_MASK_DOCUMENT_CAUSAL)
+    return ATTN_ERR_INVALID_ARG;
+  if (mask_kind != ATTN_MASK_NONE && Nq != Nk) return ATTN_ERR_UNSUPPORTED;
+  if (mask_kind == ATTN_MASK_SLIDING_CAUSAL && window < 0) return ATTN_ERR_INVALID_ARG;
+  if (mask_kind == ATTN_MASK_DOCUMENT_CAUSAL) {
+    if (doc_offsets == nullptr || num_docs < 1) return ATTN_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(doc_offsets) & 3u) return ATTN_ERR_MISALIGNED;
+  }
+  return ATTN_OK;
+}
+
+MaskParams mask_params(int mask_kind, int window, const int* doc_offsets, int num_docs, int Nq,
+                       int Nk) {
+  MaskParams m;
+  m.kind = mask_kind;
+  m.window = window;
+  m.doc_offsets = doc_offsets;
+  m.num_docs = num_docs;
+  m.Nq = Nq;
+  m.Nk = Nk;
+  return m;
+}
+
+int sm_count(int device) {
+  static int cached[64] = {0};
+  if (device >= 0 && device < 64 && cached[device] > 0) return cached[device];
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, device) != cudaSuccess || n < 1)
+    n = 148;
+  if (device >= 0 && device < 64) cached[device] = n;
+  return n;
+}
+
+int current_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  return dev;
+}
+
+}  // namespace
+}  // namespace attn
+
+using namespace attn;
+
+extern "C" int attn_version(void) { return 100; }
+
+extern "C" const char* attn_status_string(int status) {
+  switch (status) {
+    case ATTN_OK: return "ok";
+    case ATTN_ERR_INVALID_ARG: return "invalid argument";
+    case ATTN_ERR_UNSUPPORTED: return "unsupported configuration";
+    case ATTN_ERR_MISALIGNED: return "pointer not 16-byte aligned";
+    case ATTN_ERR_CUDA: return "CUDA error";
+    case ATTN_ERR_DEVICE_TIMEOUT: return "device wait timed out";
+    case ATTN_ERR_WORKSPACE: return "workspace missing or too small";
+    default: return "unknown status";
+  }
+}
+
+extern "C" int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                        int Hq, int Hkv, int Nq, int Nk, int d, float scale, int mask_kind,
+                        int window, float softcap, const int* doc_offsets, int num_docs,
+                        cudaStream_t stream) {
+  if (B < 0 || Hq < 0 || Hkv < 0 || Nq < 0 || Nk < 0) return ATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (Hkv == 0 && Hq > 0) return ATTN_ERR_INVALID_ARG;
+  if (Hkv > 0 && Hq % Hkv != 0) return ATTN_ERR_UNSUPPORTED;
+  int st = check_mask(mask_kind, window, doc_offsets, num_docs, Nq, Nk);
+  if (st != ATTN_OK) return st;
+  if (std::isnan(scale) || std::isnan(softcap)) return ATTN_ERR_INVALID_ARG;
+  if (B == 0 || Hq == 0 || Nq == 0) return ATTN_OK;
+  if (o == nullptr || lse == nullptr || q == nullptr) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(o) || !aligned16(lse) || !aligned16(q)) return ATTN_ERR_MISALIGNED;
+  const long long rows = (long long)B * Hq * Nq;
+  if (Nk == 0) return launch_fill_empty(o, lse, (size_t)rows, d, stream) == 0 ? ATTN_OK : ATTN_ERR_CUDA;
+  if (k == nullptr || v == nullptr) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(k) || !aligned16(v)) return ATTN_ERR_MISALIGNED;
+  if ((long long)B * Hq > (1LL << 31) - 1) return ATTN_ERR_UNSUPPORTED;
+
+  if (scale <= 0.f) scale = 1.0f / std::sqrt((float)d);
+  FwdParams p;
+  p.o = o;
+  p.lse = lse;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.Nq = Nq;
+  p.Nk = Nk;
+  p.G = Hq / Hkv;
+  p.num_pairs = (Nq + 255) / 256;
+  p.kscale = scale * kLog2e;
+  p.softcap = softcap > 0.f ? softcap : 0.f;
+  p.cap_scale = softcap > 0.f ? scale / softcap : 0.f;
+  p.cap_log2 = softcap > 0.f ? softcap * kLog2e : 0.f;
+  p.mask = mask_params(mask_kind, window, doc_offsets, num_docs, Nq, Nk);
+  if ((long long)p.num_pairs * B * Hq > (1LL << 31) - 1) return ATTN_ERR_UNSUPPORTED;
+
+  CUtensorMap tq, tk, tv;
+  if (!make_map_3d(&tq, q, d, Nq, (long long)B * Hq, 128) ||
+      !make_map_3d(&tk, k, d, Nk, (long long)B * Hkv, 128) ||
+      !make_map_3d(&tv, v, d, Nk, (long long)B * Hkv, 128))
+    return ATTN_ERR_CUDA;
+  return launch_attn_fwd(tq, tk, tv, p, d, stream) == 0 ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+extern "C" int attn_blockmap(int B, int Nq, int Nk, int mask_kind, int window,
+                             const int* doc_offsets, int num_docs, unsigned char* map,
+                             cudaStream_t stream) {
+  if (B < 0 || Nq < 0 || Nk < 0) return ATTN_ERR_INVALID_ARG;
+  int st = check_mask(mask_kind, window, doc_offsets, num_docs, Nq, Nk);
+  if (st != ATTN_OK) return st;
+  if (B == 0 || Nq == 0 || Nk == 0) return ATTN_OK;
+  if (map == nullptr) return ATTN_ERR_INVALID_ARG;
+  MaskParams m = mask_params(mask_kind, window, doc_offsets, num_docs, Nq, Nk);
+  return launch_blockmap(m, B, Nq, Nk, map, stream) == 0 ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+extern "C" size_t attn_decode_workspace_bytes(int B, int Hq, int d, int num_splits) {
+  if (B <= 0 || Hq <= 0 || d <= 0 || num_splits <= 0) return 0;
+  const size_t rows = (size_t)B * Hq * num_splits;
+  const size_t o_bytes = (rows * d * 4 + 255) & ~(size_t)255;
+  return o_bytes + rows * 4;
+}
+
+extern "C" int attn_decode_default_splits(int B, int Hkv, int T, int device) {
+  // Work items are (batch, kv head, split); a persistent grid of (SMs x resident CTAs)
+  // slots walks them.  Take the smallest split count whose items fill the slots in whole
+  // waves to within 1 %, keeping at least 128 keys per split.
+  if (B <= 0 || Hkv <= 0 || T <= 0) return 1;
+  const long long slots = (long long)sm_count(device) * 2;   // 2 resident CTAs at d=128, G<=8
+  const long long heads = (long long)B * Hkv;
+  const int max_splits = (int)std::max(1LL, std::min<long long>(256, (long long)T / 128));
+  int best = 1;
+  double best_eff = -1.0;
+  for (int s = 1; s <= max_splits; ++s) {
+    const long long items = heads * s;
+    const long long waves = (items + slots - 1) / slots;
+    const double eff = (double)items / (double)(waves * slots);
+    if (eff > best_eff + 1e-9) {
+      best_eff = eff;
+      best = s;
+    }
+    if (eff >= 0.99) break;
+  }
+  return best;
+}
+
+extern "C" int attn_decode_merge(const float* o_part, const float* lse_part, void* o, float* lse,
+                                 long long rows, int num_splits, int d, cudaStream_t stream) {
+  if (rows < 0 || num_splits < 1) return ATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (rows == 0) return ATTN_OK;
+  if (!o_part || !lse_part || !o || !lse) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(o_part) || !aligned16(o) || ((uintptr_t)lse_part & 3u) || ((uintptr_t)lse & 3u))
+    return ATTN_ERR_MISALIGNED;
+  return launch_merge(o_part, lse_part, o, lse, rows, num_splits, d, stream) == 0 ? ATTN_OK
+                                                                                  : ATTN_ERR_CUDA;
+}
+
+extern "C" int attn_decode_splitkv(const void* q, const void* k_cache, const void* v_cache,
+                                   void* o, float* lse, int B, int Hq, int Hkv, int T, int d,
+                                   float scale, int num_splits, void* workspace,
+                                   size_t workspace_bytes, cudaStream_t stream) {
+  if (B < 0 || Hq < 0 || Hkv < 0 || T < 0) return ATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (Hkv == 0 && Hq > 0) return ATTN_ERR_INVALID_ARG;
+  if (Hkv > 0 && Hq % Hkv != 0) return ATTN_ERR_UNSUPPORTED;
+  if (std::isnan(scale)) return ATTN_ERR_INVALID_ARG;
+  if (B == 0 || Hq == 0) return ATTN_OK;
+  const int G = Hq / Hkv;
+  if (G > 16) return ATTN_ERR_UNSUPPORTED;
+  if (!q || !o || !lse) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(o) || !aligned16(lse)) return ATTN_ERR_MISALIGNED;
+  if (T == 0) return launch_fill_empty(o, lse, (size_t)B * Hq, d, stream) == 0 ? ATTN_OK : ATTN_ERR_CUDA;
+  if (!k_cache || !v_cache) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(k_cache) || !aligned16(v_cache)) return ATTN_ERR_MISALIGNED;
+  const int dev = current_device();
+  if (num_splits <= 0) num_splits = attn_decode_default_splits(B, Hkv, T, dev);
+  if (num_splits > T) num_splits = T;
+  const size_t need = attn_decode_workspace_bytes(B, Hq, d, num_splits);
+  if (workspace == nullptr || workspace_bytes < need) return ATTN_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return ATTN_ERR_MISALIGNED;
+  if (scale <= 0.f) scale = 1.0f / std::sqrt((float)d);
+
+  DecParams p;
+  p.q = q;
+  p.o_part = reinterpret_cast<float*>(workspace);
+  const size_t rows = (size_t)B * Hq * num_splits;
+  p.lse_part = reinterpret_cast<float*>(reinterpret_cast<char*>(workspace) +
+                                        ((rows * d * 4 + 255) & ~(size_t)255));
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.T = T;
+  p.S = num_splits;
+  p.num_items = B * Hkv * num_splits;
+  p.kscale = scale * kLog2e;
+  if ((long long)B * Hkv * num_splits > (1LL << 31) - 1) return ATTN_ERR_UNSUPPORTED;
+
+  CUtensorMap tk, tv;
+  if (!make_map_3d(&tk, k_cache, d, T, (long long)B * Hkv, 64) ||
+      !make_map_3d(&tv, v_cache, d, T, (long long)B * Hkv, 64))
+    return ATTN_ERR_CUDA;
+  const int slots = sm_count(dev) * decode_ctas_per_sm(d, G);
+  const int grid = (int)std::min<long long>(p.num_items, slots);
+  if (launch_decode_split(tk, tv, p, d, G, grid, stream) != 0) return ATTN_ERR_CUDA;
+  return launch_merge(p.o_part, p.lse_part, o, lse, (long long)B * Hq, num_splits, d, stream) == 0
+             ? ATTN_OK
+             : ATTN_ERR_CUDA;
+}
+
+static int g_last_site = 0;
+
+extern "C" int attn_get_device_status(cudaStream_t stream) {
+  if (cudaStreamSynchronize(stream) != cudaSuccess) return ATTN_ERR_CUDA;
+  uint32_t word = 0, site = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&word, g_error_word, sizeof(word)) != cudaSuccess) return ATTN_ERR_CUDA;
+  if (cudaMemcpyFromSymbol(&site, g_error_site, sizeof(site)) != cudaSuccess) return ATTN_ERR_CUDA;
+  if (word == 0) return ATTN_OK;
+  if (cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero)) != cudaSuccess) return ATTN_ERR_CUDA;
+  if (cudaMemcpyToSymbol(g_error_site, &zero, sizeof(zero)) != cudaSuccess) return ATTN_ERR_CUDA;
+  g_last_site = (int)site;
+  return (word & kErrWaitTimeout) ? ATTN_ERR_DEVICE_TIMEOUT : ATTN_ERR_CUDA;
+}
+
+extern "C" int attn_last_error_site(void) { return g_last_site; }

@@ -1,0 +1,46 @@
+// Declarations shared by the kernels' launch wrappers and the C-ABI entry points.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "mask.cuh"
+
+namespace attn {
+
+struct FwdParams {
+  void* o;            // bf16 [B, Hq, Nq, d]
+  float* lse;         // fp32 [B, Hq, Nq]
+  int B, Hq, Hkv, Nq, Nk;
+  int G;              // Hq / Hkv
+  int num_pairs;      // ceil(Nq / 256): CTAs per (b, h)
+  float kscale;       // scale * log2(e)
+  float softcap;      // > 0: soft-cap enabled
+  float cap_scale;    // scale / softcap
+  float cap_log2;     // softcap * log2(e)
+  MaskParams mask;
+};
+
+struct DecParams {
+  const void* q;      // bf16 [B, Hq, 1, d]
+  float* o_part;      // fp32 [B, Hq, S, d]: each split normalised by its own sum
+  float* lse_part;    // fp32 [B, Hq, S]: natural-log LSE of each split (-inf if empty)
+  int B, Hq, Hkv, T, S;
+  int num_items;      // B * Hkv * S
+  float kscale;       // scale * log2(e)
+};
+
+int launch_attn_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                    const FwdParams& p, int d, cudaStream_t stream);
+int launch_fill_empty(void* o, float* lse, size_t rows, int d, cudaStream_t stream);
+int launch_blockmap(const MaskParams& m, int B, int Nq, int Nk, uint8_t* map,
+                    cudaStream_t stream);
+int launch_decode_split(const CUtensorMap& tk, const CUtensorMap& tv, const DecParams& p,
+                        int d, int G, int grid, cudaStream_t stream);
+int decode_ctas_per_sm(int d, int G);
+int launch_merge(const float* o_part, const float* lse_part, void* o, float* lse, long long rows,
+                 int S, int d, cudaStream_t stream);
+
+}  // namespace attn

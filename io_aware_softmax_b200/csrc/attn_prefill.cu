@@ -1,0 +1,451 @@
+// Fused exact attention forward for sm_100a: O = softmax(scale * Q K^T + mask) V and the
+// row log-sum-exp, in one pass; S and P never leave the SM.
+//
+// The algorithm is the tiled online softmax of "FlashAttention 논문 분석: IO-Aware Exact
+// Attention" (sections "Online Softmax와 블록 단위 누적" and "알고리즘 의사코드"): for each
+// K/V tile the running row max m and exp-sum l are updated and the output is rescaled, so
+// each row's softmax is exact even though no tile sees the whole row ("Attention 최적화가
+// 어려운 이유", section "나머지 점수가 바꾸는 확률").  The FlashAttention-2/3 refinements the
+// same page lists -- one final normalisation instead of one per tile, mask math only on
+// tiles that need it, the grid over query blocks, producer/consumer warp specialisation,
+// TMA loads and the GEMM/softmax overlap between two query tiles -- are re-expressed for
+// Blackwell:
+//
+//   * one CTA owns two 128-row query tiles (t = 0, 1) of one (batch, head) and streams the
+//     K/V tiles both need through a 4-stage TMA ring in shared memory (128B-swizzled);
+//   * warp 8 issues tcgen05.mma: S_t = Q_t K_j^T into TMEM columns [128t, 128t+128), then
+//     O_t += P_t V_j with P_t read straight from TMEM columns [128t+64, 128t+128) and O_t
+//     accumulated in TMEM columns [256+128t, ...);
+//   * warp 9 issues the TMA loads (warps 10-11 are spare);
+//   * warps 0-3 and 4-7 are the softmax warpgroups of tile 0 and tile 1: thread r owns row
+//     r of its tile, reads its 128 scores from TMEM, applies scale / soft-cap / mask,
+//     updates (m, l), rescales its O row in TMEM only when the running max has grown by
+//     more than 2^8 (exact: the final division uses the same reference max), and writes
+//     P back to TMEM as bf16;
+//   * the two softmax warpgroups ping-pong: while one computes exponentials, the tensor
+//     core runs the other tile's MMAs.
+// The epilogue divides O by l, rounds to bf16 and writes LSE = (m + log2 l) * ln 2.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "attn_internal.h"
+#include "mask.cuh"
+#include "sm100_ptx.cuh"
+#include "tmem_ldst.cuh"
+
+namespace attn {
+
+namespace {
+
+constexpr int kBM = 128;               // rows per query tile (TMEM lanes)
+constexpr int kBN = 128;               // keys per K/V tile
+constexpr int kThreads = 384;          // 2 softmax warpgroups + {MMA, TMA, 2 spare} warps
+constexpr int kMmaWarp = 8;
+constexpr int kTmaWarp = 9;
+// Registers per thread after the split; the launch gives 168 (65536 / 384, rounded down to
+// a multiple of 8): 2 * 128 * 208 + 128 * 56 = 60416 <= 384 * 168 = 64512.
+constexpr uint32_t kRegsSoftmax = 208;
+constexpr uint32_t kRegsOther = 56;
+constexpr uint32_t kTmemCols = 512;
+constexpr float kRescaleThreshold = 8.0f;   // log2 units: rescale when max grows > 2^8
+constexpr float kLn2 = 0.69314718055994531f;
+
+template <int D>
+struct Cfg {
+  static constexpr int kChunks = D / 64;            // 128-byte swizzle atoms along d
+  static constexpr int kChunkBytes = kBM * 128;     // 128 rows x 128 bytes
+  static constexpr int kTileBytes = kBM * D * 2;    // one Q, K or V tile (bf16)
+  static constexpr int kStages = (D == 128) ? 4 : 8;
+  static constexpr int kQOff = 0;
+  static constexpr int kRingOff = 2 * kTileBytes;
+  static constexpr int kBarOff = kRingOff + kStages * kTileBytes;
+  // barriers: q, full[S], empty[S], s_full[2], p_full[2], o_final[2], mma_done
+  static constexpr int kNumBars = 1 + 2 * kStages + 7;
+  static constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 16 + 1024;
+};
+
+enum : uint32_t {
+  kSiteQ = 1, kSiteEmpty, kSiteFullK, kSiteFullV, kSitePFull, kSiteSFull, kSiteOFinal,
+  kSiteDrain,
+};
+
+template <bool kSoftcap, bool kMasked>
+__device__ __forceinline__ float scores_to_log2(uint32_t (&s)[128], const FwdParams& p, int k0,
+                                                int row_lo, int row_hi) {
+  float mx = -INFINITY;
+#pragma unroll
+  for (int c = 0; c < 128; ++c) {
+    float x = __uint_as_float(s[c]);
+    if (kSoftcap) {
+      x = p.cap_log2 * tanh_via_ex2(x * p.cap_scale);
+    } else {
+      x *= p.kscale;
+    }
+    if (kMasked) {
+      const int kv = k0 + c;
+      if (kv < row_lo || kv > row_hi) x = -INFINITY;
+    }
+    s[c] = __float_as_uint(x);
+    mx = fmaxf(mx, x);
+  }
+  return mx;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
+                      const __grid_constant__ CUtensorMap tmK,
+                      const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
+  using C = Cfg<D>;
+  constexpr int NS = C::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_u32 = smem_u32(smem_raw);
+  const uint32_t base_u32 = (raw_u32 + 1023u) & ~1023u;
+  uint8_t* base = smem_raw + (base_u32 - raw_u32);
+  const uint32_t sQ = base_u32 + C::kQOff;
+  const uint32_t sRing = base_u32 + C::kRingOff;
+  const uint32_t sBar = base_u32 + C::kBarOff;
+  auto bar = [&](int i) -> uint32_t { return sBar + 8u * (uint32_t)i; };
+  const int BAR_Q = 0, BAR_FULL = 1, BAR_EMPTY = 1 + NS, BAR_S = 1 + 2 * NS,
+            BAR_P = 3 + 2 * NS, BAR_O = 5 + 2 * NS, BAR_DONE = 7 + 2 * NS;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + C::kBarOff + C::kNumBars * 8);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // ---- work unit: query rows [q_first, q_first + 256) of (b, h); heaviest pairs first
+  const int bh_count = p.B * p.Hq;
+  const int pair = p.num_pairs - 1 - (int)(blockIdx.x / bh_count);
+  const int bh = (int)(blockIdx.x % bh_count);
+  const int b = bh / p.Hq;
+  const int h = bh % p.Hq;
+  const int hk = h / p.G;
+  const int q_first = pair * 2 * kBM;
+  const int q_last = min(q_first + 2 * kBM - 1, p.Nq - 1);
+  int lo_a, hi_a, lo_b, hi_b;
+  row_interval(p.mask, q_first, lo_a, hi_a);
+  row_interval(p.mask, q_last, lo_b, hi_b);
+  int jt0 = 0, n_tiles = 0;
+  if (hi_b >= lo_a && p.Nk > 0) {
+    jt0 = lo_a / kBN;
+    n_tiles = hi_b / kBN - jt0 + 1;
+  }
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(BAR_Q), 1);
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(bar(BAR_FULL + s), 1);
+      mbar_init(bar(BAR_EMPTY + s), 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(bar(BAR_S + t), 1);
+      mbar_init(bar(BAR_P + t), 4);
+      mbar_init(bar(BAR_O + t), 1);
+    }
+    mbar_init(bar(BAR_DONE), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp >= kMmaWarp) {
+   regs_decrease<kRegsOther>();
+   if (warp == kTmaWarp) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      const int zq = b * p.Hq + h;
+      const int zkv = b * p.Hkv + hk;
+      mbar_arrive_expect_tx(bar(BAR_Q), 2 * C::kTileBytes);
+#pragma unroll
+      for (int t = 0; t < 2; ++t)
+#pragma unroll
+        for (int c = 0; c < C::kChunks; ++c)
+          tma_load_3d(sQ + t * C::kTileBytes + c * C::kChunkBytes, &tmQ, bar(BAR_Q), c * 64,
+                      q_first + t * kBM, zq);
+      int issued = 0;
+      for (int i = 0; i < 2 * n_tiles; ++i) {
+        const int s = i % NS;
+        const int round = i / NS;
+        if (round > 0 && !mbar_wait(bar(BAR_EMPTY + s), (round - 1) & 1, abort_flag, kSiteEmpty))
+          break;
+        mbar_arrive_expect_tx(bar(BAR_FULL + s), C::kTileBytes);
+        const int row = (jt0 + (i >> 1)) * kBN;
+        const CUtensorMap* m = (i & 1) ? &tmV : &tmK;
+#pragma unroll
+        for (int c = 0; c < C::kChunks; ++c)
+          tma_load_3d(sRing + s * C::kTileBytes + c * C::kChunkBytes, m, bar(BAR_FULL + s),
+                      c * 64, row, zkv);
+        issued = i + 1;
+      }
+      // Outstanding copies must land before the CTA may exit (matters only on abort).
+      mbar_wait(bar(BAR_Q), 0, nullptr, kSiteDrain);
+      for (int s = 0; s < NS && s < issued; ++s) {
+        const int last = s + ((issued - 1 - s) / NS) * NS;
+        mbar_wait(bar(BAR_FULL + s), (last / NS) & 1, nullptr, kSiteDrain);
+      }
+    }
+    __syncwarp();
+   } else if (warp == kMmaWarp) {
+    // -------------------------------------------------------------- tcgen05 issuer
+    if (lane == 0 && n_tiles > 0) {
+      constexpr uint32_t idesc_qk = idesc_bf16_f32(kBM, kBN, false);
+      constexpr uint32_t idesc_pv = idesc_bf16_f32(kBM, D, true);
+      auto issue_qk = [&](int t, int sk) {
+        const uint32_t d_tmem = tmem + 128u * t;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * C::kChunkBytes + (kk & 3) * 32;
+          const uint64_t a = smem_desc(sQ + t * C::kTileBytes + off, 16, 1024);
+          const uint64_t bd = smem_desc(sRing + sk * C::kTileBytes + off, 16, 1024);
+          umma_ss(d_tmem, a, bd, idesc_qk, kk > 0 ? 1u : 0u);
+        }
+      };
+      auto issue_pv = [&](int t, int sv, bool first) {
+        const uint32_t d_tmem = tmem + 256u + 128u * t;
+        const uint32_t a_tmem = tmem + 128u * t + 64u;
+#pragma unroll
+        for (int kk = 0; kk < kBN / 16; ++kk) {
+          const uint64_t bd = smem_desc(sRing + sv * C::kTileBytes + kk * 16 * 128,
+                                        C::kChunkBytes, 1024);
+          umma_ts(d_tmem, a_tmem + 8u * kk, bd, idesc_pv, (!first || kk > 0) ? 1u : 0u);
+        }
+      };
+      bool ok = mbar_wait(bar(BAR_Q), 0, abort_flag, kSiteQ);
+      tc_fence_after();
+      for (int j = 0; ok && j < n_tiles; ++j) {
+        const int ik = 2 * j;
+        const int sk = ik % NS;
+        ok = mbar_wait(bar(BAR_FULL + sk), (ik / NS) & 1, abort_flag, kSiteFullK);
+        if (!ok) break;
+        tc_fence_after();
+        int sv = 0;
+        if (j > 0) {
+          const int iv = 2 * (j - 1) + 1;
+          sv = iv % NS;
+          ok = mbar_wait(bar(BAR_FULL + sv), (iv / NS) & 1, abort_flag, kSiteFullV);
+          if (!ok) break;
+          tc_fence_after();
+        }
+        for (int t = 0; t < 2; ++t) {
+          if (j > 0) {
+            ok = mbar_wait(bar(BAR_P + t), (j - 1) & 1, abort_flag, kSitePFull);
+            if (!ok) break;
+            tc_fence_after();
+            issue_pv(t, sv, j == 1);
+          }
+          // In-order tensor pipe: this overwrites S_t (and P_t inside it) only after the
+          // PV MMA just issued has read P_t.
+          issue_qk(t, sk);
+          umma_commit(bar(BAR_S + t));
+        }
+        if (!ok) break;
+        if (j > 0) umma_commit(bar(BAR_EMPTY + sv));
+        umma_commit(bar(BAR_EMPTY + sk));
+      }
+      if (ok) {
+        const int iv = 2 * (n_tiles - 1) + 1;
+        const int sv = iv % NS;
+        ok = mbar_wait(bar(BAR_FULL + sv), (iv / NS) & 1, abort_flag, kSiteFullV);
+        if (ok) {
+          tc_fence_after();
+          for (int t = 0; t < 2; ++t) {
+            ok = mbar_wait(bar(BAR_P + t), (n_tiles - 1) & 1, abort_flag, kSitePFull);
+            if (!ok) break;
+            tc_fence_after();
+            issue_pv(t, sv, n_tiles == 1);
+            umma_commit(bar(BAR_O + t));
+          }
+        }
+        umma_commit(bar(BAR_EMPTY + sv));
+      }
+      // Every MMA issued above must be complete before TMEM is released.
+      umma_commit(bar(BAR_DONE));
+      mbar_wait(bar(BAR_DONE), 0, nullptr, kSiteDrain);
+    }
+    __syncwarp();
+   }
+  } else {
+    regs_increase<kRegsSoftmax>();
+    // ------------------------------------------------------------ softmax warpgroups
+    const int t = warp >> 2;                 // query tile of this warpgroup
+    const int wq = warp & 3;                 // TMEM lane quarter this warp may access
+    const int r = wq * 32 + lane;            // row inside the tile
+    const int tq0 = q_first + t * kBM;
+    const int row = tq0 + r;
+    const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+    const uint32_t tS = tmem + lane_off + 128u * t;
+    const uint32_t tP = tS + 64u;
+    const uint32_t tO = tmem + lane_off + 256u + 128u * t;
+
+    int row_lo, row_hi;
+    row_interval(p.mask, row, row_lo, row_hi);
+    // Tile-level bounds: a K/V tile needs no mask when every valid row of this query tile
+    // sees every key of it.  A query tile entirely past Nq is never stored.
+    const bool rows_live = tq0 < p.Nq;
+    int lo_last = 0, hi_first = 0;
+    if (rows_live) {
+      int a0, a1;
+      row_interval(p.mask, min(tq0 + kBM, p.Nq) - 1, lo_last, a0);
+      row_interval(p.mask, tq0, a1, hi_first);
+    }
+
+    float m_ref = -INFINITY;   // reference max (log2 units) of the exponentials in O and l
+    float l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < n_tiles; ++j) {
+      ok = mbar_wait(bar(BAR_S + t), j & 1, abort_flag, kSiteSFull);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t s[128];
+      tmem_ld_x128(tS, s);
+      const int k0 = (jt0 + j) * kBN;
+      const bool masked =
+          rows_live && !(lo_last <= k0 && k0 + kBN - 1 <= hi_first && k0 + kBN <= p.Nk);
+      float mx;
+      if (p.softcap > 0.f) {
+        mx = masked ? scores_to_log2<true, true>(s, p, k0, row_lo, row_hi)
+                    : scores_to_log2<true, false>(s, p, k0, row_lo, row_hi);
+      } else {
+        mx = masked ? scores_to_log2<false, true>(s, p, k0, row_lo, row_hi)
+                    : scores_to_log2<false, false>(s, p, k0, row_lo, row_hi);
+      }
+      const float m_new = fmaxf(m_ref, mx);
+      const bool need = m_new > m_ref + kRescaleThreshold;
+      float alpha = 1.f;
+      if (need) {
+        alpha = ex2_approx(m_ref - m_new);
+        m_ref = m_new;
+      }
+      // P = 2^(x - m_ref) as bf16 pairs, written over the upper half of S in TMEM; each
+      // 32-column half is stored as soon as it is packed so the score registers die early.
+      const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
+      float sum = 0.f;
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          const float a = ex2_approx(__uint_as_float(s[64 * half + 2 * c]) - m_use);
+          const float bb = ex2_approx(__uint_as_float(s[64 * half + 2 * c + 1]) - m_use);
+          sum += a + bb;
+          pk[c] = pack_bf16x2(a, bb);
+        }
+        tmem_st_x32(tP + 32u * half, pk);
+      }
+      l = l * alpha + sum;
+      if (j > 0 && __any_sync(0xffffffffu, need)) {
+        // Rescale this row of O.  PV of tile j-1 is complete: the commit that signalled S_j
+        // was issued after it.  PV of tile j is issued only after the arrive below.
+#pragma unroll
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint32_t o[32];
+          tmem_ld_x32(tO + 32u * cc, o);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          tmem_st_x32(tO + 32u * cc, o);
+        }
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(BAR_P + t));
+    }
+
+    if (ok && n_tiles > 0) {
+      ok = mbar_wait(bar(BAR_O + t), 0, abort_flag, kSiteOFinal);
+      ok = __all_sync(0xffffffffu, ok);
+    }
+    if (ok) {
+      tc_fence_after();
+      const bool valid = row < p.Nq;
+      const float inv_l = (l > 0.f) ? 1.0f / l : 0.f;
+      const float lse = (l > 0.f) ? (m_ref + log2f(l)) * kLn2 : -INFINITY;
+      const size_t row_index = (size_t)(b * p.Hq + h) * (size_t)p.Nq + (size_t)row;
+      __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.o) + row_index * D;
+#pragma unroll
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t o[32];
+        if (n_tiles > 0) {
+          tmem_ld_x32(tO + 32u * cc, o);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = 0u;
+        }
+        uint32_t w[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          w[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv_l,
+                             __uint_as_float(o[2 * i + 1]) * inv_l);
+        if (valid) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + 32 * cc);
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+        }
+      }
+      if (valid) p.lse[row_index] = lse;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// Rows with no key at all (Nk == 0): O = 0 and LSE = -inf, the degenerate case of the
+// definition (empty softmax).
+__global__ void attn_fill_empty_kernel(__nv_bfloat16* o, float* lse, size_t rows, int D) {
+  const size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x;
+  if (i < rows * (size_t)D) o[i] = __float2bfloat16(0.f);
+  if (i < rows) lse[i] = -INFINITY;
+}
+
+template <int D>
+int launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+               const FwdParams& p, cudaStream_t stream) {
+  using C = Cfg<D>;
+  static_assert(C::kSmemBytes <= 227 * 1024, "shared memory budget");
+  cudaError_t e = cudaFuncSetAttribute(attn_fwd_sm100_kernel<D>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       C::kSmemBytes);
+  if (e != cudaSuccess) return -4;
+  const long long grid = (long long)p.num_pairs * p.B * p.Hq;
+  attn_fwd_sm100_kernel<D><<<(unsigned)grid, kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, p);
+  return cudaGetLastError() == cudaSuccess ? 0 : -4;
+}
+
+}  // namespace
+
+int launch_attn_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                    const FwdParams& p, int d, cudaStream_t stream) {
+  if (d == 128) return launch_fwd<128>(tq, tk, tv, p, stream);
+  if (d == 64) return launch_fwd<64>(tq, tk, tv, p, stream);
+  return -2;
+}
+
+int launch_fill_empty(void* o, float* lse, size_t rows, int d, cudaStream_t stream) {
+  const size_t n = rows * (size_t)d;
+  const unsigned blocks = (unsigned)((n + 255) / 256);
+  if (blocks == 0) return 0;
+  attn_fill_empty_kernel<<<blocks, 256, 0, stream>>>(reinterpret_cast<__nv_bfloat16*>(o), lse,
+                                                     rows, d);
+  return cudaGetLastError() == cudaSuccess ? 0 : -4;
+}
+
+}  // namespace attn

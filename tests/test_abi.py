@@ -1,0 +1,121 @@
+"""The C-ABI library builds for sm_100a, loads, and exports every symbol include/attn.h
+declares.  Only calls that return before any CUDA work run here (no GPU on this host)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from io_aware_softmax_b200 import _lib, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "attn.h")
+
+
+def header_symbols():
+    text = open(HEADER, encoding="utf-8").read()
+    return re.findall(r"ATTN_API\s+[A-Za-z_][\w\s\*]*?\b(attn_\w+)\s*\(", text)
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return _lib.load()
+
+
+def test_header_declares_the_entry_points():
+    syms = header_symbols()
+    for name in ["attn_fwd", "attn_blockmap", "attn_decode_splitkv", "attn_decode_merge",
+                 "attn_decode_workspace_bytes", "attn_decode_default_splits",
+                 "attn_get_device_status", "attn_status_string"]:
+        assert name in syms
+    assert set(syms) == set(_lib.SIGNATURES), "binding and header disagree"
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in header_symbols():
+        assert hasattr(lib, name), name
+    # exported with C linkage, nothing else leaks from the internal namespace
+    out = os.popen(f"nm -D --defined-only {_lib.LIB_PATH}").read()
+    exported = {ln.split()[-1] for ln in out.splitlines() if " T " in ln}
+    assert set(header_symbols()) <= exported
+    assert not [s for s in exported if s.startswith("_ZN4attn")]
+
+
+def test_built_for_sm100a_only():
+    log = open(os.path.join(os.path.dirname(_lib.LIB_PATH), "ptxas_info.txt")).read()
+    assert "for 'sm_100a'" in log
+    assert re.search(r"for 'sm_(?!100a)", log) is None
+    regs = build.check_register_budget(log)
+    assert regs and all(r * build.PREFILL_THREADS >= build.PREFILL_SPLIT_REGS for r in regs.values())
+
+
+def test_no_spills_in_any_kernel():
+    log = open(os.path.join(os.path.dirname(_lib.LIB_PATH), "ptxas_info.txt")).read()
+    spills = [int(x) for x in re.findall(r"(\d+) bytes spill stores", log)]
+    assert spills and max(spills) == 0
+
+
+def test_status_strings_and_version(lib):
+    assert lib.attn_status_string(0) == b"ok"
+    assert lib.attn_status_string(-2) == b"unsupported configuration"
+    assert lib.attn_status_string(12345) == b"unknown status"
+    assert lib.attn_version() >= 100
+
+
+def test_validation_happens_before_any_launch(lib):
+    f = lib.attn_fwd
+    P = ctypes.c_void_p(16)       # never dereferenced: every call below fails validation first
+    # head dim outside {64, 128}
+    assert f(P, P, P, P, P, 1, 2, 2, 8, 8, 96, 0.0, 0, 0, 0.0, None, 0, None) == -2
+    # Hq not a multiple of Hkv
+    assert f(P, P, P, P, P, 1, 3, 2, 8, 8, 64, 0.0, 0, 0, 0.0, None, 0, None) == -2
+    # a mask needs Nq == Nk
+    assert f(P, P, P, P, P, 1, 2, 2, 8, 9, 64, 0.0, 1, 0, 0.0, None, 0, None) == -2
+    # unknown mask kind, negative window, document mask without offsets
+    assert f(P, P, P, P, P, 1, 2, 2, 8, 8, 64, 0.0, 7, 0, 0.0, None, 0, None) == -1
+    assert f(P, P, P, P, P, 1, 2, 2, 8, 8, 64, 0.0, 2, -1, 0.0, None, 0, None) == -1
+    assert f(P, P, P, P, P, 1, 2, 2, 8, 8, 64, 0.0, 3, 0, 0.0, None, 0, None) == -1
+    # negative sizes
+    assert f(P, P, P, P, P, -1, 2, 2, 8, 8, 64, 0.0, 0, 0, 0.0, None, 0, None) == -1
+    # misaligned pointer
+    Q = ctypes.c_void_p(24)
+    assert f(Q, P, P, P, P, 1, 2, 2, 8, 8, 64, 0.0, 0, 0, 0.0, None, 0, None) == -3
+    # empty problems are a no-op success
+    assert f(None, None, None, None, None, 0, 2, 2, 8, 8, 64, 0.0, 0, 0, 0.0, None, 0, None) == 0
+    assert f(None, None, None, None, None, 1, 2, 2, 0, 0, 64, 0.0, 1, 0, 0.0, None, 0, None) == 0
+
+
+def test_decode_validation_and_workspace(lib):
+    d = lib.attn_decode_splitkv
+    P = ctypes.c_void_p(16)
+    assert d(P, P, P, P, P, 1, 64, 2, 8, 128, 0.0, 1, P, 1 << 20, None) == -2      # G = 32
+    assert d(P, P, P, P, P, 1, 4, 2, 8, 80, 0.0, 1, P, 1 << 20, None) == -2        # d = 80
+    assert d(P, P, P, P, P, 1, 4, 2, 8, 128, 0.0, 2, None, 0, None) == -6          # no workspace
+    assert d(P, P, P, P, P, 1, 4, 2, 8, 128, 0.0, 2, P, 10, None) == -6            # too small
+    need = lib.attn_decode_workspace_bytes(64, 32, 128, 15)
+    rows = 64 * 32 * 15
+    assert need == ((rows * 128 * 4 + 255) // 256) * 256 + rows * 4
+    assert lib.attn_decode_workspace_bytes(0, 32, 128, 15) == 0
+    m = lib.attn_decode_merge
+    assert m(P, P, P, P, 4, 3, 96, None) == -2
+    assert m(P, P, P, P, 4, 0, 128, None) == -1
+    assert m(None, None, None, None, 0, 3, 128, None) == 0
+
+
+def test_blockmap_validation(lib):
+    b = lib.attn_blockmap
+    assert b(1, 8, 9, 1, 0, None, 0, ctypes.c_void_p(16), None) == -2
+    assert b(1, 8, 8, 3, 0, None, 0, ctypes.c_void_p(16), None) == -1
+    assert b(0, 8, 8, 1, 0, None, 0, None, None) == 0
+
+
+def test_default_split_heuristic(lib):
+    # 512 KV heads on 148 SMs x 2 resident CTAs: 15 splits fill 26 waves to 99.8 %
+    s = lib.attn_decode_default_splits(64, 8, 32768, 0)
+    items = 64 * 8 * s
+    slots = 148 * 2
+    waves = -(-items // slots)
+    assert items / (waves * slots) >= 0.99 and 32768 // s >= 128
+    assert lib.attn_decode_default_splits(1, 1, 100, 0) == 1
+    assert lib.attn_decode_default_splits(1, 1, 0, 0) == 1

@@ -1,0 +1,159 @@
+"""Parity of the fused prefill kernel (attn_fwd through the C ABI) with the fp64 oracle."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+from io_aware_softmax_b200 import attn_fwd, device_status
+from tests.gpu_common import compare, f64, sample_rows
+
+pytestmark = pytest.mark.gpu
+
+MASK_ID = {"none": 0, "causal": 1, "sliding_causal": 2, "document_causal": 3}
+
+
+def _inputs(B, Hq, Hkv, Nq, Nk, d, seed, std=1.0):
+    q = workloads.randn_bf16((B, Hq, Nq, d), seed, 0, std).cuda()
+    k = workloads.randn_bf16((B, Hkv, Nk, d), seed, 1, std).cuda()
+    v = workloads.randn_bf16((B, Hkv, Nk, d), seed, 2, std).cuda()
+    return q, k, v
+
+
+def _run_full(B, Hq, Hkv, Nq, Nk, d, mask="none", window=0, softcap=0.0, docs=None, seed=0,
+              std=1.0, scale=None):
+    q, k, v = _inputs(B, Hq, Hkv, Nq, Nk, d, seed, std)
+    doc_t = None if docs is None else torch.tensor(docs, dtype=torch.int32, device="cuda")
+    # guard bands around the outputs catch writes past the last row
+    o_buf = torch.full((B * Hq * Nq * d + 4096,), float("nan"), dtype=torch.bfloat16, device="cuda")
+    l_buf = torch.full((B * Hq * Nq + 1024,), float("nan"), dtype=torch.float32, device="cuda")
+    o = o_buf[: B * Hq * Nq * d].view(B, Hq, Nq, d)
+    lse = l_buf[: B * Hq * Nq].view(B, Hq, Nq)
+    attn_fwd(q, k, v, scale=scale, mask=mask, window=window, softcap=softcap, doc_offsets=doc_t,
+             out=o, lse=lse)
+    assert device_status() == 0
+    assert torch.isnan(o_buf[B * Hq * Nq * d:]).all() and torch.isnan(l_buf[B * Hq * Nq:]).all()
+    O_ref, L_ref = oracle.attention(f64(q), f64(k), f64(v), scale=scale, mask_kind=MASK_ID[mask],
+                                    window=window, softcap=softcap, doc_offsets=docs)
+    return compare(o, lse, O_ref, L_ref, f"{B}x{Hq}/{Hkv}x{Nq}x{Nk}x{d} {mask} w{window} c{softcap}")
+
+
+def test_tiny_workload_noncausal_and_causal():
+    w = workloads.TINY
+    for mask in ("none", "causal"):
+        q, k, v = workloads.make_inputs(w)
+        q, k, v = q.cuda(), k.cuda(), v.cuda()
+        o, lse = attn_fwd(q, k, v, scale=w.scale, mask=mask)
+        assert device_status() == 0
+        assert o.shape == (1, 2, 128, 64) and lse.shape == (1, 2, 128)
+        O_ref, L_ref = oracle.attention(f64(q), f64(k), f64(v), scale=w.scale,
+                                        mask_kind=MASK_ID[mask])
+        compare(o, lse, O_ref, L_ref, f"tiny {mask}")
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("N", [1, 5, 127, 128, 129, 255, 256, 257, 700])
+@pytest.mark.parametrize("mask", ["none", "causal"])
+def test_ragged_lengths(d, N, mask):
+    _run_full(1, 2, 2, N, N, d, mask=mask, seed=N)
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(4, 1), (8, 2), (6, 3)])
+def test_gqa_mqa_head_mapping(Hq, Hkv):
+    _run_full(2, Hq, Hkv, 300, 300, 128, mask="causal", seed=Hq * 10 + Hkv)
+
+
+@pytest.mark.parametrize("window", [0, 1, 100, 127, 128, 129, 255, 600])
+def test_sliding_window(window):
+    _run_full(1, 2, 1, 777, 777, 128, mask="sliding_causal", window=window, seed=window)
+
+
+@pytest.mark.parametrize("docs", [[0, 1000], [0, 1, 2, 3, 1000], [0, 127, 128, 129, 384, 700, 1000],
+                                  [0, 300, 301, 555, 1000]])
+def test_document_mask(docs):
+    _run_full(1, 3, 3, 1000, 1000, 128, mask="document_causal", docs=docs, seed=len(docs))
+
+
+@pytest.mark.parametrize("mask", ["none", "causal", "document_causal"])
+def test_softcap(mask):
+    docs = [0, 200, 513, 800] if mask == "document_causal" else None
+    _run_full(1, 2, 2, 800, 800, 128, mask=mask, softcap=50.0, docs=docs, seed=3, std=2.0)
+    _run_full(1, 2, 2, 300, 300, 64, mask=mask if mask != "document_causal" else "causal",
+              softcap=5.0, seed=4, std=3.0)
+
+
+@pytest.mark.parametrize("Nq,Nk", [(1, 300), (100, 1000), (300, 129), (513, 64)])
+def test_non_square_unmasked(Nq, Nk):
+    _run_full(2, 2, 1, Nq, Nk, 128, seed=Nq + Nk)
+
+
+def test_explicit_scale_and_large_values():
+    _run_full(1, 2, 2, 400, 400, 128, mask="causal", scale=0.3, std=3.0, seed=9)
+
+
+def test_no_keys_gives_zero_and_minus_inf():
+    q, k, v = _inputs(1, 2, 2, 10, 1, 64, 1)
+    o, lse = attn_fwd(q, k[:, :, :0].contiguous(), v[:, :, :0].contiguous())
+    assert device_status() == 0
+    assert torch.all(o == 0) and torch.all(torch.isneginf(lse))
+
+
+def test_empty_batch_is_a_noop():
+    q = torch.empty((0, 2, 8, 64), dtype=torch.bfloat16, device="cuda")
+    o, lse = attn_fwd(q, q, q)
+    assert o.shape == (0, 2, 8, 64)
+
+
+def test_unsupported_raises_instead_of_falling_back():
+    q, k, v = _inputs(1, 2, 2, 8, 8, 64, 2)
+    q96 = torch.zeros((1, 2, 8, 96), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(RuntimeError, match="unsupported"):
+        attn_fwd(q96, q96, q96)
+    with pytest.raises(RuntimeError, match="unsupported"):
+        attn_fwd(q, k[:, :, :4].contiguous(), v[:, :, :4].contiguous(), mask="causal")
+
+
+# ------------------------------------------------------------------ full-size workloads
+
+def _sampled_full_size(w: workloads.Workload, n_heads: int = 3, seed: int = 0):
+    q, k, v = workloads.make_inputs(w, device="cuda")
+    docs = workloads.workload_doc_offsets(w)
+    doc_t = None if docs is None else torch.tensor(docs, dtype=torch.int32, device="cuda")
+    o, lse = attn_fwd(q, k, v, scale=w.scale, mask=w.mask_kind, window=w.window,
+                      softcap=w.softcap, doc_offsets=doc_t)
+    assert device_status() == 0
+    assert torch.isfinite(o).all() and torch.isfinite(lse).all()
+    rng = np.random.default_rng(seed)
+    G = w.Hq // w.Hkv
+    pairs = {(0, 0), (w.B - 1, w.Hq - 1)}
+    while len(pairs) < n_heads + 2:
+        pairs.add((int(rng.integers(w.B)), int(rng.integers(w.Hq))))
+    for b, h in sorted(pairs):
+        rows = sample_rows(w.Nq, rng)
+        K = f64(k[b, h // G])
+        V = f64(v[b, h // G])
+        O_ref, L_ref = oracle.attention_head(f64(q[b, h, rows]), rows, K, V, w.scale,
+                                             w.mask_kind, w.window, w.softcap, docs)
+        compare(o[b, h, rows], lse[b, h, rows], O_ref, L_ref, f"{w.name} b{b} h{h}")
+
+
+def test_causal_mha_full_size_sampled():
+    _sampled_full_size(workloads.CAUSAL_MHA)
+
+
+def test_sliding_gqa_full_size_sampled():
+    _sampled_full_size(workloads.SWA_GQA)
+
+
+def test_document_softcap_full_size_sampled():
+    _sampled_full_size(workloads.DOC_SOFTCAP)
+
+
+def test_repeated_calls_are_deterministic():
+    q, k, v = _inputs(2, 4, 2, 1000, 1000, 128, 11)
+    o1, l1 = attn_fwd(q, k, v, mask="causal")
+    o2, l2 = attn_fwd(q, k, v, mask="causal")
+    assert device_status() == 0
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
