@@ -227,6 +227,8 @@ def run_ours(args, world, rank, local):
     import io_aware_softmax_b200 as attn
 
     peaks, peak_src = load_peaks()
+    if args.only == "decode":
+        return bench_decode(args, world, local, peaks, peak_src)
     w = workloads.CAUSAL_MHA
     dev = torch.device("cuda", torch.cuda.current_device())
     q, k, v = workloads.make_inputs(w, device=dev)
@@ -273,7 +275,7 @@ def run_ours(args, world, rank, local):
 
     if not args.no_e2e:
         out["e2e"] = e2e_prefill(w, args, world, q, k, v)
-    if not args.no_decode:
+    if not args.no_decode and args.only == "all":
         del q, k, v, o, lse
         torch.cuda.empty_cache()
         out["decode"] = bench_decode(args, world, local, peaks, peak_src)
@@ -319,8 +321,12 @@ def e2e_prefill(w, args, world, q, k, v):
 
 def bench_decode(args, world, local, peaks, peak_src):
     import torch
+    import dataclasses
     import io_aware_softmax_b200 as attn
     w = workloads.DECODE
+    if args.decode_batch:
+        w = dataclasses.replace(w, B=args.decode_batch, name=w.name.replace(
+            f"b{w.B}_", f"b{args.decode_batch}_"))
     dev = torch.device("cuda", torch.cuda.current_device())
     q, kc, vc = workloads.make_inputs(w, device=dev)
     S = attn.default_splits(w.B, w.Hkv, w.Nk, dev.index)
@@ -427,6 +433,10 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle time")
+    ap.add_argument("--only", choices=["all", "prefill", "decode"], default="all",
+                    help="run one part only (profiling runs)")
+    ap.add_argument("--decode-batch", type=int, default=None,
+                    help="decode batch size override (smaller caches for ncu captures)")
     args = ap.parse_args(argv)
     args.warmup = max(3, args.warmup)
 

@@ -37,7 +37,9 @@ def _run_full(B, Hq, Hkv, Nq, Nk, d, mask="none", window=0, softcap=0.0, docs=No
     assert torch.isnan(o_buf[B * Hq * Nq * d:]).all() and torch.isnan(l_buf[B * Hq * Nq:]).all()
     O_ref, L_ref = oracle.attention(f64(q), f64(k), f64(v), scale=scale, mask_kind=MASK_ID[mask],
                                     window=window, softcap=softcap, doc_offsets=docs)
-    return compare(o, lse, O_ref, L_ref, f"{B}x{Hq}/{Hkv}x{Nq}x{Nk}x{d} {mask} w{window} c{softcap}")
+    vmax = float(v.abs().max()) if std > 1.0 else None
+    return compare(o, lse, O_ref, L_ref, f"{B}x{Hq}/{Hkv}x{Nq}x{Nk}x{d} {mask} w{window} c{softcap}",
+                   vmax=vmax)
 
 
 def test_tiny_workload_noncausal_and_causal():
