@@ -120,6 +120,26 @@ ATTN_API int attn_decode_splitkv(const void* q, const void* k_cache, const void*
                         cudaStream_t stream);
 
 /*
+ * attn_decode_splitkv_noalloc -- attn_decode_splitkv for callers that cannot allocate
+ * device memory (a plugin inside a host that owns every allocation, code that must not
+ * allocate while a stream is captured, a loop with a fixed memory budget).  This entry point
+ * has no counterpart in the pages; it only moves the workspace into the library.
+ *   Arguments as attn_decode_splitkv without workspace/workspace_bytes: the split partials
+ *   live in a library-owned device array of 32 MiB that every GPU loading the library holds
+ *   until exit.  Requests whose partials exceed it (B * Hq * splits * (d + 1) * 4 bytes plus
+ *   alignment) return ATTN_ERR_WORKSPACE before anything runs.
+ *   All calls on a device share that array and it keeps the last call's contents: calls that
+ *   overlap on the GPU race, so issue them on one stream.  The first call on each device looks
+ *   up the array's device address (with that device current); make that first call before
+ *   any stream capture.  No allocation happens in any call.
+ * Errors: as attn_decode_splitkv.
+ */
+ATTN_API int attn_decode_splitkv_noalloc(const void* q, const void* k_cache, const void* v_cache,
+                                         void* o, float* lse, int B, int Hq, int Hkv, int T,
+                                         int d, float scale, int num_splits,
+                                         cudaStream_t stream);
+
+/*
  * attn_decode_merge -- merge S partial results per row by the rescaling rule ("3.7 어텐션
  * II", 3.7.4): L = max_s LSE_s, w_s = exp(LSE_s - L), O = sum_s w_s O_s / sum_s w_s,
  * LSE = L + ln sum_s w_s.  Partials with LSE = -inf have weight 0.

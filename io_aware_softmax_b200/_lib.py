@@ -28,6 +28,9 @@ SIGNATURES = {
     "attn_decode_splitkv": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int,
                                     c_int, c_int, c_int, c_int, c_float, c_int, c_void_p,
                                     c_size_t, c_void_p]),
+    "attn_decode_splitkv_noalloc": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                            c_int, c_int, c_int, c_int, c_int, c_float, c_int,
+                                            c_void_p]),
     "attn_decode_merge": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_longlong, c_int,
                                   c_int, c_void_p]),
     "attn_get_device_status": (c_int, [c_void_p]),
