@@ -25,11 +25,11 @@ HEADERS = ["attn_internal.h", "mask.cuh", "sm100_ptx.cuh", "tmem_ldst.cuh"]
 ARCH_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 # The prefill kernel splits its launch registers between warpgroups with setmaxnreg
-# (two softmax warpgroups at 208, one at 56, 384 threads).  The split must fit in what the
+# (two softmax warpgroups at 208, one at 80, 384 threads).  The split must fit in what the
 # CTA is launched with, or the increase would wait forever: check the count ptxas chose.
 PREFILL_KERNEL = "attn_fwd_sm100_kernel"
 PREFILL_THREADS = 384
-PREFILL_SPLIT_REGS = 2 * 128 * 208 + 128 * 56
+PREFILL_SPLIT_REGS = 2 * 128 * 208 + 128 * 80
 
 
 def check_register_budget(ptxas_log: str) -> dict:
@@ -80,7 +80,7 @@ def up_to_date() -> bool:
 def build(force: bool = False, verbose: bool = False) -> str:
     if not force and up_to_date():
         return LIB_PATH
-    cmd = [nvcc_path(), *ARCH_FLAGS, "-O3", "-lineinfo", "-std=c++17", "-rdc=true", "-shared",
+    cmd = [nvcc_path(), *ARCH_FLAGS, "-O3", "-lineinfo", "-std=c++17", "-shared",
            "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
            "-I", os.path.join(ROOT, "include"), "-Xptxas", "-v", "-o", LIB_PATH + ".tmp"]
     cmd += [os.path.join(CSRC, s) for s in SOURCES]
@@ -88,6 +88,9 @@ def build(force: bool = False, verbose: bool = False) -> str:
     if res.returncode != 0:
         raise RuntimeError("nvcc failed:\n" + " ".join(cmd) + "\n" + res.stdout + res.stderr)
     log = res.stdout + res.stderr
+    if "setmaxnreg' ignored" in log:
+        os.remove(LIB_PATH + ".tmp")
+        raise RuntimeError("ptxas ignored setmaxnreg; the warpgroup register split is lost")
     try:
         check_register_budget(log)
     except RuntimeError:

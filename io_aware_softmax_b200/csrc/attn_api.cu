@@ -15,8 +15,8 @@
 
 namespace attn {
 
-__device__ uint32_t g_error_word = 0;
-__device__ uint32_t g_error_site = 0;
+// The library's device error word: [0] = error bits, [1] = first failing wait site.
+__device__ uint32_t g_error[2] = {0u, 0u};
 
 namespace {
 
@@ -88,6 +88,20 @@ int sm_count(int device) {
   return n;
 }
 
+// Device address of g_error on the current device (looked up once per device).
+uint32_t* error_word_ptr(int device) {
+  static std::mutex mu;
+  static uint32_t* cache[64] = {};
+  if (device < 0 || device >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (cache[device] == nullptr) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_error) != cudaSuccess) return nullptr;
+    cache[device] = reinterpret_cast<uint32_t*>(ptr);
+  }
+  return cache[device];
+}
+
 int current_device() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 0;
@@ -151,6 +165,8 @@ extern "C" int attn_fwd(const void* q, const void* k, const void* v, void* o, fl
   p.cap_log2 = softcap > 0.f ? softcap * kLog2e : 0.f;
   p.mask = mask_params(mask_kind, window, doc_offsets, num_docs, Nq, Nk);
   if ((long long)p.num_pairs * B * Hq > (1LL << 31) - 1) return ATTN_ERR_UNSUPPORTED;
+  p.err = error_word_ptr(current_device());
+  if (p.err == nullptr) return ATTN_ERR_CUDA;
 
   CUtensorMap tq, tk, tv;
   if (!make_map_3d(&tq, q, d, Nq, (long long)B * Hq, 128) ||
@@ -253,6 +269,8 @@ extern "C" int attn_decode_splitkv(const void* q, const void* k_cache, const voi
   p.num_items = B * Hkv * num_splits;
   p.kscale = scale * kLog2e;
   if ((long long)B * Hkv * num_splits > (1LL << 31) - 1) return ATTN_ERR_UNSUPPORTED;
+  p.err = error_word_ptr(dev);
+  if (p.err == nullptr) return ATTN_ERR_CUDA;
 
   CUtensorMap tk, tv;
   if (!make_map_3d(&tk, k_cache, d, T, (long long)B * Hkv, 64) ||
@@ -270,14 +288,13 @@ static int g_last_site = 0;
 
 extern "C" int attn_get_device_status(cudaStream_t stream) {
   if (cudaStreamSynchronize(stream) != cudaSuccess) return ATTN_ERR_CUDA;
-  uint32_t word = 0, site = 0, zero = 0;
-  if (cudaMemcpyFromSymbol(&word, g_error_word, sizeof(word)) != cudaSuccess) return ATTN_ERR_CUDA;
-  if (cudaMemcpyFromSymbol(&site, g_error_site, sizeof(site)) != cudaSuccess) return ATTN_ERR_CUDA;
-  if (word == 0) return ATTN_OK;
-  if (cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero)) != cudaSuccess) return ATTN_ERR_CUDA;
-  if (cudaMemcpyToSymbol(g_error_site, &zero, sizeof(zero)) != cudaSuccess) return ATTN_ERR_CUDA;
-  g_last_site = (int)site;
-  return (word & kErrWaitTimeout) ? ATTN_ERR_DEVICE_TIMEOUT : ATTN_ERR_CUDA;
+  uint32_t word[2] = {0u, 0u};
+  const uint32_t zero[2] = {0u, 0u};
+  if (cudaMemcpyFromSymbol(word, g_error, sizeof(word)) != cudaSuccess) return ATTN_ERR_CUDA;
+  if (word[0] == 0) return ATTN_OK;
+  if (cudaMemcpyToSymbol(g_error, zero, sizeof(zero)) != cudaSuccess) return ATTN_ERR_CUDA;
+  g_last_site = (int)word[1];
+  return (word[0] & kErrWaitTimeout) ? ATTN_ERR_DEVICE_TIMEOUT : ATTN_ERR_CUDA;
 }
 
 extern "C" int attn_last_error_site(void) { return g_last_site; }

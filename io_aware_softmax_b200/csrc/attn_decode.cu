@@ -137,7 +137,7 @@ attn_decode_split_kernel(const __grid_constant__ CUtensorMap tmK,
           const int sidx = gi % NS;
           const int round = gi / NS;
           if (round > 0 &&
-              !mbar_wait(empty_bar(sidx), (round - 1) & 1, abort_flag, kSiteDecEmpty)) {
+              !mbar_wait(empty_bar(sidx), (round - 1) & 1, abort_flag, p.err, kSiteDecEmpty)) {
             ok = false;
             break;
           }
@@ -155,7 +155,7 @@ attn_decode_split_kernel(const __grid_constant__ CUtensorMap tmK,
       // Outstanding copies must land before the CTA may exit.
       for (int s = 0; s < NS && (uint32_t)s < gi; ++s) {
         const uint32_t last = s + ((gi - 1 - s) / NS) * NS;
-        mbar_wait(full_bar(s), (last / NS) & 1, nullptr, kSiteDecDrain);
+        mbar_wait(full_bar(s), (last / NS) & 1, nullptr, p.err, kSiteDecDrain);
       }
     }
     __syncwarp();
@@ -198,7 +198,7 @@ attn_decode_split_kernel(const __grid_constant__ CUtensorMap tmK,
       for (int st = 0; st < n_st; ++st, ++gi) {
         const int sidx = gi % NS;
         if (ok) {
-          ok = mbar_wait(full_bar(sidx), (gi / NS) & 1, abort_flag, kSiteDecFull);
+          ok = mbar_wait(full_bar(sidx), (gi / NS) & 1, abort_flag, p.err, kSiteDecFull);
           ok = __all_sync(0xffffffffu, ok);
         }
         if (!ok) continue;

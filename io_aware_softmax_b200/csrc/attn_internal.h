@@ -21,6 +21,7 @@ struct FwdParams {
   float cap_scale;    // scale / softcap
   float cap_log2;     // softcap * log2(e)
   MaskParams mask;
+  uint32_t* err;      // device error word of the library (bits, first site)
 };
 
 struct DecParams {
@@ -30,6 +31,7 @@ struct DecParams {
   int B, Hq, Hkv, T, S;
   int num_items;      // B * Hkv * S
   float kscale;       // scale * log2(e)
+  uint32_t* err;      // device error word of the library (bits, first site)
 };
 
 int launch_attn_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,

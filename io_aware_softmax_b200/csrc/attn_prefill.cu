@@ -12,13 +12,14 @@
 // Blackwell:
 //
 //   * one CTA owns two 128-row query tiles (t = 0, 1) of one (batch, head) and streams the
-//     K/V tiles both need through a 4-stage TMA ring in shared memory (128B-swizzled);
+//     K/V tiles they need through a TMA ring in shared memory (128B-swizzled); each query
+//     tile only visits the K/V tiles its own rows can see;
 //   * warp 8 issues tcgen05.mma: S_t = Q_t K_j^T into TMEM columns [128t, 128t+128), then
 //     O_t += P_t V_j with P_t read straight from TMEM columns [128t+64, 128t+128) and O_t
 //     accumulated in TMEM columns [256+128t, ...);
 //   * warp 9 issues the TMA loads (warps 10-11 are spare);
 //   * warps 0-3 and 4-7 are the softmax warpgroups of tile 0 and tile 1: thread r owns row
-//     r of its tile, reads its 128 scores from TMEM, applies scale / soft-cap / mask,
+//     r of its tile, reads its 128 scores from TMEM, applies mask / scale / soft-cap,
 //     updates (m, l), rescales its O row in TMEM only when the running max has grown by
 //     more than 2^8 (exact: the final division uses the same reference max), and writes
 //     P back to TMEM as bf16;
@@ -44,12 +45,13 @@ constexpr int kThreads = 384;          // 2 softmax warpgroups + {MMA, TMA, 2 sp
 constexpr int kMmaWarp = 8;
 constexpr int kTmaWarp = 9;
 // Registers per thread after the split; the launch gives 168 (65536 / 384, rounded down to
-// a multiple of 8): 2 * 128 * 208 + 128 * 56 = 60416 <= 384 * 168 = 64512.
+// a multiple of 8): 2 * 128 * 208 + 128 * 80 = 63488 <= 384 * 168 = 64512.
 constexpr uint32_t kRegsSoftmax = 208;
-constexpr uint32_t kRegsOther = 56;
+constexpr uint32_t kRegsOther = 80;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units: rescale when max grows > 2^8
 constexpr float kLn2 = 0.69314718055994531f;
+constexpr uint32_t kNegInfBits = 0xff800000u;
 
 template <int D>
 struct Cfg {
@@ -70,26 +72,86 @@ enum : uint32_t {
   kSiteDrain,
 };
 
-template <bool kSoftcap, bool kMasked>
-__device__ __forceinline__ float scores_to_log2(uint32_t (&s)[128], const FwdParams& p, int k0,
-                                                int row_lo, int row_hi) {
-  float mx = -INFINITY;
+__device__ __forceinline__ float f32(uint32_t u) { return __uint_as_float(u); }
+
+// Row maximum of the raw scores of one tile row.  Masked columns (outside [c_lo, c_hi])
+// are overwritten with -inf first.  The scale is positive and the soft-cap is increasing,
+// so the maximum of the transformed scores is the transform of this maximum.  Four
+// independent chains of 3-input maxima keep the dependency depth at 16.
+template <bool kMasked>
+__device__ __forceinline__ float tile_row_max(uint32_t (&s)[128], int c_lo, int c_hi) {
+  if (kMasked) {
 #pragma unroll
-  for (int c = 0; c < 128; ++c) {
-    float x = __uint_as_float(s[c]);
-    if (kSoftcap) {
-      x = p.cap_log2 * tanh_via_ex2(x * p.cap_scale);
-    } else {
-      x *= p.kscale;
-    }
-    if (kMasked) {
-      const int kv = k0 + c;
-      if (kv < row_lo || kv > row_hi) x = -INFINITY;
-    }
-    s[c] = __float_as_uint(x);
-    mx = fmaxf(mx, x);
+    for (int c = 0; c < 128; ++c)
+      if ((unsigned)(c - c_lo) > (unsigned)(c_hi - c_lo)) s[c] = kNegInfBits;
   }
-  return mx;
+  float m0 = -INFINITY, m1 = -INFINITY, m2 = -INFINITY, m3 = -INFINITY;
+#pragma unroll
+  for (int c = 0; c < 128; c += 8) {
+    m0 = max3f(m0, f32(s[c]), f32(s[c + 1]));
+    m1 = max3f(m1, f32(s[c + 2]), f32(s[c + 3]));
+    m2 = max3f(m2, f32(s[c + 4]), f32(s[c + 5]));
+    m3 = max3f(m3, f32(s[c + 6]), f32(s[c + 7]));
+  }
+  return max3f(m0, m1, fmaxf(m2, m3));
+}
+
+// Scaled (base-2) score of a raw score: s * scale * log2(e), or with the soft-cap
+// c * log2(e) * tanh(s * scale / c).  -inf (masked) stays -inf.
+template <bool kSoftcap>
+__device__ __forceinline__ float scaled_score(float s, const FwdParams& p) {
+  if (!kSoftcap) return s * p.kscale;
+  if (s == -INFINITY) return -INFINITY;
+  return p.cap_log2 * tanh_via_ex2(s * p.cap_scale);
+}
+
+// P = 2^(x - m_use) for one 64-column half of a tile row, packed as bf16 pairs; returns
+// the half's fp32 sum (four independent packed accumulators).
+template <bool kSoftcap>
+__device__ __forceinline__ float tile_row_exp_half(const uint32_t (&s)[128], int base,
+                                                   const FwdParams& p, float m_use,
+                                                   uint32_t (&pk)[32]) {
+  float a0 = 0.f, a1 = 0.f, b0 = 0.f, b1 = 0.f, c0 = 0.f, c1 = 0.f, d0 = 0.f, d1 = 0.f;
+#pragma unroll
+  for (int c = 0; c < 64; c += 2) {
+    float x0, x1;
+    if (!kSoftcap) {
+      ffma2(x0, x1, f32(s[base + c]), f32(s[base + c + 1]), p.kscale, p.kscale, -m_use, -m_use);
+    } else {
+      x0 = scaled_score<true>(f32(s[base + c]), p) - m_use;
+      x1 = scaled_score<true>(f32(s[base + c + 1]), p) - m_use;
+    }
+    const float e0 = ex2_approx(x0);
+    const float e1 = ex2_approx(x1);
+    switch ((c >> 1) & 3) {
+      case 0: add2(a0, a1, e0, e1); break;
+      case 1: add2(b0, b1, e0, e1); break;
+      case 2: add2(c0, c1, e0, e1); break;
+      default: add2(d0, d1, e0, e1); break;
+    }
+    pk[c >> 1] = pack_bf16x2(e0, e1);
+  }
+  return ((a0 + a1) + (b0 + b1)) + ((c0 + c1) + (d0 + d1));
+}
+
+// K/V tiles [a, b] (relative to the CTA's first tile) that query tile t must visit; n = 0
+// when the tile has no valid row.
+struct TileRange {
+  int a, b, n;
+};
+
+__device__ __forceinline__ TileRange tile_range(const FwdParams& p, int tq0, int jt0,
+                                                int n_tiles) {
+  TileRange r{0, -1, 0};
+  if (tq0 >= p.Nq || n_tiles == 0) return r;
+  int lo, hi, lo2, hi2;
+  row_interval(p.mask, tq0, lo, hi);
+  row_interval(p.mask, min(tq0 + kBM, p.Nq) - 1, lo2, hi2);
+  if (hi2 < lo) return r;
+  r.a = lo / kBN - jt0;
+  r.b = hi2 / kBN - jt0;
+  r.n = r.b - r.a + 1;
+  return r;
 }
 
 template <int D>
@@ -115,10 +177,10 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // ---- work unit: query rows [q_first, q_first + 256) of (b, h); heaviest pairs first
-  const int bh_count = p.B * p.Hq;
-  const int pair = p.num_pairs - 1 - (int)(blockIdx.x / bh_count);
-  const int bh = (int)(blockIdx.x % bh_count);
+  // ---- work unit: query rows [q_first, q_first + 256) of (b, h).  CTAs of one head are
+  // adjacent (they share K/V through L2), heaviest query pairs of each head first.
+  const int bh = (int)(blockIdx.x / p.num_pairs);
+  const int pair = p.num_pairs - 1 - (int)(blockIdx.x % p.num_pairs);
   const int b = bh / p.Hq;
   const int h = bh % p.Hq;
   const int hk = h / p.G;
@@ -132,6 +194,8 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
     jt0 = lo_a / kBN;
     n_tiles = hi_b / kBN - jt0 + 1;
   }
+  const TileRange rng0 = tile_range(p, q_first, jt0, n_tiles);
+  const TileRange rng1 = tile_range(p, q_first + kBM, jt0, n_tiles);
 
   if (threadIdx.x == 0) {
     mbar_init(bar(BAR_Q), 1);
@@ -178,7 +242,8 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
       for (int i = 0; i < 2 * n_tiles; ++i) {
         const int s = i % NS;
         const int round = i / NS;
-        if (round > 0 && !mbar_wait(bar(BAR_EMPTY + s), (round - 1) & 1, abort_flag, kSiteEmpty))
+        if (round > 0 &&
+            !mbar_wait(bar(BAR_EMPTY + s), (round - 1) & 1, abort_flag, p.err, kSiteEmpty))
           break;
         mbar_arrive_expect_tx(bar(BAR_FULL + s), C::kTileBytes);
         const int row = (jt0 + (i >> 1)) * kBN;
@@ -190,10 +255,10 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
         issued = i + 1;
       }
       // Outstanding copies must land before the CTA may exit (matters only on abort).
-      mbar_wait(bar(BAR_Q), 0, nullptr, kSiteDrain);
+      mbar_wait(bar(BAR_Q), 0, nullptr, p.err, kSiteDrain);
       for (int s = 0; s < NS && s < issued; ++s) {
         const int last = s + ((issued - 1 - s) / NS) * NS;
-        mbar_wait(bar(BAR_FULL + s), (last / NS) & 1, nullptr, kSiteDrain);
+        mbar_wait(bar(BAR_FULL + s), (last / NS) & 1, nullptr, p.err, kSiteDrain);
       }
     }
     __syncwarp();
@@ -202,53 +267,68 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
     if (lane == 0 && n_tiles > 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(kBM, kBN, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(kBM, D, true);
+      const TileRange rng[2] = {rng0, rng1};
+      // Descriptors differ only in their start-address field (address >> 4, 14 bits; the
+      // CTA's shared memory stays below 2^18 bytes, so adding an offset never carries out
+      // of it): keep three base descriptors and add offsets in 16-byte units.
+      const uint64_t dQ = smem_desc(sQ, 16, 1024);
+      const uint64_t dK = smem_desc(sRing, 16, 1024);
+      const uint64_t dV = smem_desc(sRing, C::kChunkBytes, 1024);
       auto issue_qk = [&](int t, int sk) {
         const uint32_t d_tmem = tmem + 128u * t;
+        const uint32_t q_off = (uint32_t)(t * C::kTileBytes) >> 4;
+        const uint32_t k_off = (uint32_t)(sk * C::kTileBytes) >> 4;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * C::kChunkBytes + (kk & 3) * 32;
-          const uint64_t a = smem_desc(sQ + t * C::kTileBytes + off, 16, 1024);
-          const uint64_t bd = smem_desc(sRing + sk * C::kTileBytes + off, 16, 1024);
-          umma_ss(d_tmem, a, bd, idesc_qk, kk > 0 ? 1u : 0u);
+          const uint32_t off = ((kk >> 2) * C::kChunkBytes + (kk & 3) * 32) >> 4;
+          umma_ss(d_tmem, dQ + q_off + off, dK + k_off + off, idesc_qk, kk > 0 ? 1u : 0u);
         }
       };
       auto issue_pv = [&](int t, int sv, bool first) {
         const uint32_t d_tmem = tmem + 256u + 128u * t;
         const uint32_t a_tmem = tmem + 128u * t + 64u;
+        const uint32_t v_off = (uint32_t)(sv * C::kTileBytes) >> 4;
 #pragma unroll
         for (int kk = 0; kk < kBN / 16; ++kk) {
-          const uint64_t bd = smem_desc(sRing + sv * C::kTileBytes + kk * 16 * 128,
-                                        C::kChunkBytes, 1024);
-          umma_ts(d_tmem, a_tmem + 8u * kk, bd, idesc_pv, (!first || kk > 0) ? 1u : 0u);
+          umma_ts(d_tmem, a_tmem + 8u * kk, dV + v_off + ((kk * 16 * 128) >> 4), idesc_pv,
+                  (!first || kk > 0) ? 1u : 0u);
         }
       };
-      bool ok = mbar_wait(bar(BAR_Q), 0, abort_flag, kSiteQ);
+      // PV of union step jv for query tile t, if t visits it: wait for P, issue, and
+      // signal the epilogue after the tile's last PV.
+      auto pv_for = [&](int t, int jv, int sv) -> bool {
+        if (jv < rng[t].a || jv > rng[t].b) return true;
+        if (!mbar_wait(bar(BAR_P + t), (jv - rng[t].a) & 1, abort_flag, p.err, kSitePFull))
+          return false;
+        tc_fence_after();
+        issue_pv(t, sv, jv == rng[t].a);
+        if (jv == rng[t].b) umma_commit(bar(BAR_O + t));
+        return true;
+      };
+      bool ok = mbar_wait(bar(BAR_Q), 0, abort_flag, p.err, kSiteQ);
       tc_fence_after();
       for (int j = 0; ok && j < n_tiles; ++j) {
         const int ik = 2 * j;
         const int sk = ik % NS;
-        ok = mbar_wait(bar(BAR_FULL + sk), (ik / NS) & 1, abort_flag, kSiteFullK);
+        ok = mbar_wait(bar(BAR_FULL + sk), (ik / NS) & 1, abort_flag, p.err, kSiteFullK);
         if (!ok) break;
         tc_fence_after();
         int sv = 0;
         if (j > 0) {
           const int iv = 2 * (j - 1) + 1;
           sv = iv % NS;
-          ok = mbar_wait(bar(BAR_FULL + sv), (iv / NS) & 1, abort_flag, kSiteFullV);
+          ok = mbar_wait(bar(BAR_FULL + sv), (iv / NS) & 1, abort_flag, p.err, kSiteFullV);
           if (!ok) break;
           tc_fence_after();
         }
-        for (int t = 0; t < 2; ++t) {
-          if (j > 0) {
-            ok = mbar_wait(bar(BAR_P + t), (j - 1) & 1, abort_flag, kSitePFull);
-            if (!ok) break;
-            tc_fence_after();
-            issue_pv(t, sv, j == 1);
+        for (int t = 0; t < 2 && ok; ++t) {
+          if (j > 0) ok = pv_for(t, j - 1, sv);
+          if (ok && j >= rng[t].a && j <= rng[t].b) {
+            // In-order tensor pipe: this overwrites S_t (and P_t inside it) only after
+            // the PV MMA just issued has read P_t.
+            issue_qk(t, sk);
+            umma_commit(bar(BAR_S + t));
           }
-          // In-order tensor pipe: this overwrites S_t (and P_t inside it) only after the
-          // PV MMA just issued has read P_t.
-          issue_qk(t, sk);
-          umma_commit(bar(BAR_S + t));
         }
         if (!ok) break;
         if (j > 0) umma_commit(bar(BAR_EMPTY + sv));
@@ -257,22 +337,16 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
       if (ok) {
         const int iv = 2 * (n_tiles - 1) + 1;
         const int sv = iv % NS;
-        ok = mbar_wait(bar(BAR_FULL + sv), (iv / NS) & 1, abort_flag, kSiteFullV);
+        ok = mbar_wait(bar(BAR_FULL + sv), (iv / NS) & 1, abort_flag, p.err, kSiteFullV);
         if (ok) {
           tc_fence_after();
-          for (int t = 0; t < 2; ++t) {
-            ok = mbar_wait(bar(BAR_P + t), (n_tiles - 1) & 1, abort_flag, kSitePFull);
-            if (!ok) break;
-            tc_fence_after();
-            issue_pv(t, sv, n_tiles == 1);
-            umma_commit(bar(BAR_O + t));
-          }
+          for (int t = 0; t < 2 && ok; ++t) ok = pv_for(t, n_tiles - 1, sv);
         }
         umma_commit(bar(BAR_EMPTY + sv));
       }
       // Every MMA issued above must be complete before TMEM is released.
       umma_commit(bar(BAR_DONE));
-      mbar_wait(bar(BAR_DONE), 0, nullptr, kSiteDrain);
+      mbar_wait(bar(BAR_DONE), 0, nullptr, p.err, kSiteDrain);
     }
     __syncwarp();
    }
@@ -284,6 +358,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
     const int r = wq * 32 + lane;            // row inside the tile
     const int tq0 = q_first + t * kBM;
     const int row = tq0 + r;
+    const TileRange rng = t ? rng1 : rng0;
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
     const uint32_t tS = tmem + lane_off + 128u * t;
     const uint32_t tP = tS + 64u;
@@ -292,10 +367,9 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
     int row_lo, row_hi;
     row_interval(p.mask, row, row_lo, row_hi);
     // Tile-level bounds: a K/V tile needs no mask when every valid row of this query tile
-    // sees every key of it.  A query tile entirely past Nq is never stored.
-    const bool rows_live = tq0 < p.Nq;
+    // sees every key of it and it lies inside Nk.
     int lo_last = 0, hi_first = 0;
-    if (rows_live) {
+    if (rng.n > 0) {
       int a0, a1;
       row_interval(p.mask, min(tq0 + kBM, p.Nq) - 1, lo_last, a0);
       row_interval(p.mask, tq0, a1, hi_first);
@@ -304,24 +378,19 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
     float m_ref = -INFINITY;   // reference max (log2 units) of the exponentials in O and l
     float l = 0.f;
     bool ok = true;
-    for (int j = 0; j < n_tiles; ++j) {
-      ok = mbar_wait(bar(BAR_S + t), j & 1, abort_flag, kSiteSFull);
+    for (int i = 0; i < rng.n; ++i) {
+      ok = mbar_wait(bar(BAR_S + t), i & 1, abort_flag, p.err, kSiteSFull);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
       uint32_t s[128];
       tmem_ld_x128(tS, s);
-      const int k0 = (jt0 + j) * kBN;
-      const bool masked =
-          rows_live && !(lo_last <= k0 && k0 + kBN - 1 <= hi_first && k0 + kBN <= p.Nk);
-      float mx;
-      if (p.softcap > 0.f) {
-        mx = masked ? scores_to_log2<true, true>(s, p, k0, row_lo, row_hi)
-                    : scores_to_log2<true, false>(s, p, k0, row_lo, row_hi);
-      } else {
-        mx = masked ? scores_to_log2<false, true>(s, p, k0, row_lo, row_hi)
-                    : scores_to_log2<false, false>(s, p, k0, row_lo, row_hi);
-      }
+      const int k0 = (jt0 + rng.a + i) * kBN;
+      const bool masked = !(lo_last <= k0 && k0 + kBN - 1 <= hi_first && k0 + kBN <= p.Nk);
+      const float mx_raw = masked ? tile_row_max<true>(s, row_lo - k0, row_hi - k0)
+                                  : tile_row_max<false>(s, 0, 0);
+      const float mx = (p.softcap > 0.f) ? scaled_score<true>(mx_raw, p)
+                                         : scaled_score<false>(mx_raw, p);
       const float m_new = fmaxf(m_ref, mx);
       const bool need = m_new > m_ref + kRescaleThreshold;
       float alpha = 1.f;
@@ -330,31 +399,31 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
         m_ref = m_new;
       }
       // P = 2^(x - m_ref) as bf16 pairs, written over the upper half of S in TMEM; each
-      // 32-column half is stored as soon as it is packed so the score registers die early.
+      // 64-column half is stored as soon as it is packed.  Masked scores are -inf, so
+      // their exponentials are exactly 0.
       const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
       float sum = 0.f;
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
         uint32_t pk[32];
-#pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          const float a = ex2_approx(__uint_as_float(s[64 * half + 2 * c]) - m_use);
-          const float bb = ex2_approx(__uint_as_float(s[64 * half + 2 * c + 1]) - m_use);
-          sum += a + bb;
-          pk[c] = pack_bf16x2(a, bb);
+        if (p.softcap > 0.f) {
+          sum += tile_row_exp_half<true>(s, 64 * half, p, m_use, pk);
+        } else {
+          sum += tile_row_exp_half<false>(s, 64 * half, p, m_use, pk);
         }
         tmem_st_x32(tP + 32u * half, pk);
       }
       l = l * alpha + sum;
-      if (j > 0 && __any_sync(0xffffffffu, need)) {
-        // Rescale this row of O.  PV of tile j-1 is complete: the commit that signalled S_j
-        // was issued after it.  PV of tile j is issued only after the arrive below.
+      if (i > 0 && __any_sync(0xffffffffu, need)) {
+        // Rescale this row of O.  PV of the previous tile is complete: the commit that
+        // signalled this S was issued after it.  The next PV is issued only after the
+        // arrive below.
 #pragma unroll
         for (int cc = 0; cc < D / 32; ++cc) {
           uint32_t o[32];
           tmem_ld_x32(tO + 32u * cc, o);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(f32(o[k]) * alpha);
           tmem_st_x32(tO + 32u * cc, o);
         }
       }
@@ -364,8 +433,8 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
       if (lane == 0) mbar_arrive(bar(BAR_P + t));
     }
 
-    if (ok && n_tiles > 0) {
-      ok = mbar_wait(bar(BAR_O + t), 0, abort_flag, kSiteOFinal);
+    if (ok && rng.n > 0) {
+      ok = mbar_wait(bar(BAR_O + t), 0, abort_flag, p.err, kSiteOFinal);
       ok = __all_sync(0xffffffffu, ok);
     }
     if (ok) {
@@ -378,22 +447,21 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
 #pragma unroll
       for (int cc = 0; cc < D / 32; ++cc) {
         uint32_t o[32];
-        if (n_tiles > 0) {
+        if (rng.n > 0) {
           tmem_ld_x32(tO + 32u * cc, o);
         } else {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = 0u;
+          for (int k = 0; k < 32; ++k) o[k] = 0u;
         }
         uint32_t w[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
-          w[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv_l,
-                             __uint_as_float(o[2 * i + 1]) * inv_l);
+        for (int k = 0; k < 16; ++k)
+          w[k] = pack_bf16x2(f32(o[2 * k]) * inv_l, f32(o[2 * k + 1]) * inv_l);
         if (valid) {
           uint4* dst = reinterpret_cast<uint4*>(orow + 32 * cc);
 #pragma unroll
-          for (int i = 0; i < 4; ++i)
-            dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+          for (int k = 0; k < 4; ++k)
+            dst[k] = make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
         }
       }
       if (valid) p.lse[row_index] = lse;

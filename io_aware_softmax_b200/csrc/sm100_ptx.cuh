@@ -10,16 +10,14 @@
 namespace attn {
 
 // ------------------------------------------------------------------ error reporting
-// Every wait in every kernel is bounded.  A wait that runs out records an error word in
-// device memory, raises the CTA's abort flag and returns false; the kernel then unwinds,
+// Every wait in every kernel is bounded.  A wait that runs out records an error in the
+// library's device error word (err[0] = bits, err[1] = first site; its address is passed to
+// every kernel), raises the CTA's abort flag and returns false; the kernel then unwinds,
 // frees its TMEM and exits.  The host reads the word with attn_get_device_status().
 enum : uint32_t {
   kErrWaitTimeout = 1u << 0,
   kErrBadArgument = 1u << 1,
 };
-
-extern __device__ uint32_t g_error_word;
-extern __device__ uint32_t g_error_site;
 
 constexpr uint64_t kWaitLimitNs = 500ull * 1000ull * 1000ull;   // 0.5 s
 
@@ -29,9 +27,9 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
-__device__ __forceinline__ void report_error(uint32_t bits, uint32_t site) {
-  atomicOr(&g_error_word, bits);
-  atomicCAS(&g_error_site, 0u, site);
+__device__ __forceinline__ void report_error(uint32_t* err, uint32_t bits, uint32_t site) {
+  atomicOr(err, bits);
+  atomicCAS(err + 1, 0u, site);
 }
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -82,7 +80,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // thread of the CTA has already raised *abort.  With abort == nullptr (the drain waits of
 // the teardown) only the time limit ends the wait.
 static __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort,
-                                       uint32_t site) {
+                                                 uint32_t* err, uint32_t site) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
@@ -90,7 +88,7 @@ static __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, 
     if ((it & 63u) == 0) {
       if (abort != nullptr && *abort) return false;
       if (globaltimer_ns() - t0 > kWaitLimitNs) {
-        report_error(kErrWaitTimeout, site);
+        report_error(err, kErrWaitTimeout, site);
         if (abort != nullptr) *abort = 1;
         return false;
       }
@@ -218,6 +216,30 @@ __device__ __forceinline__ float rcp_approx(float x) {
 __device__ __forceinline__ float tanh_via_ex2(float y) {
   const float e = ex2_approx(y * 2.8853900817779268f);   // 2*log2(e)
   return 1.0f - 2.0f * rcp_approx(e + 1.0f);
+}
+
+// 3-input maximum (sm_100).
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// Packed pair arithmetic on sm_100 (two fp32 lanes per instruction).
+__device__ __forceinline__ void ffma2(float& d0, float& d1, float a0, float a1, float b0, float b1,
+                                      float c0, float c1) {
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
+}
+__device__ __forceinline__ void add2(float& a0, float& a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 ra, rb;\n\t"
+      "mov.b64 ra, {%0, %1};\n\tmov.b64 rb, {%2, %3};\n\t"
+      "add.rn.f32x2 ra, ra, rb;\n\tmov.b64 {%0, %1}, ra;\n\t}"
+      : "+f"(a0), "+f"(a1)
+      : "f"(b0), "f"(b1));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
