@@ -159,6 +159,7 @@ extern "C" int attn_fwd(const void* q, const void* k, const void* v, void* o, fl
   p.Nk = Nk;
   p.G = Hq / Hkv;
   p.num_pairs = (Nq + 255) / 256;
+  p.num_sms = sm_count(current_device());
   p.kscale = scale * kLog2e;
   p.softcap = softcap > 0.f ? softcap : 0.f;
   p.cap_scale = softcap > 0.f ? scale / softcap : 0.f;

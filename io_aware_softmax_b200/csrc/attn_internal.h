@@ -15,7 +15,8 @@ struct FwdParams {
   float* lse;         // fp32 [B, Hq, Nq]
   int B, Hq, Hkv, Nq, Nk;
   int G;              // Hq / Hkv
-  int num_pairs;      // ceil(Nq / 256): CTAs per (b, h)
+  int num_pairs;      // ceil(Nq / 256): query pairs per (b, h)
+  int num_sms;        // persistent grid size (SMs of the device)
   float kscale;       // scale * log2(e)
   float softcap;      // > 0: soft-cap enabled
   float cap_scale;    // scale / softcap

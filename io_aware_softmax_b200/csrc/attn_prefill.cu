@@ -11,13 +11,15 @@
 // TMA loads and the GEMM/softmax overlap between two query tiles -- are re-expressed for
 // Blackwell:
 //
-//   * one CTA owns two 128-row query tiles (t = 0, 1) of one (batch, head) and streams the
-//     K/V tiles they need through a TMA ring in shared memory (128B-swizzled); each query
-//     tile only visits the K/V tiles its own rows can see;
+//   * a persistent grid (one CTA per SM) walks query pairs: two 128-row query tiles
+//     (t = 0, 1) of one (batch, head); the K/V tiles they need stream through a TMA ring in
+//     shared memory (128B-swizzled) that never drains between pairs; each query tile only
+//     visits the K/V tiles its own rows can see;
 //   * warp 8 issues tcgen05.mma: S_t = Q_t K_j^T into TMEM columns [128t, 128t+128), then
 //     O_t += P_t V_j with P_t read straight from TMEM columns [128t+64, 128t+128) and O_t
 //     accumulated in TMEM columns [256+128t, ...);
-//   * warp 9 issues the TMA loads (warps 10-11 are spare);
+//   * warp 9 issues the K/V TMA loads, warp 10 reloads each query tile's Q as soon as its
+//     last QK^T of the previous pair is done (warp 11 is spare);
 //   * warps 0-3 and 4-7 are the softmax warpgroups of tile 0 and tile 1: thread r owns row
 //     r of its tile, reads its 128 scores from TMEM, applies mask / scale / soft-cap,
 //     updates (m, l), rescales its O row in TMEM only when the running max has grown by
@@ -41,13 +43,14 @@ namespace {
 
 constexpr int kBM = 128;               // rows per query tile (TMEM lanes)
 constexpr int kBN = 128;               // keys per K/V tile
-constexpr int kThreads = 384;          // 2 softmax warpgroups + {MMA, TMA, 2 spare} warps
+constexpr int kThreads = 384;          // 2 softmax warpgroups + {MMA, K/V TMA, Q TMA, spare}
 constexpr int kMmaWarp = 8;
 constexpr int kTmaWarp = 9;
+constexpr int kQWarp = 10;
 // Registers per thread after the split; the launch gives 168 (65536 / 384, rounded down to
-// a multiple of 8): 2 * 128 * 208 + 128 * 80 = 63488 <= 384 * 168 = 64512.
-constexpr uint32_t kRegsSoftmax = 208;
-constexpr uint32_t kRegsOther = 80;
+// a multiple of 8): 2 * 128 * 200 + 128 * 96 = 63488 <= 384 * 168 = 64512.
+constexpr uint32_t kRegsSoftmax = 200;
+constexpr uint32_t kRegsOther = 96;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units: rescale when max grows > 2^8
 constexpr float kLn2 = 0.69314718055994531f;
@@ -62,14 +65,14 @@ struct Cfg {
   static constexpr int kQOff = 0;
   static constexpr int kRingOff = 2 * kTileBytes;
   static constexpr int kBarOff = kRingOff + kStages * kTileBytes;
-  // barriers: q, full[S], empty[S], s_full[2], p_full[2], o_final[2], mma_done
-  static constexpr int kNumBars = 1 + 2 * kStages + 7;
+  // barriers: q[2], q_free[2], full[S], empty[S], s[2], p[2], o[2], done
+  static constexpr int kNumBars = 11 + 2 * kStages;
   static constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 16 + 1024;
 };
 
 enum : uint32_t {
   kSiteQ = 1, kSiteEmpty, kSiteFullK, kSiteFullV, kSitePFull, kSiteSFull, kSiteOFinal,
-  kSiteDrain,
+  kSiteDrain, kSiteQFree,
 };
 
 __device__ __forceinline__ float f32(uint32_t u) { return __uint_as_float(u); }
@@ -154,6 +157,52 @@ __device__ __forceinline__ TileRange tile_range(const FwdParams& p, int tq0, int
   return r;
 }
 
+// One query pair: rows [q_first, q_first + 256) of (b, h), the K/V tiles the pair visits,
+// [jt0, jt0 + n_tiles), and each query tile's own sub-range of them.
+struct PairWork {
+  int b, h, hk, q_first, jt0, n_tiles;
+  TileRange rng[2];
+};
+
+__device__ __forceinline__ PairWork make_pair_work(const FwdParams& p, int bh, int pair) {
+  PairWork w;
+  w.b = bh / p.Hq;
+  w.h = bh % p.Hq;
+  w.hk = w.h / p.G;
+  w.q_first = pair * 2 * kBM;
+  const int q_last = min(w.q_first + 2 * kBM - 1, p.Nq - 1);
+  int lo_a, hi_a, lo_b, hi_b;
+  row_interval(p.mask, w.q_first, lo_a, hi_a);
+  row_interval(p.mask, q_last, lo_b, hi_b);
+  w.jt0 = 0;
+  w.n_tiles = 0;
+  if (hi_b >= lo_a && p.Nk > 0) {
+    w.jt0 = lo_a / kBN;
+    w.n_tiles = hi_b / kBN - w.jt0 + 1;
+  }
+  w.rng[0] = tile_range(p, w.q_first, w.jt0, w.n_tiles);
+  w.rng[1] = tile_range(p, w.q_first + kBM, w.jt0, w.n_tiles);
+  return w;
+}
+
+// The CTA's sequence of query pairs (the grid is persistent: one CTA per SM).  Unit u of a
+// head combines pair P-1-k with pair k (k = u mod ceil(P/2)): under a causal mask their
+// costs add up to the same total for every k, so handing units to CTAs round-robin
+// balances the work, and consecutive units share a head, so the K/V tiles of the heads in
+// flight stay in L2.  f returns false to stop (abort).
+template <typename F>
+__device__ __forceinline__ void for_each_pair(const FwdParams& p, F&& f) {
+  const int P = p.num_pairs;
+  const int upb = (P + 1) / 2;
+  const long long total = (long long)p.B * p.Hq * upb;
+  for (long long u = blockIdx.x; u < total; u += gridDim.x) {
+    const int bh = (int)(u / upb);
+    const int k = (int)(u % upb);
+    if (!f(bh, P - 1 - k)) return;
+    if (k != P - 1 - k && !f(bh, k)) return;
+  }
+}
+
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
@@ -169,44 +218,27 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
   const uint32_t sRing = base_u32 + C::kRingOff;
   const uint32_t sBar = base_u32 + C::kBarOff;
   auto bar = [&](int i) -> uint32_t { return sBar + 8u * (uint32_t)i; };
-  const int BAR_Q = 0, BAR_FULL = 1, BAR_EMPTY = 1 + NS, BAR_S = 1 + 2 * NS,
-            BAR_P = 3 + 2 * NS, BAR_O = 5 + 2 * NS, BAR_DONE = 7 + 2 * NS;
+  // Q_t loaded, Q_t free (its last QK^T done), K/V ring full/empty, S_t ready, P_t ready,
+  // O_t final, all MMAs done.
+  const int BAR_Q = 0, BAR_QF = 2, BAR_FULL = 4, BAR_EMPTY = 4 + NS, BAR_S = 4 + 2 * NS,
+            BAR_P = 6 + 2 * NS, BAR_O = 8 + 2 * NS, BAR_DONE = 10 + 2 * NS;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + C::kBarOff + C::kNumBars * 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // ---- work unit: query rows [q_first, q_first + 256) of (b, h).  CTAs of one head are
-  // adjacent (they share K/V through L2), heaviest query pairs of each head first.
-  const int bh = (int)(blockIdx.x / p.num_pairs);
-  const int pair = p.num_pairs - 1 - (int)(blockIdx.x % p.num_pairs);
-  const int b = bh / p.Hq;
-  const int h = bh % p.Hq;
-  const int hk = h / p.G;
-  const int q_first = pair * 2 * kBM;
-  const int q_last = min(q_first + 2 * kBM - 1, p.Nq - 1);
-  int lo_a, hi_a, lo_b, hi_b;
-  row_interval(p.mask, q_first, lo_a, hi_a);
-  row_interval(p.mask, q_last, lo_b, hi_b);
-  int jt0 = 0, n_tiles = 0;
-  if (hi_b >= lo_a && p.Nk > 0) {
-    jt0 = lo_a / kBN;
-    n_tiles = hi_b / kBN - jt0 + 1;
-  }
-  const TileRange rng0 = tile_range(p, q_first, jt0, n_tiles);
-  const TileRange rng1 = tile_range(p, q_first + kBM, jt0, n_tiles);
-
   if (threadIdx.x == 0) {
-    mbar_init(bar(BAR_Q), 1);
-    for (int s = 0; s < NS; ++s) {
-      mbar_init(bar(BAR_FULL + s), 1);
-      mbar_init(bar(BAR_EMPTY + s), 1);
-    }
     for (int t = 0; t < 2; ++t) {
+      mbar_init(bar(BAR_Q + t), 1);
+      mbar_init(bar(BAR_QF + t), 1);
       mbar_init(bar(BAR_S + t), 1);
       mbar_init(bar(BAR_P + t), 4);
       mbar_init(bar(BAR_O + t), 1);
+    }
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(bar(BAR_FULL + s), 1);
+      mbar_init(bar(BAR_EMPTY + s), 1);
     }
     mbar_init(bar(BAR_DONE), 1);
     *abort_flag = 0;
@@ -224,50 +256,70 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
   if (warp >= kMmaWarp) {
    regs_decrease<kRegsOther>();
    if (warp == kTmaWarp) {
-    // ------------------------------------------------------------------ TMA producer
+    // ------------------------------------------------------------ K/V TMA producer
     if (lane == 0) {
-      tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
-      const int zq = b * p.Hq + h;
-      const int zkv = b * p.Hkv + hk;
-      mbar_arrive_expect_tx(bar(BAR_Q), 2 * C::kTileBytes);
+      int issued = 0;          // ring loads issued so far, across all pairs
+      for_each_pair(p, [&](int bh, int pair) -> bool {
+        const PairWork w = make_pair_work(p, bh, pair);
+        const int zkv = w.b * p.Hkv + w.hk;
+        for (int i = 0; i < 2 * w.n_tiles; ++i) {
+          const int s = issued % NS;
+          const int round = issued / NS;
+          if (round > 0 &&
+              !mbar_wait(bar(BAR_EMPTY + s), (round - 1) & 1, abort_flag, p.err, kSiteEmpty))
+            return false;
+          mbar_arrive_expect_tx(bar(BAR_FULL + s), C::kTileBytes);
+          const int row = (w.jt0 + (i >> 1)) * kBN;
+          const CUtensorMap* m = (i & 1) ? &tmV : &tmK;
 #pragma unroll
-      for (int t = 0; t < 2; ++t)
-#pragma unroll
-        for (int c = 0; c < C::kChunks; ++c)
-          tma_load_3d(sQ + t * C::kTileBytes + c * C::kChunkBytes, &tmQ, bar(BAR_Q), c * 64,
-                      q_first + t * kBM, zq);
-      int issued = 0;
-      for (int i = 0; i < 2 * n_tiles; ++i) {
-        const int s = i % NS;
-        const int round = i / NS;
-        if (round > 0 &&
-            !mbar_wait(bar(BAR_EMPTY + s), (round - 1) & 1, abort_flag, p.err, kSiteEmpty))
-          break;
-        mbar_arrive_expect_tx(bar(BAR_FULL + s), C::kTileBytes);
-        const int row = (jt0 + (i >> 1)) * kBN;
-        const CUtensorMap* m = (i & 1) ? &tmV : &tmK;
-#pragma unroll
-        for (int c = 0; c < C::kChunks; ++c)
-          tma_load_3d(sRing + s * C::kTileBytes + c * C::kChunkBytes, m, bar(BAR_FULL + s),
-                      c * 64, row, zkv);
-        issued = i + 1;
-      }
+          for (int c = 0; c < C::kChunks; ++c)
+            tma_load_3d(sRing + s * C::kTileBytes + c * C::kChunkBytes, m, bar(BAR_FULL + s),
+                        c * 64, row, zkv);
+          ++issued;
+        }
+        return true;
+      });
       // Outstanding copies must land before the CTA may exit (matters only on abort).
-      mbar_wait(bar(BAR_Q), 0, nullptr, p.err, kSiteDrain);
       for (int s = 0; s < NS && s < issued; ++s) {
         const int last = s + ((issued - 1 - s) / NS) * NS;
         mbar_wait(bar(BAR_FULL + s), (last / NS) & 1, nullptr, p.err, kSiteDrain);
       }
     }
     __syncwarp();
+   } else if (warp == kQWarp) {
+    // -------------------------------------------------------------- Q TMA producer
+    // Each query tile's Q is reloaded as soon as the previous pair's last QK^T of that
+    // tile has completed, independently of the K/V ring.
+    if (lane == 0) {
+      tma_prefetch_desc(&tmQ);
+      int pairs = 0;
+      for_each_pair(p, [&](int bh, int pair) -> bool {
+        const PairWork w = make_pair_work(p, bh, pair);
+        for (int t = 0; t < 2; ++t) {
+          if (pairs > 0 &&
+              !mbar_wait(bar(BAR_QF + t), (pairs - 1) & 1, abort_flag, p.err, kSiteQFree))
+            return false;
+          mbar_arrive_expect_tx(bar(BAR_Q + t), C::kTileBytes);
+#pragma unroll
+          for (int c = 0; c < C::kChunks; ++c)
+            tma_load_3d(sQ + t * C::kTileBytes + c * C::kChunkBytes, &tmQ, bar(BAR_Q + t),
+                        c * 64, w.q_first + t * kBM, w.b * p.Hq + w.h);
+        }
+        ++pairs;
+        return true;
+      });
+      if (pairs > 0)
+        for (int t = 0; t < 2; ++t)
+          mbar_wait(bar(BAR_Q + t), (pairs - 1) & 1, nullptr, p.err, kSiteDrain);
+    }
+    __syncwarp();
    } else if (warp == kMmaWarp) {
     // -------------------------------------------------------------- tcgen05 issuer
-    if (lane == 0 && n_tiles > 0) {
+    if (lane == 0) {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(kBM, kBN, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(kBM, D, true);
-      const TileRange rng[2] = {rng0, rng1};
       // Descriptors differ only in their start-address field (address >> 4, 14 bits; the
       // CTA's shared memory stays below 2^18 bytes, so adding an offset never carries out
       // of it): keep three base descriptors and add offsets in 16-byte units.
@@ -294,56 +346,76 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
                   (!first || kk > 0) ? 1u : 0u);
         }
       };
-      // PV of union step jv for query tile t, if t visits it: wait for P, issue, and
-      // signal the epilogue after the tile's last PV.
-      auto pv_for = [&](int t, int jv, int sv) -> bool {
-        if (jv < rng[t].a || jv > rng[t].b) return true;
-        if (!mbar_wait(bar(BAR_P + t), (jv - rng[t].a) & 1, abort_flag, p.err, kSitePFull))
-          return false;
+      int pairs = 0;        // pairs started
+      int kv = 0;           // ring index of the next K tile
+      int pcount0 = 0, pcount1 = 0;
+      bool ok = true;
+      // PV of union step jv for query tile t (a compile-time constant at every call), if t
+      // visits it: wait for P, issue, and signal the epilogue after the tile's last PV.
+      auto pv_for = [&](const TileRange& rg, int t, int& pcount, int jv, int sv) -> bool {
+        if (jv < rg.a || jv > rg.b) return true;
+        if (!mbar_wait(bar(BAR_P + t), pcount & 1, abort_flag, p.err, kSitePFull)) return false;
+        ++pcount;
         tc_fence_after();
-        issue_pv(t, sv, jv == rng[t].a);
-        if (jv == rng[t].b) umma_commit(bar(BAR_O + t));
+        issue_pv(t, sv, jv == rg.a);
+        if (jv == rg.b) umma_commit(bar(BAR_O + t));
         return true;
       };
-      bool ok = mbar_wait(bar(BAR_Q), 0, abort_flag, p.err, kSiteQ);
-      tc_fence_after();
-      for (int j = 0; ok && j < n_tiles; ++j) {
-        const int ik = 2 * j;
-        const int sk = ik % NS;
-        ok = mbar_wait(bar(BAR_FULL + sk), (ik / NS) & 1, abort_flag, p.err, kSiteFullK);
-        if (!ok) break;
+      for_each_pair(p, [&](int bh, int pair) -> bool {
+        const PairWork w = make_pair_work(p, bh, pair);
+        const TileRange r0 = w.rng[0], r1 = w.rng[1];
+        if (!mbar_wait(bar(BAR_Q + 0), pairs & 1, abort_flag, p.err, kSiteQ)) return ok = false;
+        if (!mbar_wait(bar(BAR_Q + 1), pairs & 1, abort_flag, p.err, kSiteQ)) return ok = false;
+        ++pairs;
         tc_fence_after();
-        int sv = 0;
-        if (j > 0) {
-          const int iv = 2 * (j - 1) + 1;
-          sv = iv % NS;
-          ok = mbar_wait(bar(BAR_FULL + sv), (iv / NS) & 1, abort_flag, p.err, kSiteFullV);
-          if (!ok) break;
+        if (r0.n == 0) umma_commit(bar(BAR_QF + 0));
+        if (r1.n == 0) umma_commit(bar(BAR_QF + 1));
+        const int n = w.n_tiles;
+        for (int j = 0; j < n; ++j) {
+          const int ik = kv + 2 * j;
+          const int sk = ik % NS;
+          if (!mbar_wait(bar(BAR_FULL + sk), (ik / NS) & 1, abort_flag, p.err, kSiteFullK))
+            return ok = false;
           tc_fence_after();
-        }
-        for (int t = 0; t < 2 && ok; ++t) {
-          if (j > 0) ok = pv_for(t, j - 1, sv);
-          if (ok && j >= rng[t].a && j <= rng[t].b) {
-            // In-order tensor pipe: this overwrites S_t (and P_t inside it) only after
-            // the PV MMA just issued has read P_t.
-            issue_qk(t, sk);
-            umma_commit(bar(BAR_S + t));
+          int sv = 0;
+          if (j > 0) {
+            const int iv = ik - 1;
+            sv = iv % NS;
+            if (!mbar_wait(bar(BAR_FULL + sv), (iv / NS) & 1, abort_flag, p.err, kSiteFullV))
+              return ok = false;
+            tc_fence_after();
           }
+          // Per query tile: PV of the previous step, then QK^T of this one.  In-order
+          // tensor pipe: the QK^T overwrites S_t (and P_t inside it) only after the PV MMA
+          // just issued has read P_t.
+          if (j > 0 && !pv_for(r0, 0, pcount0, j - 1, sv)) return ok = false;
+          if (j >= r0.a && j <= r0.b) {
+            issue_qk(0, sk);
+            umma_commit(bar(BAR_S + 0));
+            if (j == r0.b) umma_commit(bar(BAR_QF + 0));
+          }
+          if (j > 0 && !pv_for(r1, 1, pcount1, j - 1, sv)) return ok = false;
+          if (j >= r1.a && j <= r1.b) {
+            issue_qk(1, sk);
+            umma_commit(bar(BAR_S + 1));
+            if (j == r1.b) umma_commit(bar(BAR_QF + 1));
+          }
+          if (j > 0) umma_commit(bar(BAR_EMPTY + sv));
+          umma_commit(bar(BAR_EMPTY + sk));
         }
-        if (!ok) break;
-        if (j > 0) umma_commit(bar(BAR_EMPTY + sv));
-        umma_commit(bar(BAR_EMPTY + sk));
-      }
-      if (ok) {
-        const int iv = 2 * (n_tiles - 1) + 1;
-        const int sv = iv % NS;
-        ok = mbar_wait(bar(BAR_FULL + sv), (iv / NS) & 1, abort_flag, p.err, kSiteFullV);
-        if (ok) {
+        if (n > 0) {
+          const int iv = kv + 2 * n - 1;
+          const int sv = iv % NS;
+          if (!mbar_wait(bar(BAR_FULL + sv), (iv / NS) & 1, abort_flag, p.err, kSiteFullV))
+            return ok = false;
           tc_fence_after();
-          for (int t = 0; t < 2 && ok; ++t) ok = pv_for(t, n_tiles - 1, sv);
+          if (!pv_for(r0, 0, pcount0, n - 1, sv)) return ok = false;
+          if (!pv_for(r1, 1, pcount1, n - 1, sv)) return ok = false;
+          umma_commit(bar(BAR_EMPTY + sv));
         }
-        umma_commit(bar(BAR_EMPTY + sv));
-      }
+        kv += 2 * n;
+        return true;
+      });
       // Every MMA issued above must be complete before TMEM is released.
       umma_commit(bar(BAR_DONE));
       mbar_wait(bar(BAR_DONE), 0, nullptr, p.err, kSiteDrain);
@@ -356,116 +428,119 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
     const int t = warp >> 2;                 // query tile of this warpgroup
     const int wq = warp & 3;                 // TMEM lane quarter this warp may access
     const int r = wq * 32 + lane;            // row inside the tile
-    const int tq0 = q_first + t * kBM;
-    const int row = tq0 + r;
-    const TileRange rng = t ? rng1 : rng0;
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
     const uint32_t tS = tmem + lane_off + 128u * t;
     const uint32_t tP = tS + 64u;
     const uint32_t tO = tmem + lane_off + 256u + 128u * t;
+    int scount = 0, ocount = 0;
 
-    int row_lo, row_hi;
-    row_interval(p.mask, row, row_lo, row_hi);
-    // Tile-level bounds: a K/V tile needs no mask when every valid row of this query tile
-    // sees every key of it and it lies inside Nk.
-    int lo_last = 0, hi_first = 0;
-    if (rng.n > 0) {
-      int a0, a1;
-      row_interval(p.mask, min(tq0 + kBM, p.Nq) - 1, lo_last, a0);
-      row_interval(p.mask, tq0, a1, hi_first);
-    }
-
-    float m_ref = -INFINITY;   // reference max (log2 units) of the exponentials in O and l
-    float l = 0.f;
-    bool ok = true;
-    for (int i = 0; i < rng.n; ++i) {
-      ok = mbar_wait(bar(BAR_S + t), i & 1, abort_flag, p.err, kSiteSFull);
-      ok = __all_sync(0xffffffffu, ok);
-      if (!ok) break;
-      tc_fence_after();
-      uint32_t s[128];
-      tmem_ld_x128(tS, s);
-      const int k0 = (jt0 + rng.a + i) * kBN;
-      const bool masked = !(lo_last <= k0 && k0 + kBN - 1 <= hi_first && k0 + kBN <= p.Nk);
-      const float mx_raw = masked ? tile_row_max<true>(s, row_lo - k0, row_hi - k0)
-                                  : tile_row_max<false>(s, 0, 0);
-      const float mx = (p.softcap > 0.f) ? scaled_score<true>(mx_raw, p)
-                                         : scaled_score<false>(mx_raw, p);
-      const float m_new = fmaxf(m_ref, mx);
-      const bool need = m_new > m_ref + kRescaleThreshold;
-      float alpha = 1.f;
-      if (need) {
-        alpha = ex2_approx(m_ref - m_new);
-        m_ref = m_new;
+    for_each_pair(p, [&](int bh, int pair) -> bool {
+      const PairWork w = make_pair_work(p, bh, pair);
+      const TileRange rng = t ? w.rng[1] : w.rng[0];
+      const int tq0 = w.q_first + t * kBM;
+      const int row = tq0 + r;
+      int row_lo, row_hi;
+      row_interval(p.mask, row, row_lo, row_hi);
+      // Tile-level bounds: a K/V tile needs no mask when every valid row of this query
+      // tile sees every key of it and it lies inside Nk.
+      int lo_last = 0, hi_first = 0;
+      if (rng.n > 0) {
+        int a0, a1;
+        row_interval(p.mask, min(tq0 + kBM, p.Nq) - 1, lo_last, a0);
+        row_interval(p.mask, tq0, a1, hi_first);
       }
-      // P = 2^(x - m_ref) as bf16 pairs, written over the upper half of S in TMEM; each
-      // 64-column half is stored as soon as it is packed.  Masked scores are -inf, so
-      // their exponentials are exactly 0.
-      const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
-      float sum = 0.f;
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t pk[32];
-        if (p.softcap > 0.f) {
-          sum += tile_row_exp_half<true>(s, 64 * half, p, m_use, pk);
-        } else {
-          sum += tile_row_exp_half<false>(s, 64 * half, p, m_use, pk);
+
+      float m_ref = -INFINITY;   // reference max (log2 units) of the exponentials in O, l
+      float l = 0.f;
+      for (int i = 0; i < rng.n; ++i) {
+        bool ok = mbar_wait(bar(BAR_S + t), scount & 1, abort_flag, p.err, kSiteSFull);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) return false;
+        ++scount;
+        tc_fence_after();
+        uint32_t s[128];
+        tmem_ld_x128(tS, s);
+        const int k0 = (w.jt0 + rng.a + i) * kBN;
+        const bool masked =
+            !(lo_last <= k0 && k0 + kBN - 1 <= hi_first && k0 + kBN <= p.Nk);
+        const float mx_raw = masked ? tile_row_max<true>(s, row_lo - k0, row_hi - k0)
+                                    : tile_row_max<false>(s, 0, 0);
+        const float mx = (p.softcap > 0.f) ? scaled_score<true>(mx_raw, p)
+                                           : scaled_score<false>(mx_raw, p);
+        const float m_new = fmaxf(m_ref, mx);
+        const bool need = m_new > m_ref + kRescaleThreshold;
+        float alpha = 1.f;
+        if (need) {
+          alpha = ex2_approx(m_ref - m_new);
+          m_ref = m_new;
         }
-        tmem_st_x32(tP + 32u * half, pk);
-      }
-      l = l * alpha + sum;
-      if (i > 0 && __any_sync(0xffffffffu, need)) {
-        // Rescale this row of O.  PV of the previous tile is complete: the commit that
-        // signalled this S was issued after it.  The next PV is issued only after the
-        // arrive below.
+        // P = 2^(x - m_ref) as bf16 pairs, written over the upper half of S in TMEM; each
+        // 64-column half is stored as soon as it is packed.  Masked scores are -inf, so
+        // their exponentials are exactly 0.
+        const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
+        float sum = 0.f;
 #pragma unroll
-        for (int cc = 0; cc < D / 32; ++cc) {
-          uint32_t o[32];
-          tmem_ld_x32(tO + 32u * cc, o);
-#pragma unroll
-          for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(f32(o[k]) * alpha);
-          tmem_st_x32(tO + 32u * cc, o);
+        for (int half = 0; half < 2; ++half) {
+          uint32_t pk[32];
+          if (p.softcap > 0.f) {
+            sum += tile_row_exp_half<true>(s, 64 * half, p, m_use, pk);
+          } else {
+            sum += tile_row_exp_half<false>(s, 64 * half, p, m_use, pk);
+          }
+          tmem_st_x32(tP + 32u * half, pk);
         }
+        l = l * alpha + sum;
+        if (i > 0 && __any_sync(0xffffffffu, need)) {
+          // Rescale this row of O.  PV of the previous tile is complete: the commit that
+          // signalled this S was issued after it.  The next PV is issued only after the
+          // arrive below.
+#pragma unroll
+          for (int cc = 0; cc < D / 32; ++cc) {
+            uint32_t o[32];
+            tmem_ld_x32(tO + 32u * cc, o);
+#pragma unroll
+            for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(f32(o[k]) * alpha);
+            tmem_st_x32(tO + 32u * cc, o);
+          }
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(BAR_P + t));
       }
-      tmem_wait_st();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(BAR_P + t));
-    }
+      if (rng.n == 0) return true;   // no valid row in this query tile
 
-    if (ok && rng.n > 0) {
-      ok = mbar_wait(bar(BAR_O + t), 0, abort_flag, p.err, kSiteOFinal);
+      // Epilogue.  Reading O here, before this warpgroup's next arrive on P, orders it
+      // before the next pair's first PV (which overwrites O).
+      bool ok = mbar_wait(bar(BAR_O + t), ocount & 1, abort_flag, p.err, kSiteOFinal);
       ok = __all_sync(0xffffffffu, ok);
-    }
-    if (ok) {
+      if (!ok) return false;
+      ++ocount;
       tc_fence_after();
       const bool valid = row < p.Nq;
       const float inv_l = (l > 0.f) ? 1.0f / l : 0.f;
       const float lse = (l > 0.f) ? (m_ref + log2f(l)) * kLn2 : -INFINITY;
-      const size_t row_index = (size_t)(b * p.Hq + h) * (size_t)p.Nq + (size_t)row;
+      const size_t row_index = (size_t)(w.b * p.Hq + w.h) * (size_t)p.Nq + (size_t)row;
       __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.o) + row_index * D;
 #pragma unroll
       for (int cc = 0; cc < D / 32; ++cc) {
         uint32_t o[32];
-        if (rng.n > 0) {
-          tmem_ld_x32(tO + 32u * cc, o);
-        } else {
-#pragma unroll
-          for (int k = 0; k < 32; ++k) o[k] = 0u;
-        }
-        uint32_t w[16];
+        tmem_ld_x32(tO + 32u * cc, o);
+        uint32_t wv[16];
 #pragma unroll
         for (int k = 0; k < 16; ++k)
-          w[k] = pack_bf16x2(f32(o[2 * k]) * inv_l, f32(o[2 * k + 1]) * inv_l);
+          wv[k] = pack_bf16x2(f32(o[2 * k]) * inv_l, f32(o[2 * k + 1]) * inv_l);
         if (valid) {
           uint4* dst = reinterpret_cast<uint4*>(orow + 32 * cc);
 #pragma unroll
           for (int k = 0; k < 4; ++k)
-            dst[k] = make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+            dst[k] = make_uint4(wv[4 * k], wv[4 * k + 1], wv[4 * k + 2], wv[4 * k + 3]);
         }
       }
       if (valid) p.lse[row_index] = lse;
-    }
+      tc_fence_before();
+      return true;
+    });
   }
 
   tc_fence_before();
@@ -493,7 +568,8 @@ int launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& 
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        C::kSmemBytes);
   if (e != cudaSuccess) return -4;
-  const long long grid = (long long)p.num_pairs * p.B * p.Hq;
+  const long long units = (long long)((p.num_pairs + 1) / 2) * p.B * p.Hq;
+  const long long grid = units < p.num_sms ? units : p.num_sms;
   attn_fwd_sm100_kernel<D><<<(unsigned)grid, kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, p);
   return cudaGetLastError() == cudaSuccess ? 0 : -4;
 }
