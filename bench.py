@@ -138,17 +138,22 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ distributed plumbing
-def dist_setup(n_gpus: int):
+def dist_setup(n_gpus: int, backend: str | None = None):
+    """One process per GPU under torchrun: NCCL when CUDA is present (gloo only for the
+    CPU tests of this plumbing). Returns (world, rank, local rank)."""
     import torch
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    if backend is None:
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
     if world > 1:
         import datetime
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
-    else:
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+    elif torch.cuda.is_available():
         torch.cuda.set_device(0)
     return world, rank, local
 
@@ -160,13 +165,20 @@ def barrier(world):
 
 
 def max_over_ranks(world, x: float) -> float:
+    """The slowest rank's figure (all ranks take part; every rank gets the result)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def whole_job_rate(units_per_rank: float, world: int, ms_max: float) -> float:
+    """Weak scaling of independent replicas: all ranks' units over the slowest rank's time."""
+    return units_per_rank * world / (ms_max * 1e-3)
 
 
 # ----------------------------------------------------------------------- CPU baseline
@@ -284,7 +296,7 @@ def run_ours(args, world, rank, local):
         raise RuntimeError("device status not ok after timed steps")
     ms_step = max_over_ranks(world, total_ms / args.steps)
     kernel_ms = max_over_ranks(world, sum(per) / len(per))
-    value = flops * world / (ms_step * 1e-3) / 1e12
+    value = whole_job_rate(flops, world, ms_step) / 1e12
     achieved = flops / (kernel_ms * 1e-3) / 1e12
     peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     out = {
@@ -384,7 +396,7 @@ def bench_decode(args, world, local, peaks, peak_src):
     kv = accounting.decode_kv_bytes(w.B, w.Hkv, w.Nk, w.d)
     io = accounting.decode_io_bytes(w.B, w.Hq, w.Hkv, w.Nk, w.d)
     peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
-    gbs = kv * world / (ms * 1e-3) / 1e9
+    gbs = whole_job_rate(kv, world, ms) / 1e9
     res = {"workload": w.name, "value": round(gbs, 1), "unit": "GB/s (KV cache)",
            "tokens_per_s": round(w.B * world / (ms * 1e-3), 1), "ms_per_step": round(ms, 4),
            "num_splits": S, "kv_bytes_per_step": kv,
