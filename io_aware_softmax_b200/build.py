@@ -25,11 +25,21 @@ HEADERS = ["attn_internal.h", "mask.cuh", "sm100_ptx.cuh", "tmem_ldst.cuh"]
 ARCH_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 # The prefill kernel splits its launch registers between warpgroups with setmaxnreg
-# (two softmax warpgroups at 200, one at 96, 384 threads).  The split must fit in what the
-# CTA is launched with, or the increase would wait forever: check the count ptxas chose.
+# (two softmax warpgroups, one warpgroup of MMA/TMA warps, 384 threads).  The split must fit
+# in what the CTA is launched with, or the increase would wait forever: check the count
+# ptxas chose against the split constants read from the kernel source.
 PREFILL_KERNEL = "attn_fwd_sm100_kernel"
 PREFILL_THREADS = 384
-PREFILL_SPLIT_REGS = 2 * 128 * 200 + 128 * 96
+
+
+def _prefill_split_regs() -> int:
+    src = open(os.path.join(CSRC, "attn_prefill.cu"), encoding="utf-8").read()
+    soft = int(re.search(r"kRegsSoftmax\s*=\s*(\d+)", src).group(1))
+    other = int(re.search(r"kRegsOther\s*=\s*(\d+)", src).group(1))
+    return 2 * 128 * soft + 128 * other
+
+
+PREFILL_SPLIT_REGS = _prefill_split_regs()
 
 
 def check_register_budget(ptxas_log: str) -> dict:

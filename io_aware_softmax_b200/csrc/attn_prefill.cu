@@ -317,7 +317,9 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
     __syncwarp();
    } else if (warp == kMmaWarp) {
     // -------------------------------------------------------------- tcgen05 issuer
-    if (lane == 0) {
+    // The whole warp runs this role with warp-uniform values and one elected lane issues
+    // each tensor-core operation, so descriptors stay in the uniform datapath.
+    {
       constexpr uint32_t idesc_qk = idesc_bf16_f32(kBM, kBN, false);
       constexpr uint32_t idesc_pv = idesc_bf16_f32(kBM, D, true);
       // Descriptors differ only in their start-address field (address >> 4, 14 bits; the
@@ -333,7 +335,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = ((kk >> 2) * C::kChunkBytes + (kk & 3) * 32) >> 4;
-          umma_ss(d_tmem, dQ + q_off + off, dK + k_off + off, idesc_qk, kk > 0 ? 1u : 0u);
+          umma_ss_warp(d_tmem, dQ + q_off + off, dK + k_off + off, idesc_qk, kk > 0 ? 1u : 0u);
         }
       };
       auto issue_pv = [&](int t, int sv, bool first) {
@@ -342,7 +344,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
         const uint32_t v_off = (uint32_t)(sv * C::kTileBytes) >> 4;
 #pragma unroll
         for (int kk = 0; kk < kBN / 16; ++kk) {
-          umma_ts(d_tmem, a_tmem + 8u * kk, dV + v_off + ((kk * 16 * 128) >> 4), idesc_pv,
+          umma_ts_warp(d_tmem, a_tmem + 8u * kk, dV + v_off + ((kk * 16 * 128) >> 4), idesc_pv,
                   (!first || kk > 0) ? 1u : 0u);
         }
       };
@@ -354,34 +356,34 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
       // visits it: wait for P, issue, and signal the epilogue after the tile's last PV.
       auto pv_for = [&](const TileRange& rg, int t, int& pcount, int jv, int sv) -> bool {
         if (jv < rg.a || jv > rg.b) return true;
-        if (!mbar_wait(bar(BAR_P + t), pcount & 1, abort_flag, p.err, kSitePFull)) return false;
+        if (!mbar_wait_warp(bar(BAR_P + t), pcount & 1, abort_flag, p.err, kSitePFull)) return false;
         ++pcount;
         tc_fence_after();
         issue_pv(t, sv, jv == rg.a);
-        if (jv == rg.b) umma_commit(bar(BAR_O + t));
+        if (jv == rg.b) umma_commit_warp(bar(BAR_O + t));
         return true;
       };
       for_each_pair(p, [&](int bh, int pair) -> bool {
         const PairWork w = make_pair_work(p, bh, pair);
         const TileRange r0 = w.rng[0], r1 = w.rng[1];
-        if (!mbar_wait(bar(BAR_Q + 0), pairs & 1, abort_flag, p.err, kSiteQ)) return ok = false;
-        if (!mbar_wait(bar(BAR_Q + 1), pairs & 1, abort_flag, p.err, kSiteQ)) return ok = false;
+        if (!mbar_wait_warp(bar(BAR_Q + 0), pairs & 1, abort_flag, p.err, kSiteQ)) return ok = false;
+        if (!mbar_wait_warp(bar(BAR_Q + 1), pairs & 1, abort_flag, p.err, kSiteQ)) return ok = false;
         ++pairs;
         tc_fence_after();
-        if (r0.n == 0) umma_commit(bar(BAR_QF + 0));
-        if (r1.n == 0) umma_commit(bar(BAR_QF + 1));
+        if (r0.n == 0) umma_commit_warp(bar(BAR_QF + 0));
+        if (r1.n == 0) umma_commit_warp(bar(BAR_QF + 1));
         const int n = w.n_tiles;
         for (int j = 0; j < n; ++j) {
           const int ik = kv + 2 * j;
-          const int sk = ik % NS;
-          if (!mbar_wait(bar(BAR_FULL + sk), (ik / NS) & 1, abort_flag, p.err, kSiteFullK))
+          const int sk = (int)((unsigned)ik % (unsigned)NS);
+          if (!mbar_wait_warp(bar(BAR_FULL + sk), ((unsigned)ik / NS) & 1, abort_flag, p.err, kSiteFullK))
             return ok = false;
           tc_fence_after();
           int sv = 0;
           if (j > 0) {
             const int iv = ik - 1;
-            sv = iv % NS;
-            if (!mbar_wait(bar(BAR_FULL + sv), (iv / NS) & 1, abort_flag, p.err, kSiteFullV))
+            sv = (int)((unsigned)iv % (unsigned)NS);
+            if (!mbar_wait_warp(bar(BAR_FULL + sv), ((unsigned)iv / NS) & 1, abort_flag, p.err, kSiteFullV))
               return ok = false;
             tc_fence_after();
           }
@@ -391,34 +393,34 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
           if (j > 0 && !pv_for(r0, 0, pcount0, j - 1, sv)) return ok = false;
           if (j >= r0.a && j <= r0.b) {
             issue_qk(0, sk);
-            umma_commit(bar(BAR_S + 0));
-            if (j == r0.b) umma_commit(bar(BAR_QF + 0));
+            umma_commit_warp(bar(BAR_S + 0));
+            if (j == r0.b) umma_commit_warp(bar(BAR_QF + 0));
           }
           if (j > 0 && !pv_for(r1, 1, pcount1, j - 1, sv)) return ok = false;
           if (j >= r1.a && j <= r1.b) {
             issue_qk(1, sk);
-            umma_commit(bar(BAR_S + 1));
-            if (j == r1.b) umma_commit(bar(BAR_QF + 1));
+            umma_commit_warp(bar(BAR_S + 1));
+            if (j == r1.b) umma_commit_warp(bar(BAR_QF + 1));
           }
-          if (j > 0) umma_commit(bar(BAR_EMPTY + sv));
-          umma_commit(bar(BAR_EMPTY + sk));
+          if (j > 0) umma_commit_warp(bar(BAR_EMPTY + sv));
+          umma_commit_warp(bar(BAR_EMPTY + sk));
         }
         if (n > 0) {
           const int iv = kv + 2 * n - 1;
-          const int sv = iv % NS;
-          if (!mbar_wait(bar(BAR_FULL + sv), (iv / NS) & 1, abort_flag, p.err, kSiteFullV))
+          const int sv = (int)((unsigned)iv % (unsigned)NS);
+          if (!mbar_wait_warp(bar(BAR_FULL + sv), ((unsigned)iv / NS) & 1, abort_flag, p.err, kSiteFullV))
             return ok = false;
           tc_fence_after();
           if (!pv_for(r0, 0, pcount0, n - 1, sv)) return ok = false;
           if (!pv_for(r1, 1, pcount1, n - 1, sv)) return ok = false;
-          umma_commit(bar(BAR_EMPTY + sv));
+          umma_commit_warp(bar(BAR_EMPTY + sv));
         }
         kv += 2 * n;
         return true;
       });
       // Every MMA issued above must be complete before TMEM is released.
-      umma_commit(bar(BAR_DONE));
-      mbar_wait(bar(BAR_DONE), 0, nullptr, p.err, kSiteDrain);
+      umma_commit_warp(bar(BAR_DONE));
+      mbar_wait_warp(bar(BAR_DONE), 0, nullptr, p.err, kSiteDrain);
     }
     __syncwarp();
    }

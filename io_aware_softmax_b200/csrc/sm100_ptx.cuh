@@ -75,6 +75,23 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// As mbar_try_wait, but the thread may sleep (up to hint_ns) until the phase completes
+// instead of returning at once, so a waiting warp leaves its issue slots to the others.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity,
+                                                    uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
+constexpr uint32_t kWaitSleepNs = 200u * 1000u;   // one sleep of a waiting thread, at most
+
 // Waits for the phase with the given parity to complete.  Returns false (after recording
 // the error and raising *abort) if it does not complete within kWaitLimitNs, or if another
 // thread of the CTA has already raised *abort.  With abort == nullptr (the drain waits of
@@ -83,15 +100,34 @@ static __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, 
                                                  uint32_t* err, uint32_t site) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
-  for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 63u) == 0) {
-      if (abort != nullptr && *abort) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+  for (;;) {
+    if (mbar_try_wait_sleep(bar, parity, kWaitSleepNs)) return true;
+    if (abort != nullptr && *abort) return false;
+    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      report_error(err, kErrWaitTimeout, site);
+      if (abort != nullptr) *abort = 1;
+      return false;
+    }
+  }
+}
+
+// mbar_wait for a whole converged warp: every lane polls, and the warp leaves together with
+// one verdict (a phase seen complete by some lanes is complete for all of them).
+static __device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity,
+                                                      volatile int* abort, uint32_t* err,
+                                                      uint32_t site) {
+  if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (;;) {
+    if (__all_sync(0xffffffffu, mbar_try_wait_sleep(bar, parity, kWaitSleepNs))) return true;
+    const bool stop = (abort != nullptr && *abort) || globaltimer_ns() - t0 > kWaitLimitNs;
+    if (__any_sync(0xffffffffu, stop)) {
+      if ((threadIdx.x & 31) == 0 && !(abort != nullptr && *abort)) {
         report_error(err, kErrWaitTimeout, site);
         if (abort != nullptr) *abort = 1;
-        return false;
       }
+      __syncwarp();
+      return false;
     }
   }
 }
@@ -158,6 +194,35 @@ __device__ __forceinline__ void umma_commit(uint32_t bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
                    bar)
                : "memory");
+}
+
+// Warp-wide forms: the whole (converged) warp executes them with warp-uniform operands and
+// one elected lane issues the tensor-core operation, so the operands can stay in the
+// uniform datapath instead of being moved there from one thread's registers per call.
+__device__ __forceinline__ void umma_ss_warp(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                             uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred e, p;\n\telect.sync _|e, 0xffffffff;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void umma_ts_warp(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                             uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred e, p;\n\telect.sync _|e, 0xffffffff;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void umma_commit_warp(uint32_t bar) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(
+          bar)
+      : "memory");
 }
 
 __device__ __forceinline__ void tmem_wait_st() {
