@@ -48,9 +48,9 @@ constexpr int kMmaWarp = 8;
 constexpr int kTmaWarp = 9;
 constexpr int kQWarp = 10;
 // Registers per thread after the split; the launch gives 168 (65536 / 384, rounded down to
-// a multiple of 8): 2 * 128 * 200 + 128 * 96 = 63488 <= 384 * 168 = 64512.
-constexpr uint32_t kRegsSoftmax = 200;
-constexpr uint32_t kRegsOther = 96;
+// a multiple of 8): 2 * 128 * 192 + 128 * 112 = 63488 <= 384 * 168 = 64512.
+constexpr uint32_t kRegsSoftmax = 192;
+constexpr uint32_t kRegsOther = 112;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units: rescale when max grows > 2^8
 constexpr float kLn2 = 0.69314718055994531f;
@@ -65,8 +65,8 @@ struct Cfg {
   static constexpr int kQOff = 0;
   static constexpr int kRingOff = 2 * kTileBytes;
   static constexpr int kBarOff = kRingOff + kStages * kTileBytes;
-  // barriers: q[2], q_free[2], full[S], empty[S], s[2], p[2], o[2], done
-  static constexpr int kNumBars = 11 + 2 * kStages;
+  // barriers: q[2], q_free[2], full[S], empty[S], s[2], p[2][2 key halves], o[2], done
+  static constexpr int kNumBars = 13 + 2 * kStages;
   static constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 16 + 1024;
 };
 
@@ -221,7 +221,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
   // Q_t loaded, Q_t free (its last QK^T done), K/V ring full/empty, S_t ready, P_t ready,
   // O_t final, all MMAs done.
   const int BAR_Q = 0, BAR_QF = 2, BAR_FULL = 4, BAR_EMPTY = 4 + NS, BAR_S = 4 + 2 * NS,
-            BAR_P = 6 + 2 * NS, BAR_O = 8 + 2 * NS, BAR_DONE = 10 + 2 * NS;
+            BAR_P = 6 + 2 * NS, BAR_O = 10 + 2 * NS, BAR_DONE = 12 + 2 * NS;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + C::kBarOff + C::kNumBars * 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -233,7 +233,8 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
       mbar_init(bar(BAR_Q + t), 1);
       mbar_init(bar(BAR_QF + t), 1);
       mbar_init(bar(BAR_S + t), 1);
-      mbar_init(bar(BAR_P + t), 4);
+      mbar_init(bar(BAR_P + 2 * t), 4);
+      mbar_init(bar(BAR_P + 2 * t + 1), 4);
       mbar_init(bar(BAR_O + t), 1);
     }
     for (int s = 0; s < NS; ++s) {
@@ -338,14 +339,16 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
           umma_ss_warp(d_tmem, dQ + q_off + off, dK + k_off + off, idesc_qk, kk > 0 ? 1u : 0u);
         }
       };
-      auto issue_pv = [&](int t, int sv, bool first) {
+      // O_t += P_t[:, 64h : 64h + 64] V_j[64h : 64h + 64]: key half h of the PV product.
+      auto issue_pv_half = [&](int t, int sv, int h, bool first) {
         const uint32_t d_tmem = tmem + 256u + 128u * t;
         const uint32_t a_tmem = tmem + 128u * t + 64u;
         const uint32_t v_off = (uint32_t)(sv * C::kTileBytes) >> 4;
 #pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk) {
+        for (int k = 0; k < kBN / 32; ++k) {
+          const int kk = h * (kBN / 32) + k;
           umma_ts_warp(d_tmem, a_tmem + 8u * kk, dV + v_off + ((kk * 16 * 128) >> 4), idesc_pv,
-                  (!first || kk > 0) ? 1u : 0u);
+                       (!first || kk > 0) ? 1u : 0u);
         }
       };
       int pairs = 0;        // pairs started
@@ -356,10 +359,16 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
       // visits it: wait for P, issue, and signal the epilogue after the tile's last PV.
       auto pv_for = [&](const TileRange& rg, int t, int& pcount, int jv, int sv) -> bool {
         if (jv < rg.a || jv > rg.b) return true;
-        if (!mbar_wait_warp(bar(BAR_P + t), pcount & 1, abort_flag, p.err, kSitePFull)) return false;
+        // The softmax hands P over in two key halves; the first half's product runs while
+        // the second half is being computed.
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          if (!mbar_wait_warp(bar(BAR_P + 2 * t + h), pcount & 1, abort_flag, p.err, kSitePFull))
+            return false;
+          tc_fence_after();
+          issue_pv_half(t, sv, h, jv == rg.a);
+        }
         ++pcount;
-        tc_fence_after();
-        issue_pv(t, sv, jv == rg.a);
         if (jv == rg.b) umma_commit_warp(bar(BAR_O + t));
         return true;
       };
@@ -476,8 +485,21 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
           alpha = ex2_approx(m_ref - m_new);
           m_ref = m_new;
         }
-        // P = 2^(x - m_ref) as bf16 pairs, written over the upper half of S in TMEM; each
-        // 64-column half is stored as soon as it is packed.  Masked scores are -inf, so
+        if (i > 0 && __any_sync(0xffffffffu, need)) {
+          // Rescale this row of O.  PV of the previous tile is complete: the commit that
+          // signalled this S was issued after it.  The next PV is issued only after the
+          // arrives below.
+#pragma unroll 1
+          for (int cc = 0; cc < D / 16; ++cc) {
+            uint32_t o[16];
+            tmem_ld_x16(tO + 16u * cc, o);
+#pragma unroll
+            for (int k = 0; k < 16; ++k) o[k] = __float_as_uint(f32(o[k]) * alpha);
+            tmem_st_x16(tO + 16u * cc, o);
+          }
+        }
+        // P = 2^(x - m_ref) as bf16 pairs, written over the upper half of S in TMEM and
+        // handed to the tensor core one 64-key half at a time.  Masked scores are -inf, so
         // their exponentials are exactly 0.
         const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
         float sum = 0.f;
@@ -490,25 +512,12 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
             sum += tile_row_exp_half<false>(s, 64 * half, p, m_use, pk);
           }
           tmem_st_x32(tP + 32u * half, pk);
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(BAR_P + 2 * t + half));
         }
         l = l * alpha + sum;
-        if (i > 0 && __any_sync(0xffffffffu, need)) {
-          // Rescale this row of O.  PV of the previous tile is complete: the commit that
-          // signalled this S was issued after it.  The next PV is issued only after the
-          // arrive below.
-#pragma unroll
-          for (int cc = 0; cc < D / 32; ++cc) {
-            uint32_t o[32];
-            tmem_ld_x32(tO + 32u * cc, o);
-#pragma unroll
-            for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(f32(o[k]) * alpha);
-            tmem_st_x32(tO + 32u * cc, o);
-          }
-        }
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(BAR_P + t));
       }
       if (rng.n == 0) return true;   // no valid row in this query tile
 
