@@ -29,6 +29,10 @@ What it computes, and where that is written down (pages cited by title and secti
   "3.7 어텐션 II", section 3.7.5; FlashAttention page, "사례 4: GQA/MQA 지원 문제".
 * Packed documents delimited by cumulative boundaries (``cu_seqlens``):
   "3.7 어텐션 II", section 3.7.6.
+* ALiBi: a distance-based positional bias added to the score before the softmax, fused in
+  the kernel rather than passed as a mask tensor: "3.7 어텐션 II", section 3.7.5
+  ("ALiBi·위치 바이어스").  The symmetric (non-causal) window is the FlexAttention page's
+  ``sliding_window_mod`` as written, |q_idx - kv_idx| <= window.
 * The tiled online-softmax form (normalised-O update with alpha = exp(m_old - m_new),
   beta = exp(m_local - m_new)): FlashAttention page, sections "Online Softmax와 블록 단위
   누적" and "알고리즘 의사코드".
@@ -39,7 +43,10 @@ Readings taken where the pages are silent (each is listed in the design doc as well):
 
 * soft-cap acts on the *scaled* score: s <- c * tanh(s / c) with s = scale * q.k;
 * causal means kv <= q (diagonal visible); the sliding window is one-sided and causal:
-  visible iff 0 <= q - kv <= window;
+  visible iff 0 <= q - kv <= window; the symmetric window (mask kind 4) is
+  visible iff |q - kv| <= window, with no causality;
+* the ALiBi bias of query head h is -slope_h * |q - kv| (natural-log units, the slopes
+  given per query head), added after the soft-cap and before the mask;
 * the document mask is "same document AND kv <= q", the documents given by int32
   boundaries [0, ..., Nk] shared by every batch entry;
 * masks other than "none" need Nq == Nk;
@@ -61,6 +68,7 @@ MASK_NONE = 0
 MASK_CAUSAL = 1
 MASK_SLIDING_CAUSAL = 2
 MASK_DOCUMENT_CAUSAL = 3
+MASK_SLIDING = 4
 
 TILE_EMPTY = 0
 TILE_PARTIAL = 1
@@ -98,6 +106,8 @@ def visible(q_idx, kv_idx, mask_kind: int, window: int = 0, doc_offsets=None) ->
     kv = np.asarray(kv_idx, dtype=np.int64)
     if mask_kind == MASK_NONE:
         return np.ones(np.broadcast(q, kv).shape, dtype=bool)
+    if mask_kind == MASK_SLIDING:
+        return np.abs(q - kv) <= window
     causal = kv <= q
     if mask_kind == MASK_CAUSAL:
         return causal
@@ -118,11 +128,12 @@ def softcap_scores(s: np.ndarray, softcap: float) -> np.ndarray:
 
 
 def head_scores(q_rows, K, scale: float, softcap: float, row_idx, mask_kind: int,
-                window: int, doc_offsets, kv_idx=None) -> np.ndarray:
+                window: int, doc_offsets, kv_idx=None, alibi_slope: float = 0.0) -> np.ndarray:
     """Materialised score block S (rows x keys), -inf where masked.
 
-    S = scale * Q K^T, then the score hook (soft-cap), then the mask: FlexAttention page
-    section 2 (the hook sees the score right after Q.K^T); the standard_attention listing
+    S = scale * Q K^T, then the score hook (soft-cap), then the ALiBi distance bias, then
+    the mask: FlexAttention page section 2 (the hook sees the score right after Q.K^T);
+    "3.7 어텐션 II" 3.7.5 (bias added before the softmax); the standard_attention listing
     on the FlashAttention page (masked_fill with -inf)."""
     Q = _f64(q_rows)
     Kf = _f64(K)
@@ -130,6 +141,10 @@ def head_scores(q_rows, K, scale: float, softcap: float, row_idx, mask_kind: int
     S = softcap_scores(S, softcap)
     if kv_idx is None:
         kv_idx = np.arange(Kf.shape[0])
+    if alibi_slope:
+        dist = np.abs(np.asarray(row_idx, dtype=np.float64)[:, None]
+                      - np.asarray(kv_idx, dtype=np.float64)[None, :])
+        S = S - float(alibi_slope) * dist
     vis = visible(np.asarray(row_idx)[:, None], np.asarray(kv_idx)[None, :],
                   mask_kind, window, doc_offsets)
     return np.where(vis, S, -np.inf)
@@ -151,13 +166,13 @@ def softmax_rows(S: np.ndarray):
 
 def attention_head(q_rows, row_idx, K, V, scale: float, mask_kind: int = MASK_NONE,
                    window: int = 0, softcap: float = 0.0, doc_offsets=None,
-                   return_probs: bool = False, kv_idx=None):
+                   return_probs: bool = False, kv_idx=None, alibi_slope: float = 0.0):
     """Exact attention for some query rows of one (batch, head) against all keys.
 
     O_i = sum_j P_ij V_j and LSE_i = m_i + ln(l_i) ("어텐션 최적화" Step 3;
     FlashAttention page "Recomputation 전략" for the saved m, l)."""
     S = head_scores(q_rows, K, scale, softcap, row_idx, mask_kind, window, doc_offsets,
-                    kv_idx=kv_idx)
+                    kv_idx=kv_idx, alibi_slope=alibi_slope)
     P, m, l = softmax_rows(S)
     O = P @ _f64(V)
     with np.errstate(divide="ignore"):
@@ -168,10 +183,11 @@ def attention_head(q_rows, row_idx, K, V, scale: float, mask_kind: int = MASK_NO
 
 
 def attention(q, k, v, scale=None, mask_kind: int = MASK_NONE, window: int = 0,
-              softcap: float = 0.0, doc_offsets=None, row_chunk: int = 256):
+              softcap: float = 0.0, doc_offsets=None, row_chunk: int = 256, alibi_slopes=None):
     """Full oracle: q [B,Hq,Nq,d], k/v [B,Hkv,Nk,d] (any real dtype) -> (O, LSE) in fp64.
 
-    O is [B,Hq,Nq,dv], LSE is [B,Hq,Nq].  Query head h reads KV head h // (Hq // Hkv)."""
+    O is [B,Hq,Nq,dv], LSE is [B,Hq,Nq].  Query head h reads KV head h // (Hq // Hkv);
+    ``alibi_slopes`` (length Hq, or None) gives head h the bias -slope_h * |q - kv|."""
     q = _f64(q)
     k = _f64(k)
     v = _f64(v)
@@ -193,13 +209,14 @@ def attention(q, k, v, scale=None, mask_kind: int = MASK_NONE, window: int = 0,
                 rows = np.arange(r0, min(Nq, r0 + row_chunk))
                 O[b, h, rows], lse[b, h, rows] = attention_head(
                     q[b, h, rows], rows, k[b, hk], v[b, hk], scale, mask_kind, window,
-                    softcap, doc_offsets)
+                    softcap, doc_offsets,
+                    alibi_slope=0.0 if alibi_slopes is None else float(alibi_slopes[h]))
     return O, lse
 
 
 def attention_tiled_online(q, k, v, scale=None, block_q: int = 2, block_kv: int = 3,
                            mask_kind: int = MASK_NONE, window: int = 0,
-                           softcap: float = 0.0, doc_offsets=None):
+                           softcap: float = 0.0, doc_offsets=None, alibi_slopes=None):
     """The blockwise online-softmax form of the FlashAttention page ("Online Softmax와 블록
     단위 누적", "알고리즘 의사코드"), kept in its normalised-O form.
 
@@ -232,7 +249,9 @@ def attention_tiled_online(q, k, v, scale=None, block_q: int = 2, block_kv: int 
                 for j0 in range(0, Nk, block_kv):
                     cols = np.arange(j0, min(Nk, j0 + block_kv))
                     S = head_scores(q[b, h, rows], k[b, hk, cols], scale, softcap, rows,
-                                    mask_kind, window, doc_offsets, kv_idx=cols)
+                                    mask_kind, window, doc_offsets, kv_idx=cols,
+                                    alibi_slope=0.0 if alibi_slopes is None
+                                    else float(alibi_slopes[h]))
                     m_loc = S.max(axis=1)
                     has = np.isfinite(m_loc)
                     P_loc = np.where(has[:, None],

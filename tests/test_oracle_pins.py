@@ -13,8 +13,8 @@ import pytest
 import torch
 
 import oracle
-from oracle import (MASK_CAUSAL, MASK_DOCUMENT_CAUSAL, MASK_NONE, MASK_SLIDING_CAUSAL,
-                    TILE_EMPTY, TILE_FULL, TILE_PARTIAL)
+from oracle import (MASK_CAUSAL, MASK_DOCUMENT_CAUSAL, MASK_NONE, MASK_SLIDING,
+                    MASK_SLIDING_CAUSAL, TILE_EMPTY, TILE_FULL, TILE_PARTIAL)
 import workloads
 from workloads import accounting
 
@@ -108,7 +108,7 @@ def _rand_qkv(B, Hq, Hkv, N, d, seed, std=1.0, Nk=None):
 
 DOCS_SMALL = np.array([0, 5, 6, 13, 20], dtype=np.int32)   # lengths 5, 1, 7, 7
 MASKS = [(MASK_NONE, 0, None), (MASK_CAUSAL, 0, None), (MASK_SLIDING_CAUSAL, 3, None),
-         (MASK_DOCUMENT_CAUSAL, 0, DOCS_SMALL)]
+         (MASK_DOCUMENT_CAUSAL, 0, DOCS_SMALL), (MASK_SLIDING, 3, None)]
 
 
 @pytest.mark.parametrize("mask_kind,window,docs", MASKS)
@@ -133,6 +133,8 @@ def _visible_counts_by_hand(N, mask_kind, window, docs):
             out.append(i + 1)
         elif mask_kind == MASK_SLIDING_CAUSAL:
             out.append(min(i, window) + 1)
+        elif mask_kind == MASK_SLIDING:
+            out.append(min(N - 1, i + window) - max(0, i - window) + 1)
         else:
             start = max(int(o) for o in docs if o <= i)
             out.append(i - start + 1)
@@ -153,6 +155,8 @@ def test_equal_scores_give_mean_of_visible_values(mask_kind, window, docs):
             lo, hi = 0, i + 1
         elif mask_kind == MASK_SLIDING_CAUSAL:
             lo, hi = max(0, i - window), i + 1
+        elif mask_kind == MASK_SLIDING:
+            lo, hi = max(0, i - window), min(N, i + window + 1)
         else:
             lo, hi = max(int(o) for o in docs if o <= i), i + 1
         assert hi - lo == counts[i]
@@ -180,6 +184,8 @@ def _torch_mask(N, mask_kind, window, docs):
         m = torch.tril(m)
     if mask_kind == MASK_SLIDING_CAUSAL:
         m = m & torch.triu(torch.ones(N, N, dtype=torch.bool), diagonal=-window)
+    if mask_kind == MASK_SLIDING:
+        m = torch.triu(m, diagonal=-window) & torch.tril(m, diagonal=window)
     if mask_kind == MASK_DOCUMENT_CAUSAL:
         blk = torch.zeros(N, N, dtype=torch.bool)
         for s, e in zip(docs[:-1], docs[1:]):
@@ -316,6 +322,8 @@ def _tile_class_by_intervals(i, j, N, bq, bk, mask_kind, window, docs):
             lo, hi = 0, qq
         elif mask_kind == MASK_SLIDING_CAUSAL:
             lo, hi = max(0, qq - window), qq
+        elif mask_kind == MASK_SLIDING:
+            lo, hi = max(0, qq - window), min(N - 1, qq + window)
         else:
             lo, hi = max(int(o) for o in docs if o <= qq), qq
         a, b = max(lo, k0), min(hi, k1 - 1)
@@ -358,7 +366,8 @@ def test_visible_pair_closed_forms_match_element_counts():
     docs = workloads.doc_offsets_for(3000, 100, 700, seed=3)
     for (kind, w, dd) in [(MASK_NONE, 0, None), (MASK_CAUSAL, 0, None),
                           (MASK_SLIDING_CAUSAL, 257, None), (MASK_SLIDING_CAUSAL, 5000, None),
-                          (MASK_DOCUMENT_CAUSAL, 0, docs)]:
+                          (MASK_DOCUMENT_CAUSAL, 0, docs), (MASK_SLIDING, 0, None),
+                          (MASK_SLIDING, 257, None), (MASK_SLIDING, 5000, None)]:
         assert accounting.visible_pairs(3000, 3000, kind, w, dd) == \
             oracle.visible_pairs(3000, 3000, kind, w, dd)
     assert accounting.visible_pairs(16384, 16384, MASK_SLIDING_CAUSAL, 1024) == 16268800
@@ -405,3 +414,79 @@ def test_useful_flops_of_the_prefill_workloads():
     docs = workloads.workload_doc_offsets(w)
     pairs = accounting.visible_pairs(w.Nq, w.Nk, w.mask_kind, 0, docs)
     assert pairs == sum(L * (L + 1) // 2 for L in workloads.doc_lengths(32768))
+
+
+# ------------------------------------------------------------------------ ALiBi bias
+
+def _alibi_weights(i, N, slope, mask_kind):
+    """Softmax weights of row i when every raw score is 0: exp(-slope * |i - j|) over the
+    visible keys, written out as the geometric sequence it is."""
+    js = np.arange(N)
+    if mask_kind == MASK_CAUSAL:
+        js = js[: i + 1]
+    return js, np.exp(-slope * np.abs(i - js).astype(np.float64))
+
+
+@pytest.mark.parametrize("mask_kind", [MASK_NONE, MASK_CAUSAL])
+def test_alibi_equal_scores_closed_form(mask_kind):
+    # Q = 0: the scores are the bias alone, so row i weighs key j by exp(-slope |i - j|).
+    # Causal: the log-sum-exp is the geometric sum ln((1 - r^(i+1)) / (1 - r)), r = e^-slope.
+    N, d = 24, 8
+    _, k, v = _rand_qkv(1, 2, 2, N, d, 11)
+    q = np.zeros((1, 2, N, d))
+    slopes = np.array([0.5, 0.0625])
+    O, lse = oracle.attention(q, k, v, mask_kind=mask_kind, alibi_slopes=slopes)
+    for h, slope in enumerate(slopes):
+        r = math.exp(-slope)
+        for i in range(N):
+            js, w = _alibi_weights(i, N, slope, mask_kind)
+            want = (w[:, None] * v[0, h, js]).sum(axis=0) / w.sum()
+            assert np.allclose(O[0, h, i], want, atol=1e-13, rtol=0)
+            if mask_kind == MASK_CAUSAL:
+                assert abs(lse[0, h, i] - math.log((1 - r ** (i + 1)) / (1 - r))) < 1e-13
+            else:
+                left = (1 - r ** (i + 1)) / (1 - r)          # j = i, i-1, ..., 0
+                right = r * (1 - r ** (N - 1 - i)) / (1 - r)   # j = i+1, ..., N-1
+                assert abs(lse[0, h, i] - math.log(left + right)) < 1e-13
+
+
+def test_alibi_zero_slopes_are_no_bias():
+    q, k, v = _rand_qkv(1, 3, 3, 17, 8, 12)
+    for kind, w in [(MASK_NONE, 0), (MASK_CAUSAL, 0), (MASK_SLIDING, 4)]:
+        O0, l0 = oracle.attention(q, k, v, mask_kind=kind, window=w)
+        O1, l1 = oracle.attention(q, k, v, mask_kind=kind, window=w, alibi_slopes=[0, 0, 0])
+        assert np.array_equal(O0, O1) and np.array_equal(l0, l1)
+
+
+@pytest.mark.parametrize("mask_kind,window,docs", MASKS)
+def test_alibi_matches_torch_sdpa_float64(mask_kind, window, docs):
+    # the bias enters torch's SDPA as an additive float mask (-inf where not visible)
+    B, Hq, Hkv, N, d = 2, 4, 2, 19, 16
+    q, k, v = _rand_qkv(B, Hq, Hkv, N, d, 13)
+    slopes = np.array([1.0, 0.5, 0.25, 0.125])
+    scale = 0.2
+    O, lse = oracle.attention(q, k, v, scale=scale, mask_kind=mask_kind, window=window,
+                              doc_offsets=docs, alibi_slopes=slopes)
+    tq, tk, tv = (torch.from_numpy(x) for x in (q, k, v))
+    tk = tk.repeat_interleave(Hq // Hkv, dim=1)
+    tv = tv.repeat_interleave(Hq // Hkv, dim=1)
+    idx = torch.arange(N, dtype=torch.float64)
+    dist = (idx[:, None] - idx[None, :]).abs()
+    bias = -torch.from_numpy(slopes)[:, None, None] * dist[None]
+    bias = bias.masked_fill(~_torch_mask(N, mask_kind, window, docs)[None], float("-inf"))
+    ref = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, attn_mask=bias[None],
+                                                           scale=scale)
+    assert np.allclose(O, ref.numpy(), atol=1e-12, rtol=0)
+    S = torch.einsum("bhid,bhjd->bhij", tq, tk) * scale + bias[None]
+    assert np.allclose(lse, torch.logsumexp(S, dim=-1).numpy(), atol=1e-12, rtol=0)
+
+
+@pytest.mark.parametrize("bq,bk", [(1, 1), (3, 5), (16, 16)])
+def test_alibi_tiled_online_equals_full(bq, bk):
+    q, k, v = _rand_qkv(1, 2, 1, 21, 8, 14)
+    slopes = [0.3, 2.0]
+    for kind, w in [(MASK_CAUSAL, 0), (MASK_SLIDING, 5)]:
+        O, l = oracle.attention(q, k, v, mask_kind=kind, window=w, alibi_slopes=slopes)
+        Ot, lt = oracle.attention_tiled_online(q, k, v, block_q=bq, block_kv=bk, mask_kind=kind,
+                                               window=w, alibi_slopes=slopes)
+        assert np.allclose(O, Ot, atol=1e-12, rtol=0) and np.allclose(l, lt, atol=1e-12, rtol=0)

@@ -20,6 +20,7 @@ MASK_NONE = 0
 MASK_CAUSAL = 1
 MASK_SLIDING_CAUSAL = 2
 MASK_DOCUMENT_CAUSAL = 3
+MASK_SLIDING = 4
 
 
 @dataclasses.dataclass(frozen=True)
@@ -62,7 +63,8 @@ class Workload:
 
 
 MASK_NAMES = {MASK_NONE: "none", MASK_CAUSAL: "causal",
-              MASK_SLIDING_CAUSAL: "sliding_causal", MASK_DOCUMENT_CAUSAL: "document_causal"}
+              MASK_SLIDING_CAUSAL: "sliding_causal", MASK_DOCUMENT_CAUSAL: "document_causal",
+              MASK_SLIDING: "sliding"}
 
 TINY = Workload("tiny_b1_h2_n128_d64", "prefill", 1, 2, 2, 128, 128, 64, seed=1001)
 TINY_CAUSAL = dataclasses.replace(TINY, name="tiny_b1_h2_n128_d64_causal",

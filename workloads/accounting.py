@@ -7,7 +7,7 @@ oracle's mask in the CPU tests.
 """
 from __future__ import annotations
 
-from . import MASK_CAUSAL, MASK_DOCUMENT_CAUSAL, MASK_NONE, MASK_SLIDING_CAUSAL
+from . import MASK_CAUSAL, MASK_DOCUMENT_CAUSAL, MASK_NONE, MASK_SLIDING, MASK_SLIDING_CAUSAL
 
 
 def visible_pairs(Nq: int, Nk: int, mask_kind: int, window: int = 0, doc_offsets=None) -> int:
@@ -20,6 +20,13 @@ def visible_pairs(Nq: int, Nk: int, mask_kind: int, window: int = 0, doc_offsets
     if mask_kind == MASK_SLIDING_CAUSAL:
         n1 = min(N, window)
         return n1 * (n1 + 1) // 2 + (N - n1) * (window + 1)
+    if mask_kind == MASK_SLIDING:
+        # row i sees [max(0, i - w), min(N - 1, i + w)]: N (2w + 1) minus the parts cut off
+        # at both ends, w - i keys for each of the first min(N, w) rows (and symmetrically)
+        w = window
+        n1 = min(N, w)
+        cut = n1 * w - n1 * (n1 - 1) // 2
+        return N * (2 * w + 1) - 2 * cut
     if mask_kind == MASK_DOCUMENT_CAUSAL:
         offs = [int(x) for x in doc_offsets]
         return sum((e - s) * (e - s + 1) // 2 for s, e in zip(offs[:-1], offs[1:]))
