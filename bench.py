@@ -325,6 +325,9 @@ def run_ours(args, world, rank, local):
         del q, k, v, o, lse
         torch.cuda.empty_cache()
         out["decode"] = bench_decode(args, world, local, peaks, peak_src)
+    if not args.no_extras and args.only == "all":
+        out["extras"] = {x.name: bench_prefill_variant(x, args, world, local, peaks, peak_src)
+                         for x in (workloads.ALIBI_MHA, workloads.SWA_SYM_GQA)}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         tf, heads, dt = oracle_prefill_sample(w, args.cpu_budget)
         out["cpu_baseline"] = {"value": round(tf, 5), "unit": "TFLOP/s",
@@ -332,6 +335,47 @@ def run_ours(args, world, rank, local):
                                "sample": f"{heads} whole heads (4096 query rows each, all keys) "
                                          f"of {w.name}, fp64, {dt:.1f} s"}
     return out
+
+
+def bench_prefill_variant(w, args, world, local, peaks, peak_src):
+    """Useful TFLOP/s of attn_fwd on another prefill workload (ALiBi, symmetric window):
+    the same timing as the headline, fewer steps."""
+    import torch
+    import io_aware_softmax_b200 as attn
+    dev = torch.device("cuda", torch.cuda.current_device())
+    q, k, v = workloads.make_inputs(w, device=dev)
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.Hq, w.Nq), dtype=torch.float32, device=dev)
+    slopes = (torch.tensor(workloads.alibi_slopes(w.Hq), dtype=torch.float32, device=dev)
+              if w.alibi else None)
+    flops = accounting.prefill_useful_flops(w.B, w.Hq, w.Nq, w.Nk, w.d, w.mask_kind, w.window)
+
+    def step():
+        attn.attn_fwd(q, k, v, scale=w.scale, mask=w.mask_kind, window=w.window,
+                      alibi_slopes=slopes, out=o, lse=lse)
+
+    steps = max(3, min(args.steps, 30))
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        total_ms, per = time_launches(step, steps, world)
+    if attn.device_status() != 0:
+        raise RuntimeError(f"device status not ok after {w.name}")
+    ms = max_over_ranks(world, total_ms / steps)
+    kernel_ms = max_over_ranks(world, sum(per) / len(per))
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    achieved = flops / (kernel_ms * 1e-3) / 1e12
+    res = {"config": w.describe(), "value": round(whole_job_rate(flops, world, ms) / 1e12, 2),
+           "unit": "TFLOP/s", "ms_per_step": round(ms, 4), "steps": steps,
+           "useful_tflop_per_step": round(flops / 1e12, 4),
+           "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak,
+                        "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                        "peak_source": f"bf16_tflops (burst, {peak_src})", "traffic": None},
+           "gpu_launches": steps, "clocks": clk.summary()}
+    del q, k, v, o, lse
+    torch.cuda.empty_cache()
+    return res
 
 
 def e2e_prefill(w, args, world, q, k, v):
@@ -477,6 +521,8 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-extras", action="store_true",
+                    help="skip the ALiBi and symmetric-window prefill lines")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle time")
     ap.add_argument("--only", choices=["all", "prefill", "decode"], default="all",

@@ -44,7 +44,8 @@ typedef enum {
   ATTN_MASK_NONE = 0,             /* every key visible                                    */
   ATTN_MASK_CAUSAL = 1,           /* kv <= q                                               */
   ATTN_MASK_SLIDING_CAUSAL = 2,   /* 0 <= q - kv <= window (window + 1 keys incl. self)    */
-  ATTN_MASK_DOCUMENT_CAUSAL = 3   /* same packed document AND kv <= q                      */
+  ATTN_MASK_DOCUMENT_CAUSAL = 3,  /* same packed document AND kv <= q                      */
+  ATTN_MASK_SLIDING = 4           /* |q - kv| <= window, no causality (2 window + 1 keys)  */
 } attn_mask_kind;
 
 typedef enum {
@@ -69,7 +70,7 @@ typedef enum { ATTN_TILE_EMPTY = 0, ATTN_TILE_PARTIAL = 1, ATTN_TILE_FULL = 2 } 
  *   o        bf16 [B, Hq,  Nq, d]     (written)   lse  fp32 [B, Hq, Nq] natural log (written)
  *   d        64 or 128; Hq % Hkv == 0; query head h reads KV head h / (Hq / Hkv)
  *   scale    multiplies q.k; <= 0 selects 1/sqrt(d)
- *   mask_kind, window   see attn_mask_kind; window >= 0 for SLIDING_CAUSAL
+ *   mask_kind, window   see attn_mask_kind; window >= 0 for SLIDING_CAUSAL and SLIDING
  *   softcap  > 0: score s (already scaled) becomes softcap * tanh(s / softcap); <= 0: off
  *   doc_offsets, num_docs   DOCUMENT_CAUSAL only: device int32 [num_docs + 1], with
  *            doc_offsets[0] = 0, non-decreasing, doc_offsets[num_docs] = Nk; the same
@@ -81,6 +82,20 @@ typedef enum { ATTN_TILE_EMPTY = 0, ATTN_TILE_PARTIAL = 1, ATTN_TILE_FULL = 2 } 
 ATTN_API int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
              int Hkv, int Nq, int Nk, int d, float scale, int mask_kind, int window,
              float softcap, const int* doc_offsets, int num_docs, cudaStream_t stream);
+
+/*
+ * attn_fwd_alibi -- attn_fwd with the ALiBi positional bias fused into the score
+ * ("3.7 어텐션 II", 3.7.5: a distance-based bias added before the softmax, fused instead of
+ * passed as a mask tensor).  Query head h adds -alibi_slopes[h] * |q - kv| (natural-log
+ * units) to the score after scaling and soft-capping and before the mask.
+ *   alibi_slopes  device fp32 [Hq], 4-byte aligned, read by the kernel; NULL behaves as
+ *                 attn_fwd.  Every other argument, the outputs and the errors as attn_fwd,
+ *                 plus UNSUPPORTED for a bias together with softcap > 0.
+ */
+ATTN_API int attn_fwd_alibi(const void* q, const void* k, const void* v, void* o, float* lse,
+             int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int mask_kind,
+             int window, float softcap, const int* doc_offsets, int num_docs,
+             const float* alibi_slopes, cudaStream_t stream);
 
 /*
  * attn_blockmap -- 128x128 block-sparsity map of a mask ("PyTorch FlexAttention 도입 분석",

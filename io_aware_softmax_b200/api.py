@@ -10,7 +10,7 @@ import torch
 
 from . import _lib
 
-MASKS = {"none": 0, "causal": 1, "sliding_causal": 2, "document_causal": 3}
+MASKS = {"none": 0, "causal": 1, "sliding_causal": 2, "document_causal": 3, "sliding": 4}
 
 ATTN_OK = 0
 
@@ -59,9 +59,13 @@ def _need(t: torch.Tensor, name: str, dtype: torch.dtype, dims: int):
 
 def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, scale: Optional[float] = None,
              mask="none", window: int = 0, softcap: float = 0.0,
-             doc_offsets: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
-             lse: Optional[torch.Tensor] = None, stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
-    """Fused prefill attention: q [B,Hq,Nq,d], k/v [B,Hkv,Nk,d] bf16 -> (O bf16, LSE fp32)."""
+             doc_offsets: Optional[torch.Tensor] = None, alibi_slopes: Optional[torch.Tensor] = None,
+             out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+             stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Fused prefill attention: q [B,Hq,Nq,d], k/v [B,Hkv,Nk,d] bf16 -> (O bf16, LSE fp32).
+
+    ``alibi_slopes`` (fp32 [Hq] on the device) adds -slope_h * |q - kv| to the scores of
+    query head h (attn_fwd_alibi)."""
     lib = _lib.load()
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _need(t, n, torch.bfloat16, 4)
@@ -75,10 +79,21 @@ def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, scale: Option
     if doc_offsets is not None:
         _need(doc_offsets, "doc_offsets", torch.int32, 1)
         num_docs = doc_offsets.numel() - 1
-    st = lib.attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, Nq, Nk, d,
-                      float(scale or 0.0), _mask_id(mask), int(window), float(softcap or 0.0),
-                      _ptr(doc_offsets), num_docs, _stream(q.device, stream))
-    _check(st, "attn_fwd")
+    if alibi_slopes is None:
+        st = lib.attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, Nq, Nk, d,
+                          float(scale or 0.0), _mask_id(mask), int(window),
+                          float(softcap or 0.0), _ptr(doc_offsets), num_docs,
+                          _stream(q.device, stream))
+        _check(st, "attn_fwd")
+    else:
+        _need(alibi_slopes, "alibi_slopes", torch.float32, 1)
+        if alibi_slopes.numel() != Hq:
+            raise ValueError(f"alibi_slopes must hold Hq={Hq} slopes")
+        st = lib.attn_fwd_alibi(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, Nq,
+                                Nk, d, float(scale or 0.0), _mask_id(mask), int(window),
+                                float(softcap or 0.0), _ptr(doc_offsets), num_docs,
+                                _ptr(alibi_slopes), _stream(q.device, stream))
+        _check(st, "attn_fwd_alibi")
     return out, lse
 
 

@@ -55,10 +55,10 @@ bool make_map_3d(CUtensorMap* map, const void* ptr, int d, long long rows, long 
 }
 
 int check_mask(int mask_kind, int window, const int* doc_offsets, int num_docs, int Nq, int Nk) {
-  if (mask_kind < ATTN_MASK_NONE || mask_kind > ATTN_MASK_DOCUMENT_CAUSAL)
-    return ATTN_ERR_INVALID_ARG;
+  if (mask_kind < ATTN_MASK_NONE || mask_kind > ATTN_MASK_SLIDING) return ATTN_ERR_INVALID_ARG;
   if (mask_kind != ATTN_MASK_NONE && Nq != Nk) return ATTN_ERR_UNSUPPORTED;
-  if (mask_kind == ATTN_MASK_SLIDING_CAUSAL && window < 0) return ATTN_ERR_INVALID_ARG;
+  if ((mask_kind == ATTN_MASK_SLIDING_CAUSAL || mask_kind == ATTN_MASK_SLIDING) && window < 0)
+    return ATTN_ERR_INVALID_ARG;
   if (mask_kind == ATTN_MASK_DOCUMENT_CAUSAL) {
     if (doc_offsets == nullptr || num_docs < 1) return ATTN_ERR_INVALID_ARG;
     if (reinterpret_cast<uintptr_t>(doc_offsets) & 3u) return ATTN_ERR_MISALIGNED;
@@ -132,6 +132,14 @@ extern "C" int attn_fwd(const void* q, const void* k, const void* v, void* o, fl
                         int Hq, int Hkv, int Nq, int Nk, int d, float scale, int mask_kind,
                         int window, float softcap, const int* doc_offsets, int num_docs,
                         cudaStream_t stream) {
+  return attn_fwd_alibi(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, scale, mask_kind, window, softcap,
+                        doc_offsets, num_docs, nullptr, stream);
+}
+
+extern "C" int attn_fwd_alibi(const void* q, const void* k, const void* v, void* o, float* lse,
+                              int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale,
+                              int mask_kind, int window, float softcap, const int* doc_offsets,
+                              int num_docs, const float* alibi_slopes, cudaStream_t stream) {
   if (B < 0 || Hq < 0 || Hkv < 0 || Nq < 0 || Nk < 0) return ATTN_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
   if (Hkv == 0 && Hq > 0) return ATTN_ERR_INVALID_ARG;
@@ -139,6 +147,8 @@ extern "C" int attn_fwd(const void* q, const void* k, const void* v, void* o, fl
   int st = check_mask(mask_kind, window, doc_offsets, num_docs, Nq, Nk);
   if (st != ATTN_OK) return st;
   if (std::isnan(scale) || std::isnan(softcap)) return ATTN_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(alibi_slopes) & 3u) return ATTN_ERR_MISALIGNED;
+  if (alibi_slopes != nullptr && softcap > 0.f) return ATTN_ERR_UNSUPPORTED;
   if (B == 0 || Hq == 0 || Nq == 0) return ATTN_OK;
   if (o == nullptr || lse == nullptr || q == nullptr) return ATTN_ERR_INVALID_ARG;
   if (!aligned16(o) || !aligned16(lse) || !aligned16(q)) return ATTN_ERR_MISALIGNED;
@@ -165,6 +175,7 @@ extern "C" int attn_fwd(const void* q, const void* k, const void* v, void* o, fl
   p.cap_scale = softcap > 0.f ? scale / softcap : 0.f;
   p.cap_log2 = softcap > 0.f ? softcap * kLog2e : 0.f;
   p.mask = mask_params(mask_kind, window, doc_offsets, num_docs, Nq, Nk);
+  p.alibi = alibi_slopes;
   if ((long long)p.num_pairs * B * Hq > (1LL << 31) - 1) return ATTN_ERR_UNSUPPORTED;
   p.err = error_word_ptr(current_device());
   if (p.err == nullptr) return ATTN_ERR_CUDA;

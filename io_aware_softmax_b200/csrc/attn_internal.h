@@ -22,6 +22,7 @@ struct FwdParams {
   float cap_scale;    // scale / softcap
   float cap_log2;     // softcap * log2(e)
   MaskParams mask;
+  const float* alibi; // fp32 [Hq] ALiBi slopes (natural-log units per key of distance) or null
   uint32_t* err;      // device error word of the library (bits, first site)
 };
 

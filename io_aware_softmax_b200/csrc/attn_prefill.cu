@@ -54,6 +54,7 @@ constexpr uint32_t kRegsOther = 112;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units: rescale when max grows > 2^8
 constexpr float kLn2 = 0.69314718055994531f;
+constexpr float kLog2eF = 1.44269504088896341f;
 constexpr uint32_t kNegInfBits = 0xff800000u;
 
 template <int D>
@@ -108,18 +109,40 @@ __device__ __forceinline__ float scaled_score(float s, const FwdParams& p) {
   return p.cap_log2 * tanh_via_ex2(s * p.cap_scale);
 }
 
+// Masked columns (outside [c_lo, c_hi]) of one tile row become -inf.
+__device__ __forceinline__ void mask_row(uint32_t (&s)[128], int c_lo, int c_hi) {
+#pragma unroll
+  for (int c = 0; c < 128; ++c)
+    if ((unsigned)(c - c_lo) > (unsigned)(c_hi - c_lo)) s[c] = kNegInfBits;
+}
+
+// ALiBi: the row's scores become base-2 biased scores in place,
+// scale * s * log2(e) - slope2 * |drow - c| with drow the row's offset from the tile's first
+// key and slope2 the head's slope times log2(e); -inf (masked) stays -inf.
+__device__ __forceinline__ void alibi_row(uint32_t (&s)[128], const FwdParams& p, float slope2,
+                                          float drow) {
+#pragma unroll
+  for (int c = 0; c < 128; c += 2) {
+    const float d0 = fabsf(drow - (float)c), d1 = fabsf(drow - (float)(c + 1));
+    float t0, t1;
+    ffma2(t0, t1, f32(s[c]), f32(s[c + 1]), p.kscale, p.kscale, -slope2 * d0, -slope2 * d1);
+    s[c] = __float_as_uint(t0);
+    s[c + 1] = __float_as_uint(t1);
+  }
+}
+
 // P = 2^(x - m_use) for one 64-column half of a tile row, packed as bf16 pairs; returns
 // the half's fp32 sum (four independent packed accumulators).
 template <bool kSoftcap>
 __device__ __forceinline__ float tile_row_exp_half(const uint32_t (&s)[128], int base,
-                                                   const FwdParams& p, float m_use,
+                                                   const FwdParams& p, float ks, float m_use,
                                                    uint32_t (&pk)[32]) {
   float a0 = 0.f, a1 = 0.f, b0 = 0.f, b1 = 0.f, c0 = 0.f, c1 = 0.f, d0 = 0.f, d1 = 0.f;
 #pragma unroll
   for (int c = 0; c < 64; c += 2) {
     float x0, x1;
     if (!kSoftcap) {
-      ffma2(x0, x1, f32(s[base + c]), f32(s[base + c + 1]), p.kscale, p.kscale, -m_use, -m_use);
+      ffma2(x0, x1, f32(s[base + c]), f32(s[base + c + 1]), ks, ks, -m_use, -m_use);
     } else {
       x0 = scaled_score<true>(f32(s[base + c]), p) - m_use;
       x1 = scaled_score<true>(f32(s[base + c + 1]), p) - m_use;
@@ -203,7 +226,7 @@ __device__ __forceinline__ void for_each_pair(const FwdParams& p, F&& f) {
   }
 }
 
-template <int D>
+template <int D, bool kAlibi>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
                       const __grid_constant__ CUtensorMap tmK,
@@ -452,6 +475,8 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
       const int row = tq0 + r;
       int row_lo, row_hi;
       row_interval(p.mask, row, row_lo, row_hi);
+      // ALiBi slope of this head in base-2 units (0: no bias).
+      const float slope2 = kAlibi ? __ldg(p.alibi + w.h) * kLog2eF : 0.f;
       // Tile-level bounds: a K/V tile needs no mask when every valid row of this query
       // tile sees every key of it and it lies inside Nk.
       int lo_last = 0, hi_first = 0;
@@ -474,10 +499,19 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
         const int k0 = (w.jt0 + rng.a + i) * kBN;
         const bool masked =
             !(lo_last <= k0 && k0 + kBN - 1 <= hi_first && k0 + kBN <= p.Nk);
-        const float mx_raw = masked ? tile_row_max<true>(s, row_lo - k0, row_hi - k0)
-                                    : tile_row_max<false>(s, 0, 0);
-        const float mx = (p.softcap > 0.f) ? scaled_score<true>(mx_raw, p)
-                                           : scaled_score<false>(mx_raw, p);
+        float mx;
+        if constexpr (!kAlibi) {
+          const float mx_raw = masked ? tile_row_max<true>(s, row_lo - k0, row_hi - k0)
+                                      : tile_row_max<false>(s, 0, 0);
+          mx = (p.softcap > 0.f) ? scaled_score<true>(mx_raw, p)
+                                 : scaled_score<false>(mx_raw, p);
+        } else {
+          // The bias changes the order of the scores, so the row max is taken over the
+          // biased, base-2 scores themselves.
+          if (masked) mask_row(s, row_lo - k0, row_hi - k0);
+          alibi_row(s, p, slope2, (float)(row - k0));   // no soft-cap with ALiBi
+          mx = tile_row_max<false>(s, 0, 0);
+        }
         const float m_new = fmaxf(m_ref, mx);
         const bool need = m_new > m_ref + kRescaleThreshold;
         float alpha = 1.f;
@@ -506,10 +540,12 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
           uint32_t pk[32];
-          if (p.softcap > 0.f) {
-            sum += tile_row_exp_half<true>(s, 64 * half, p, m_use, pk);
+          if constexpr (kAlibi) {
+            sum += tile_row_exp_half<false>(s, 64 * half, p, 1.f, m_use, pk);
+          } else if (p.softcap > 0.f) {
+            sum += tile_row_exp_half<true>(s, 64 * half, p, p.kscale, m_use, pk);
           } else {
-            sum += tile_row_exp_half<false>(s, 64 * half, p, m_use, pk);
+            sum += tile_row_exp_half<false>(s, 64 * half, p, p.kscale, m_use, pk);
           }
           tmem_st_x32(tP + 32u * half, pk);
           tmem_wait_st();
@@ -570,18 +606,19 @@ __global__ void attn_fill_empty_kernel(__nv_bfloat16* o, float* lse, size_t rows
   if (i < rows) lse[i] = -INFINITY;
 }
 
-template <int D>
+template <int D, bool kAlibi>
 int launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                const FwdParams& p, cudaStream_t stream) {
   using C = Cfg<D>;
   static_assert(C::kSmemBytes <= 227 * 1024, "shared memory budget");
-  cudaError_t e = cudaFuncSetAttribute(attn_fwd_sm100_kernel<D>,
+  cudaError_t e = cudaFuncSetAttribute(attn_fwd_sm100_kernel<D, kAlibi>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        C::kSmemBytes);
   if (e != cudaSuccess) return -4;
   const long long units = (long long)((p.num_pairs + 1) / 2) * p.B * p.Hq;
   const long long grid = units < p.num_sms ? units : p.num_sms;
-  attn_fwd_sm100_kernel<D><<<(unsigned)grid, kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, p);
+  attn_fwd_sm100_kernel<D, kAlibi>
+      <<<(unsigned)grid, kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, p);
   return cudaGetLastError() == cudaSuccess ? 0 : -4;
 }
 
@@ -589,8 +626,11 @@ int launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& 
 
 int launch_attn_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                     const FwdParams& p, int d, cudaStream_t stream) {
-  if (d == 128) return launch_fwd<128>(tq, tk, tv, p, stream);
-  if (d == 64) return launch_fwd<64>(tq, tk, tv, p, stream);
+  const bool alibi = p.alibi != nullptr;
+  if (d == 128) return alibi ? launch_fwd<128, true>(tq, tk, tv, p, stream)
+                             : launch_fwd<128, false>(tq, tk, tv, p, stream);
+  if (d == 64) return alibi ? launch_fwd<64, true>(tq, tk, tv, p, stream)
+                            : launch_fwd<64, false>(tq, tk, tv, p, stream);
   return -2;
 }
 

@@ -6,6 +6,7 @@
 //   causal            [0, q]                       key <= query, diagonal visible
 //   sliding + causal  [max(0, q - window), q]      |q - kv| <= window and kv <= q
 //   document + causal [start of q's document, q]   same packed sequence and kv <= q
+//   sliding           [max(0, q - window), q + window]   |q - kv| <= window, no causality
 // (score_mod/mask hooks of "PyTorch FlexAttention 도입 분석", section 2, with the
 // sliding_window_mod example; document boundaries as the cu_seqlens of "3.7 어텐션 II",
 // section 3.7.6; causal masking as in "Attention 최적화가 어려운 이유", "Attention의 계산
@@ -18,7 +19,9 @@
 
 namespace attn {
 
-enum MaskKind : int { kMaskNone = 0, kMaskCausal = 1, kMaskSlidingCausal = 2, kMaskDocCausal = 3 };
+enum MaskKind : int {
+  kMaskNone = 0, kMaskCausal = 1, kMaskSlidingCausal = 2, kMaskDocCausal = 3, kMaskSliding = 4
+};
 enum TileClass : uint8_t { kTileEmpty = 0, kTilePartial = 1, kTileFull = 2 };
 
 struct MaskParams {
@@ -55,6 +58,10 @@ __device__ __forceinline__ void row_interval(const MaskParams& m, int q, int& lo
       lo = doc_start(m.doc_offsets, m.num_docs, q);
       hi = min(q, last);
       break;
+    case kMaskSliding:
+      lo = max(0, q - m.window);
+      hi = (int)min((long long)q + m.window, (long long)last);
+      break;
     default:
       lo = 0;
       hi = last;
@@ -70,7 +77,9 @@ __device__ __forceinline__ int classify_tile(const MaskParams& m, int q0, int q1
   row_interval(m, q1 - 1, lo_l, hi_l);
   if (lo_l <= k0 && k1 - 1 <= hi_f) return kTileFull;
   // The row with the smallest lo whose interval reaches k0 is the first row with hi >= k0.
-  const int first = (m.kind == kMaskNone) ? q0 : max(q0, k0);
+  const int first = (m.kind == kMaskNone) ? q0
+                    : (m.kind == kMaskSliding) ? (int)max((long long)q0, (long long)k0 - m.window)
+                                               : max(q0, k0);
   if (first >= q1) return kTileEmpty;
   int lo, hi;
   row_interval(m, first, lo, hi);

@@ -94,6 +94,9 @@ def test_validation_happens_before_any_launch(lib):
     assert f(P, P, P, P, P, 1, 2, 2, 8, 9, 64, 0.0, 1, 0, 0.0, None, 0, None) == -2
     # unknown mask kind, negative window, document mask without offsets
     assert f(P, P, P, P, P, 1, 2, 2, 8, 8, 64, 0.0, 7, 0, 0.0, None, 0, None) == -1
+    assert f(P, P, P, P, P, 1, 2, 2, 8, 8, 64, 0.0, 5, 0, 0.0, None, 0, None) == -1
+    assert f(P, P, P, P, P, 1, 2, 2, 8, 8, 64, 0.0, 4, -1, 0.0, None, 0, None) == -1
+    assert f(P, P, P, P, P, 1, 2, 2, 8, 9, 64, 0.0, 4, 3, 0.0, None, 0, None) == -2
     assert f(P, P, P, P, P, 1, 2, 2, 8, 8, 64, 0.0, 2, -1, 0.0, None, 0, None) == -1
     assert f(P, P, P, P, P, 1, 2, 2, 8, 8, 64, 0.0, 3, 0, 0.0, None, 0, None) == -1
     # negative sizes
@@ -127,6 +130,7 @@ def test_blockmap_validation(lib):
     b = lib.attn_blockmap
     assert b(1, 8, 9, 1, 0, None, 0, ctypes.c_void_p(16), None) == -2
     assert b(1, 8, 8, 3, 0, None, 0, ctypes.c_void_p(16), None) == -1
+    assert b(1, 8, 8, 4, -2, None, 0, ctypes.c_void_p(16), None) == -1
     assert b(0, 8, 8, 1, 0, None, 0, None, None) == 0
 
 
@@ -139,3 +143,16 @@ def test_default_split_heuristic(lib):
     assert items / (waves * slots) >= 0.99 and 32768 // s >= 128
     assert lib.attn_decode_default_splits(1, 1, 100, 0) == 1
     assert lib.attn_decode_default_splits(1, 1, 0, 0) == 1
+
+
+def test_alibi_entry_validation(lib):
+    a = lib.attn_fwd_alibi
+    P = ctypes.c_void_p(16)
+    # slopes must be 4-byte aligned; a bias with a soft-cap is not supported
+    assert a(P, P, P, P, P, 1, 2, 2, 8, 8, 64, 0.0, 1, 0, 0.0, None, 0, ctypes.c_void_p(18),
+             None) == -3
+    assert a(P, P, P, P, P, 1, 2, 2, 8, 8, 64, 0.0, 1, 0, 30.0, None, 0, P, None) == -2
+    # the shared checks still come first, and empty problems are a no-op
+    assert a(P, P, P, P, P, 1, 2, 2, 8, 8, 96, 0.0, 1, 0, 0.0, None, 0, P, None) == -2
+    assert a(None, None, None, None, None, 0, 2, 2, 8, 8, 64, 0.0, 1, 0, 0.0, None, 0, P,
+             None) == 0

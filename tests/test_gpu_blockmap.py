@@ -35,6 +35,11 @@ def test_sliding(window):
     _check(1, 1500, 2, window=window)
 
 
+@pytest.mark.parametrize("window", [0, 1, 127, 128, 300, 2000])
+def test_symmetric_sliding(window):
+    _check(2, 1500, 4, window=window)
+
+
 def test_documents_random():
     for seed in range(4):
         docs = workloads.doc_offsets_for(3000, 1, 700, seed=seed)

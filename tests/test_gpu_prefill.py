@@ -12,7 +12,7 @@ from tests.gpu_common import compare, f64, sample_rows
 
 pytestmark = pytest.mark.gpu
 
-MASK_ID = {"none": 0, "causal": 1, "sliding_causal": 2, "document_causal": 3}
+MASK_ID = {"none": 0, "causal": 1, "sliding_causal": 2, "document_causal": 3, "sliding": 4}
 
 
 def _inputs(B, Hq, Hkv, Nq, Nk, d, seed, std=1.0):
@@ -23,7 +23,7 @@ def _inputs(B, Hq, Hkv, Nq, Nk, d, seed, std=1.0):
 
 
 def _run_full(B, Hq, Hkv, Nq, Nk, d, mask="none", window=0, softcap=0.0, docs=None, seed=0,
-              std=1.0, scale=None):
+              std=1.0, scale=None, slopes=None):
     q, k, v = _inputs(B, Hq, Hkv, Nq, Nk, d, seed, std)
     doc_t = None if docs is None else torch.tensor(docs, dtype=torch.int32, device="cuda")
     # guard bands around the outputs catch writes past the last row
@@ -31,14 +31,17 @@ def _run_full(B, Hq, Hkv, Nq, Nk, d, mask="none", window=0, softcap=0.0, docs=No
     l_buf = torch.full((B * Hq * Nq + 1024,), float("nan"), dtype=torch.float32, device="cuda")
     o = o_buf[: B * Hq * Nq * d].view(B, Hq, Nq, d)
     lse = l_buf[: B * Hq * Nq].view(B, Hq, Nq)
+    slopes_t = None if slopes is None else torch.tensor(slopes, dtype=torch.float32, device="cuda")
     attn_fwd(q, k, v, scale=scale, mask=mask, window=window, softcap=softcap, doc_offsets=doc_t,
-             out=o, lse=lse)
+             alibi_slopes=slopes_t, out=o, lse=lse)
     assert device_status() == 0
     assert torch.isnan(o_buf[B * Hq * Nq * d:]).all() and torch.isnan(l_buf[B * Hq * Nq:]).all()
     O_ref, L_ref = oracle.attention(f64(q), f64(k), f64(v), scale=scale, mask_kind=MASK_ID[mask],
-                                    window=window, softcap=softcap, doc_offsets=docs)
+                                    window=window, softcap=softcap, doc_offsets=docs,
+                                    alibi_slopes=slopes)
     vmax = float(v.abs().max()) if std > 1.0 else None
-    return compare(o, lse, O_ref, L_ref, f"{B}x{Hq}/{Hkv}x{Nq}x{Nk}x{d} {mask} w{window} c{softcap}",
+    return compare(o, lse, O_ref, L_ref,
+                   f"{B}x{Hq}/{Hkv}x{Nq}x{Nk}x{d} {mask} w{window} c{softcap} alibi{slopes}",
                    vmax=vmax)
 
 
@@ -159,3 +162,57 @@ def test_repeated_calls_are_deterministic():
     o2, l2 = attn_fwd(q, k, v, mask="causal")
     assert device_status() == 0
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+@pytest.mark.parametrize("window", [0, 1, 63, 127, 128, 129, 300, 2000])
+@pytest.mark.parametrize("N", [129, 777])
+def test_symmetric_sliding_window(window, N):
+    _run_full(1, 2, 1, N, N, 128, mask="sliding", window=window, seed=window + N)
+
+
+def test_symmetric_sliding_window_d64_gqa():
+    _run_full(2, 6, 2, 513, 513, 64, mask="sliding", window=200, seed=5)
+
+
+def _alibi_slopes(H):
+    # the usual geometric ALiBi slopes 2^(-8 (h + 1) / H)
+    return [2.0 ** (-8.0 * (h + 1) / H) for h in range(H)]
+
+
+@pytest.mark.parametrize("mask,window", [("none", 0), ("causal", 0), ("sliding_causal", 100),
+                                         ("sliding", 100), ("document_causal", 0)])
+@pytest.mark.parametrize("d", [64, 128])
+def test_alibi_bias(mask, window, d):
+    docs = [0, 130, 131, 400, 700] if mask == "document_causal" else None
+    _run_full(1, 4, 2, 700, 700, d, mask=mask, window=window, docs=docs, seed=7,
+              slopes=_alibi_slopes(4))
+
+
+@pytest.mark.parametrize("N", [1, 127, 128, 129, 257])
+def test_alibi_ragged_and_steep_slopes(N):
+    # slope 4: each step back in distance divides the weight by e^4; slope 0 is plain attention
+    _run_full(1, 3, 3, N, N, 128, mask="causal", seed=N, slopes=[4.0, 0.0, 0.03125])
+    _run_full(1, 2, 1, N, N, 128, mask="none", seed=N + 1, slopes=[1.0, 0.001])
+
+
+def test_alibi_full_size_sampled():
+    # causal MHA workload shapes (B=8, H=32, N=4096, d=128) with geometric slopes, sampled rows
+    w = workloads.CAUSAL_MHA
+    q, k, v = workloads.make_inputs(w, device="cuda")
+    slopes = torch.tensor(_alibi_slopes(w.Hq), dtype=torch.float32, device="cuda")
+    o, lse = attn_fwd(q, k, v, scale=w.scale, mask="causal", alibi_slopes=slopes)
+    assert device_status() == 0
+    rng = np.random.default_rng(5)
+    for b, h in [(0, 0), (7, 31), (3, 17)]:
+        rows = sample_rows(w.Nq, rng, 24)
+        O_ref, L_ref = oracle.attention_head(f64(q[b, h, rows]), rows, f64(k[b, h]), f64(v[b, h]),
+                                             w.scale, 1, alibi_slope=float(slopes[h]))
+        compare(o[b, h, rows], lse[b, h, rows], O_ref, L_ref, f"alibi full b{b} h{h}")
+
+
+def test_alibi_with_softcap_is_unsupported():
+    q, k, v = _inputs(1, 2, 2, 64, 64, 128, 1)
+    slopes = torch.tensor([0.5, 0.25], dtype=torch.float32, device="cuda")
+    with pytest.raises(Exception) as e:
+        attn_fwd(q, k, v, mask="causal", softcap=30.0, alibi_slopes=slopes)
+    assert "unsupported" in str(e.value).lower()

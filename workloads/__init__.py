@@ -41,6 +41,7 @@ class Workload:
     doc_len_lo: int = 512
     doc_len_hi: int = 4096
     doc_seed: int = 0
+    alibi: bool = False       # geometric ALiBi slopes 2^(-8 (h + 1) / Hq)
     seed: int = 0
 
     @property
@@ -54,6 +55,8 @@ class Workload:
             out["window"] = self.window
         if self.softcap:
             out["softcap"] = self.softcap
+        if self.alibi:
+            out["alibi_slopes"] = "2^(-8 (h + 1) / Hq)"
         if self.docs:
             out["doc_len_range"] = [self.doc_len_lo, self.doc_len_hi]
             out["doc_seed"] = self.doc_seed
@@ -78,8 +81,19 @@ DOC_SOFTCAP = Workload("doc_softcap_b1_h16_n32768_d128", "prefill", 1, 16, 16, 3
                        docs=True, seed=1004)
 DECODE = Workload("decode_b64_hq32_hkv8_t32768_d128", "decode", 64, 32, 8, 1, 32768, 128,
                   seed=1005)
+# Widening rows: the ALiBi bias on the causal MHA shapes, and the symmetric (non-causal)
+# window on the sliding-window GQA shapes.
+ALIBI_MHA = dataclasses.replace(CAUSAL_MHA, name="alibi_causal_mha_b8_h32_n4096_d128",
+                                alibi=True, seed=1006)
+SWA_SYM_GQA = dataclasses.replace(SWA_GQA, name="swa_sym_gqa_b4_hq32_hkv8_n16384_w1024_d128",
+                                  mask_kind=MASK_SLIDING, seed=1007)
 
-ALL = [TINY, TINY_CAUSAL, CAUSAL_MHA, SWA_GQA, DOC_SOFTCAP, DECODE]
+
+def alibi_slopes(H: int):
+    """The geometric ALiBi slopes 2^(-8 (h + 1) / H), one per query head."""
+    return [2.0 ** (-8.0 * (h + 1) / H) for h in range(H)]
+
+ALL = [TINY, TINY_CAUSAL, CAUSAL_MHA, SWA_GQA, DOC_SOFTCAP, DECODE, ALIBI_MHA, SWA_SYM_GQA]
 BY_NAME = {w.name: w for w in ALL}
 
 
