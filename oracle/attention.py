@@ -38,6 +38,9 @@ What it computes, and where that is written down (pages cited by title and secti
   누적" and "알고리즘 의사코드".
 * Split-KV decoding: each split produces partial (m, l, O) and the splits are combined by
   the same rescaling recurrence: "3.7 어텐션 II", section 3.7.4 (FlashDecoding).
+* Paged, variable-length KV caches for decode (in-flight batching with a page table,
+  PagedAttention): "3.7 어텐션 II", sections 3.7.4 and 3.7.8; the sequences of a batch have
+  their own lengths, as in the varlen API of section 3.7.6.
 
 Readings taken where the pages are silent (each is listed in the design doc as well):
 
@@ -330,6 +333,45 @@ def decode_splitkv(q, k_cache, v_cache, num_splits: int, scale=None):
                 lse_parts[b, h, :, s] = l
     O, lse = merge_partials(o_parts, lse_parts)
     return O, lse, o_parts, lse_parts
+
+
+def gather_paged(pages, block_table_row, length: int):
+    """The first ``length`` cache rows of one sequence from a paged cache: pages
+    [num_pages, Hkv, page_size, d], the sequence's logical page j is physical page
+    block_table_row[j] (PagedAttention's page table, "3.7 어텐션 II", 3.7.4 and 3.7.8).
+    Returns [Hkv, length, d]."""
+    pages = _f64(pages)
+    page_size = pages.shape[2]
+    n = -(-length // page_size) if length > 0 else 0
+    if n == 0:
+        return np.zeros((pages.shape[1], 0, pages.shape[3]))
+    rows = np.concatenate([pages[int(block_table_row[j])] for j in range(n)], axis=1)
+    return rows[:, :length]
+
+
+def decode_paged(q, k_pages, v_pages, block_table, seq_lens, scale=None):
+    """Decode attention over paged, variable-length caches: query row (b, h) attends to
+    the seq_lens[b] cache rows of sequence b gathered through its page table (plain
+    definition on the gathered keys; every key visible).  q [B,Hq,1,d].
+    Returns (O [B,Hq,1,dv], LSE [B,Hq,1]); a sequence of length 0 gives O = 0, LSE = -inf."""
+    q = _f64(q)
+    B, Hq, Nq, d = q.shape
+    Hkv = np.asarray(k_pages).shape[1]
+    G = Hq // Hkv
+    if scale is None or scale <= 0:
+        scale = default_scale(d)
+    O = np.zeros((B, Hq, Nq, np.asarray(v_pages).shape[3]))
+    lse = np.full((B, Hq, Nq), -np.inf)
+    for b in range(B):
+        T = int(seq_lens[b])
+        if T == 0:
+            continue
+        K = gather_paged(k_pages, block_table[b], T)
+        V = gather_paged(v_pages, block_table[b], T)
+        for h in range(Hq):
+            O[b, h], lse[b, h] = attention_head(q[b, h], np.arange(Nq), K[h // G], V[h // G],
+                                                scale)
+    return O, lse
 
 
 def tile_map(B: int, Nq: int, Nk: int, mask_kind: int, window: int = 0, doc_offsets=None,

@@ -490,3 +490,78 @@ def test_alibi_tiled_online_equals_full(bq, bk):
         Ot, lt = oracle.attention_tiled_online(q, k, v, block_q=bq, block_kv=bk, mask_kind=kind,
                                                window=w, alibi_slopes=slopes)
         assert np.allclose(O, Ot, atol=1e-12, rtol=0) and np.allclose(l, lt, atol=1e-12, rtol=0)
+
+
+# ------------------------------------------------------------- paged, varlen decode
+
+def _paged_case(seed, B=3, Hq=8, Hkv=2, page=4, d=8, lens=(9, 0, 16), max_pages=5):
+    rng = np.random.default_rng(seed)
+    num_pages = B * max_pages + 2
+    kp = rng.standard_normal((num_pages, Hkv, page, d))
+    vp = rng.standard_normal((num_pages, Hkv, page, d))
+    table = rng.permutation(num_pages)[: B * max_pages].reshape(B, max_pages).astype(np.int32)
+    q = rng.standard_normal((B, Hq, 1, d))
+    return q, kp, vp, table, np.array(lens, dtype=np.int32)
+
+
+def test_paged_decode_matches_torch_sdpa_on_gathered_keys():
+    q, kp, vp, table, lens = _paged_case(21)
+    O, lse = oracle.decode_paged(q, kp, vp, table, lens, scale=0.3)
+    B, Hq, _, d = q.shape
+    G = Hq // kp.shape[1]
+    for b in range(B):
+        T = int(lens[b])
+        if T == 0:
+            assert np.all(O[b] == 0.0) and np.all(np.isneginf(lse[b]))
+            continue
+        # gather by hand: logical row t lives in page table[b, t // page], slot t % page
+        page = kp.shape[2]
+        K = torch.stack([torch.from_numpy(kp[table[b, t // page], :, t % page]) for t in range(T)], 1)
+        V = torch.stack([torch.from_numpy(vp[table[b, t // page], :, t % page]) for t in range(T)], 1)
+        K = K.repeat_interleave(G, dim=0)[None]
+        V = V.repeat_interleave(G, dim=0)[None]
+        tq = torch.from_numpy(q[b:b + 1])
+        ref = torch.nn.functional.scaled_dot_product_attention(tq, K, V, scale=0.3)
+        assert np.allclose(O[b:b + 1], ref.numpy(), atol=1e-12, rtol=0)
+        S = torch.einsum("bhid,bhjd->bhij", tq, K) * 0.3
+        assert np.allclose(lse[b:b + 1], torch.logsumexp(S, -1).numpy(), atol=1e-12, rtol=0)
+
+
+def test_paged_decode_is_invariant_to_page_placement():
+    q, kp, vp, table, lens = _paged_case(22)
+    O, lse = oracle.decode_paged(q, kp, vp, table, lens)
+    perm = np.random.default_rng(5).permutation(kp.shape[0])     # new slot of each page
+    kp2 = np.empty_like(kp)
+    vp2 = np.empty_like(vp)
+    kp2[perm] = kp
+    vp2[perm] = vp
+    O2, lse2 = oracle.decode_paged(q, kp2, vp2, perm[table], lens)
+    assert np.array_equal(O, O2) and np.array_equal(lse, lse2)
+
+
+def test_paged_decode_ignores_rows_past_the_length():
+    q, kp, vp, table, lens = _paged_case(23, lens=(9, 5, 13))
+    O, lse = oracle.decode_paged(q, kp, vp, table, lens)
+    kp2, vp2 = kp.copy(), vp.copy()
+    page = kp.shape[2]
+    for b, T in enumerate(lens):
+        last = table[b, (T - 1) // page]
+        kp2[last, :, (T - 1) % page + 1:] = 1e6               # the unused tail of the last page
+        vp2[last, :, (T - 1) % page + 1:] = -1e6
+        for j in range(-(-T // page), table.shape[1]):
+            kp2[table[b, j]] = 7.0                           # pages past the length
+    O2, lse2 = oracle.decode_paged(q, kp2, vp2, table, lens)
+    assert np.array_equal(O, O2) and np.array_equal(lse, lse2)
+
+
+def test_paged_decode_equal_scores_give_mean_of_the_first_rows():
+    q, kp, vp, table, lens = _paged_case(24, lens=(7, 1, 16))
+    q = np.zeros_like(q)
+    O, lse = oracle.decode_paged(q, kp, vp, table, lens)
+    page = kp.shape[2]
+    G = q.shape[1] // kp.shape[1]
+    for b, T in enumerate(lens):
+        rows = np.stack([vp[table[b, t // page], :, t % page] for t in range(T)], 1)   # [Hkv, T, d]
+        for h in range(q.shape[1]):
+            assert np.allclose(O[b, h, 0], rows[h // G].mean(axis=0), atol=1e-14, rtol=0)
+            assert abs(lse[b, h, 0] - math.log(T)) < 1e-14
