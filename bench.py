@@ -328,6 +328,8 @@ def run_ours(args, world, rank, local):
     if not args.no_extras and args.only == "all":
         out["extras"] = {x.name: bench_prefill_variant(x, args, world, local, peaks, peak_src)
                          for x in (workloads.ALIBI_MHA, workloads.SWA_SYM_GQA)}
+        out["extras"]["paged_" + workloads.DECODE.name] = bench_decode_paged(
+            args, world, local, peaks, peak_src)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         tf, heads, dt = oracle_prefill_sample(w, args.cpu_budget)
         out["cpu_baseline"] = {"value": round(tf, 5), "unit": "TFLOP/s",
@@ -374,6 +376,58 @@ def bench_prefill_variant(w, args, world, local, peaks, peak_src):
                         "peak_source": f"bf16_tflops (burst, {peak_src})", "traffic": None},
            "gpu_launches": steps, "clocks": clk.summary()}
     del q, k, v, o, lse
+    torch.cuda.empty_cache()
+    return res
+
+
+def bench_decode_paged(args, world, local, peaks, peak_src, page: int = 256):
+    """The decode workload on a paged cache: 256-row pages placed by a seeded permutation,
+    every sequence at full length (the same KV bytes as the contiguous line)."""
+    import torch
+    import io_aware_softmax_b200 as attn
+    w = workloads.DECODE
+    dev = torch.device("cuda", torch.cuda.current_device())
+    max_pages = w.Nk // page
+    num_pages = w.B * max_pages
+    q = workloads.randn_bf16((w.B, w.Hq, 1, w.d), w.seed, 0, 1.0, dev)
+    kp = workloads.randn_bf16((num_pages, w.Hkv, page, w.d), w.seed, 1, 1.0, dev)
+    vp = workloads.randn_bf16((num_pages, w.Hkv, page, w.d), w.seed, 2, 1.0, dev)
+    perm = np.random.default_rng(w.seed).permutation(num_pages).astype(np.int32)
+    table = torch.from_numpy(perm.reshape(w.B, max_pages)).to(dev)
+    lens = torch.full((w.B,), w.Nk, dtype=torch.int32, device=dev)
+    S = attn.default_splits(w.B, w.Hkv, w.Nk, dev.index)
+    ws = torch.empty(attn.decode_workspace_bytes(w.B, w.Hq, w.d, S), dtype=torch.uint8, device=dev)
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.Hq, 1), dtype=torch.float32, device=dev)
+
+    def step():
+        attn.attn_decode_paged(q, kp, vp, table, lens, scale=w.scale, num_splits=S, workspace=ws,
+                               out=o, lse=lse)
+
+    steps = max(3, min(args.steps, 30))
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        total_ms, per = time_launches(step, steps, world)
+    if attn.device_status() != 0:
+        raise RuntimeError("device status not ok after paged decode")
+    ms = max_over_ranks(world, total_ms / steps)
+    call_ms = max_over_ranks(world, sum(per) / len(per))
+    kv = accounting.decode_kv_bytes(w.B, w.Hkv, w.Nk, w.d)
+    io = accounting.decode_io_bytes(w.B, w.Hq, w.Hkv, w.Nk, w.d) + w.B * max_pages * 4 + w.B * 4
+    peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    res = {"config": {**w.describe(), "page_size": page, "num_pages": num_pages,
+                      "placement": "seeded permutation", "seq_lens": "all T"},
+           "value": round(whole_job_rate(kv, world, ms) / 1e9, 1), "unit": "GB/s (KV cache)",
+           "tokens_per_s": round(w.B * world / (ms * 1e-3), 1), "ms_per_step": round(ms, 4),
+           "steps": steps, "num_splits": S,
+           "roofline": {"bound": "hbm", "achieved": round(io / (call_ms * 1e-3) / 1e9, 1),
+                        "peak": peak, "unit": "GB/s",
+                        "frac": round(io / (call_ms * 1e-3) / 1e9 / peak, 4),
+                        "peak_source": f"hbm_gbs ({peak_src})", "traffic": None},
+           "gpu_launches": 2 * steps, "clocks": clk.summary()}
+    del q, kp, vp, o, lse, ws
     torch.cuda.empty_cache()
     return res
 

@@ -155,6 +155,37 @@ ATTN_API int attn_decode_splitkv_noalloc(const void* q, const void* k_cache, con
                                          cudaStream_t stream);
 
 /*
+ * attn_decode_paged -- split-KV decode over paged, variable-length KV caches
+ * ("3.7 어텐션 II", 3.7.4: decode attention goes with paged KV management and in-flight
+ * batching; 3.7.8: PagedAttention keeps the cache in pages; 3.7.6: the sequences of a
+ * batch keep their own lengths).  Sequence b attends to its first seq_lens[b] cache rows;
+ * logical row t of sequence b is row (t % page_size) of physical page
+ * block_table[b * max_pages_per_seq + t / page_size].
+ *
+ *   q             bf16 [B, Hq, 1, d]            o bf16 [B, Hq, 1, d], lse fp32 [B, Hq, 1]
+ *   k_pages, v_pages  bf16 [num_pages, Hkv, page_size, d] (one page holds page_size rows
+ *                 of every KV head); page_size a multiple of 64
+ *   block_table   device int32 [B, max_pages_per_seq]; entries in [0, num_pages) for the
+ *                 pages a sequence uses (entries past its length are not read)
+ *   seq_lens      device int32 [B]; values are clamped to [0, max_pages_per_seq * page_size]
+ *   num_splits, workspace, workspace_bytes  as attn_decode_splitkv; splits cut each
+ *                 sequence at 64-row tile boundaries (<= 0: attn_decode_default_splits for
+ *                 max_pages_per_seq * page_size rows)
+ * A sequence of length 0 gets O = 0 and LSE = -inf.  A page index outside [0, num_pages)
+ * reads zeros (the copy engine fills rows outside the cache) rather than faulting.
+ * A contiguous cache with per-sequence lengths is the case num_pages = B,
+ * page_size = T (rounded up to 64), block_table[b] = {b}.
+ * Errors: INVALID_ARG, UNSUPPORTED (d not in {64,128}; Hq % Hkv != 0; Hq / Hkv > 16;
+ * page_size % 64 != 0), MISALIGNED (16 bytes for bf16 arrays and workspace, 4 for the int
+ * arrays), WORKSPACE, CUDA.
+ */
+ATTN_API int attn_decode_paged(const void* q, const void* k_pages, const void* v_pages,
+                      const int* block_table, const int* seq_lens, void* o, float* lse, int B,
+                      int Hq, int Hkv, int num_pages, int page_size, int max_pages_per_seq, int d,
+                      float scale, int num_splits, void* workspace, size_t workspace_bytes,
+                      cudaStream_t stream);
+
+/*
  * attn_decode_merge -- merge S partial results per row by the rescaling rule ("3.7 어텐션
  * II", 3.7.4): L = max_s LSE_s, w_s = exp(LSE_s - L), O = sum_s w_s O_s / sum_s w_s,
  * LSE = L + ln sum_s w_s.  Partials with LSE = -inf have weight 0.

@@ -156,6 +156,47 @@ def attn_decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, *
     return out, lse
 
 
+def attn_decode_paged(q: torch.Tensor, k_pages: torch.Tensor, v_pages: torch.Tensor,
+                      block_table: torch.Tensor, seq_lens: torch.Tensor, *,
+                      scale: Optional[float] = None, num_splits: Optional[int] = None,
+                      workspace: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
+                      lse: Optional[torch.Tensor] = None, stream=None
+                      ) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Split-KV decode over paged caches: q [B,Hq,1,d]; pages [num_pages,Hkv,page_size,d] bf16;
+    block_table int32 [B, max_pages]; seq_lens int32 [B] -> (O [B,Hq,1,d], LSE [B,Hq,1])."""
+    lib = _lib.load()
+    _need(q, "q", torch.bfloat16, 4)
+    for t, n in ((k_pages, "k_pages"), (v_pages, "v_pages")):
+        _need(t, n, torch.bfloat16, 4)
+    _need(block_table, "block_table", torch.int32, 2)
+    _need(seq_lens, "seq_lens", torch.int32, 1)
+    B, Hq, nq, d = q.shape
+    if nq != 1:
+        raise ValueError("decode takes one query token per sequence")
+    num_pages, Hkv, page_size = k_pages.shape[0], k_pages.shape[1], k_pages.shape[2]
+    max_pages = block_table.shape[1]
+    if block_table.shape[0] != B or seq_lens.numel() != B:
+        raise ValueError("block_table and seq_lens need one row / entry per sequence")
+    dev_index = q.device.index if q.device.index is not None else torch.cuda.current_device()
+    t_cap = max_pages * page_size
+    S = int(num_splits) if num_splits else default_splits(B, Hkv, max(t_cap, 1), dev_index)
+    S = max(1, min(S, max(-(-t_cap // 64), 1)))
+    need = decode_workspace_bytes(B, Hq, d, S)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, Hq, 1), dtype=torch.float32, device=q.device)
+    st = lib.attn_decode_paged(_ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(block_table),
+                               _ptr(seq_lens), _ptr(out), _ptr(lse), B, Hq, Hkv, num_pages,
+                               page_size, max_pages, d, float(scale or 0.0), S, _ptr(workspace),
+                               workspace.numel() * workspace.element_size(),
+                               _stream(q.device, stream))
+    _check(st, "attn_decode_paged")
+    return out, lse
+
+
 def attn_merge(o_part: torch.Tensor, lse_part: torch.Tensor, *, out: Optional[torch.Tensor] = None,
                lse: Optional[torch.Tensor] = None, stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
     """Merge partials o_part fp32 [rows, S, d], lse_part fp32 [rows, S] -> (O bf16, LSE fp32)."""

@@ -267,7 +267,7 @@ extern "C" int attn_decode_splitkv(const void* q, const void* k_cache, const voi
   if (!aligned16(workspace)) return ATTN_ERR_MISALIGNED;
   if (scale <= 0.f) scale = 1.0f / std::sqrt((float)d);
 
-  DecParams p;
+  DecParams p{};
   p.q = q;
   p.o_part = reinterpret_cast<float*>(workspace);
   const size_t rows = (size_t)B * Hq * num_splits;
@@ -310,3 +310,71 @@ extern "C" int attn_get_device_status(cudaStream_t stream) {
 }
 
 extern "C" int attn_last_error_site(void) { return g_last_site; }
+
+extern "C" int attn_decode_paged(const void* q, const void* k_pages, const void* v_pages,
+                                 const int* block_table, const int* seq_lens, void* o, float* lse,
+                                 int B, int Hq, int Hkv, int num_pages, int page_size,
+                                 int max_pages_per_seq, int d, float scale, int num_splits,
+                                 void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  if (B < 0 || Hq < 0 || Hkv < 0 || num_pages < 0 || page_size <= 0 || max_pages_per_seq < 0)
+    return ATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (page_size % 64 != 0) return ATTN_ERR_UNSUPPORTED;
+  if (Hkv == 0 && Hq > 0) return ATTN_ERR_INVALID_ARG;
+  if (Hkv > 0 && Hq % Hkv != 0) return ATTN_ERR_UNSUPPORTED;
+  if (std::isnan(scale)) return ATTN_ERR_INVALID_ARG;
+  if (B == 0 || Hq == 0) return ATTN_OK;
+  const int G = Hq / Hkv;
+  if (G > 16) return ATTN_ERR_UNSUPPORTED;
+  if (!q || !o || !lse || !seq_lens || !block_table) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(o) || !aligned16(lse)) return ATTN_ERR_MISALIGNED;
+  if ((reinterpret_cast<uintptr_t>(seq_lens) & 3u) || (reinterpret_cast<uintptr_t>(block_table) & 3u))
+    return ATTN_ERR_MISALIGNED;
+  const long long t_cap = (long long)max_pages_per_seq * page_size;
+  if (num_pages == 0 || t_cap == 0)
+    return launch_fill_empty(o, lse, (size_t)B * Hq, d, stream) == 0 ? ATTN_OK : ATTN_ERR_CUDA;
+  if (!k_pages || !v_pages) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(k_pages) || !aligned16(v_pages)) return ATTN_ERR_MISALIGNED;
+  if (t_cap > (1LL << 31) - 1 || (long long)num_pages * Hkv > (1LL << 31) - 1)
+    return ATTN_ERR_UNSUPPORTED;
+  const int dev = current_device();
+  const int tiles = (int)((t_cap + 63) / 64);
+  if (num_splits <= 0) num_splits = attn_decode_default_splits(B, Hkv, (int)t_cap, dev);
+  if (num_splits > tiles) num_splits = tiles;
+  const size_t need = attn_decode_workspace_bytes(B, Hq, d, num_splits);
+  if (workspace == nullptr || workspace_bytes < need) return ATTN_ERR_WORKSPACE;
+  if (!aligned16(workspace)) return ATTN_ERR_MISALIGNED;
+  if (scale <= 0.f) scale = 1.0f / std::sqrt((float)d);
+
+  DecParams p{};
+  p.q = q;
+  p.o_part = reinterpret_cast<float*>(workspace);
+  const size_t rows = (size_t)B * Hq * num_splits;
+  p.lse_part = reinterpret_cast<float*>(reinterpret_cast<char*>(workspace) +
+                                        ((rows * d * 4 + 255) & ~(size_t)255));
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.T = (int)t_cap;
+  p.S = num_splits;
+  if ((long long)B * Hkv * num_splits > (1LL << 31) - 1) return ATTN_ERR_UNSUPPORTED;
+  p.num_items = B * Hkv * num_splits;
+  p.kscale = scale * kLog2e;
+  p.block_table = block_table;
+  p.seq_lens = seq_lens;
+  p.page_size = page_size;
+  p.max_pages = max_pages_per_seq;
+  p.err = error_word_ptr(dev);
+  if (p.err == nullptr) return ATTN_ERR_CUDA;
+
+  CUtensorMap tk, tv;
+  if (!make_map_3d(&tk, k_pages, d, page_size, (long long)num_pages * Hkv, 64) ||
+      !make_map_3d(&tv, v_pages, d, page_size, (long long)num_pages * Hkv, 64))
+    return ATTN_ERR_CUDA;
+  const int slots = sm_count(dev) * decode_ctas_per_sm(d, G);
+  const int grid = (int)std::min<long long>(p.num_items, slots);
+  if (launch_decode_split(tk, tv, p, d, G, grid, stream) != 0) return ATTN_ERR_CUDA;
+  return launch_merge(p.o_part, p.lse_part, o, lse, (long long)B * Hq, num_splits, d, stream) == 0
+             ? ATTN_OK
+             : ATTN_ERR_CUDA;
+}

@@ -1,5 +1,7 @@
 // Split-KV decode attention for sm_100a (FlashDecoding, "3.7 어텐션 II", section 3.7.4):
-// one query token per sequence against a long contiguous KV cache.  The cache axis T is cut
+// one query token per sequence against a long KV cache, either contiguous or paged with a
+// page table and per-sequence lengths (PagedAttention-style in-flight batching, sections
+// 3.7.4 and 3.7.8).  The cache axis T is cut
 // into S splits; every split runs the online softmax over its slice and emits a partial
 // (O normalised by its own sum, natural-log LSE); a second kernel merges the splits with the
 // rescaling rule  L = max_s LSE_s, w_s = exp(LSE_s - L), O = sum w_s O_s / sum w_s,
@@ -78,17 +80,30 @@ __device__ __forceinline__ uint32_t swz_off(int tok, int d) {
   return (uint32_t)((d >> 6) * (kTok * 128) + tok * 128 + ((((d & 63) >> 3) ^ (tok & 7)) << 4));
 }
 
+// Item = (batch b, KV head hk, split s) and its rows [t0, t1).  Contiguous caches cut the
+// T rows evenly; paged caches cut the sequence's own length at 64-row tile boundaries, so
+// no tile straddles two pages (page_size is a multiple of the tile).
+template <bool kPaged>
 __device__ __forceinline__ void item_coords(const DecParams& p, int item, int& b, int& hk, int& s,
                                             int& t0, int& t1) {
   const int bk = item / p.S;
   s = item % p.S;
   b = bk / p.Hkv;
   hk = bk % p.Hkv;
-  t0 = (int)(((long long)s * p.T) / p.S);
-  t1 = (int)(((long long)(s + 1) * p.T) / p.S);
+  if (!kPaged) {
+    t0 = (int)(((long long)s * p.T) / p.S);
+    t1 = (int)(((long long)(s + 1) * p.T) / p.S);
+  } else {
+    const long long cap = (long long)p.max_pages * p.page_size;
+    const int T = (int)min(max((long long)__ldg(p.seq_lens + b), 0LL), cap);
+    const long long tiles = (T + kTok - 1) / kTok;
+    t0 = (int)((s * tiles) / p.S) * kTok;
+    t1 = (int)min((long long)T, (((s + 1) * tiles) / p.S) * kTok);
+    if (t1 < t0) t1 = t0;
+  }
 }
 
-template <int D, bool kUpper>
+template <int D, bool kUpper, bool kPaged>
 __global__ void __launch_bounds__(kDecThreads)
 attn_decode_split_kernel(const __grid_constant__ CUtensorMap tmK,
                          const __grid_constant__ CUtensorMap tmV, const DecParams p, int G) {
@@ -130,9 +145,9 @@ attn_decode_split_kernel(const __grid_constant__ CUtensorMap tmK,
       bool ok = true;
       for (int item = blockIdx.x; ok && item < p.num_items; item += gridDim.x) {
         int b, hk, s, t0, t1;
-        item_coords(p, item, b, hk, s, t0, t1);
+        item_coords<kPaged>(p, item, b, hk, s, t0, t1);
         const int n_st = (t1 - t0 + kTok - 1) / kTok;
-        const int z = b * p.Hkv + hk;
+        const int zc = b * p.Hkv + hk;
         for (int st = 0; st < n_st; ++st, ++gi) {
           const int sidx = gi % NS;
           const int round = gi / NS;
@@ -143,7 +158,16 @@ attn_decode_split_kernel(const __grid_constant__ CUtensorMap tmK,
           }
           mbar_arrive_expect_tx(full_bar(sidx), C::kStageBytes);
           const uint32_t dst = sRing + sidx * C::kStageBytes;
-          const int row = t0 + st * kTok;
+          int row = t0 + st * kTok;
+          int z = zc;
+          if (kPaged) {
+            // logical row -> (physical page, row in page); the cache map is
+            // (d, page_size, num_pages * Hkv), so a page index outside the table's range
+            // lands outside the map and reads zeros instead of faulting.
+            const int page = __ldg(p.block_table + (size_t)b * p.max_pages + row / p.page_size);
+            z = page * p.Hkv + hk;
+            row = row % p.page_size;
+          }
 #pragma unroll
           for (int c = 0; c < C::kChunks; ++c) {
             tma_load_3d(dst + c * C::kChunkBytes, &tmK, full_bar(sidx), c * 64, row, z);
@@ -171,7 +195,7 @@ attn_decode_split_kernel(const __grid_constant__ CUtensorMap tmK,
     bool ok = true;
     for (int item = blockIdx.x; item < p.num_items; item += gridDim.x) {
       int b, hk, s, t0, t1;
-      item_coords(p, item, b, hk, s, t0, t1);
+      item_coords<kPaged>(p, item, b, hk, s, t0, t1);
       const int n_st = (t1 - t0 + kTok - 1) / kTok;
       const int qrow0 = b * p.Hq + hk * G;
 
@@ -383,25 +407,25 @@ __global__ void attn_merge_kernel(const float* __restrict__ o_part,
   if (lane == 0) lse[row] = M + logf(wsum);
 }
 
-template <int D, bool kUpper>
+template <int D, bool kUpper, bool kPaged>
 int launch_split_t(const CUtensorMap& tk, const CUtensorMap& tv, const DecParams& p, int G,
                    int grid, cudaStream_t stream) {
   const int smem = dec_smem_bytes(D, G);
-  if (cudaFuncSetAttribute(attn_decode_split_kernel<D, kUpper>,
+  if (cudaFuncSetAttribute(attn_decode_split_kernel<D, kUpper, kPaged>,
                            cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return -4;
-  attn_decode_split_kernel<D, kUpper><<<grid, kDecThreads, smem, stream>>>(tk, tv, p, G);
+  attn_decode_split_kernel<D, kUpper, kPaged><<<grid, kDecThreads, smem, stream>>>(tk, tv, p, G);
   return cudaGetLastError() == cudaSuccess ? 0 : -4;
 }
 
 template <int D, bool kUpper>
 int occupancy_t(int G) {
   const int smem = dec_smem_bytes(D, G);
-  if (cudaFuncSetAttribute(attn_decode_split_kernel<D, kUpper>,
+  if (cudaFuncSetAttribute(attn_decode_split_kernel<D, kUpper, false>,
                            cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return 1;
   int n = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, attn_decode_split_kernel<D, kUpper>,
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, attn_decode_split_kernel<D, kUpper, false>,
                                                     kDecThreads, smem) != cudaSuccess || n < 1)
     return 1;
   return n;
@@ -427,12 +451,21 @@ int decode_ctas_per_sm(int d, int G) {
 
 int launch_decode_split(const CUtensorMap& tk, const CUtensorMap& tv, const DecParams& p, int d,
                         int G, int grid, cudaStream_t stream) {
-  if (d == 128)
-    return G > 8 ? launch_split_t<128, true>(tk, tv, p, G, grid, stream)
-                 : launch_split_t<128, false>(tk, tv, p, G, grid, stream);
-  if (d == 64)
-    return G > 8 ? launch_split_t<64, true>(tk, tv, p, G, grid, stream)
-                 : launch_split_t<64, false>(tk, tv, p, G, grid, stream);
+  const bool paged = p.block_table != nullptr;
+  if (d == 128) {
+    if (paged)
+      return G > 8 ? launch_split_t<128, true, true>(tk, tv, p, G, grid, stream)
+                   : launch_split_t<128, false, true>(tk, tv, p, G, grid, stream);
+    return G > 8 ? launch_split_t<128, true, false>(tk, tv, p, G, grid, stream)
+                 : launch_split_t<128, false, false>(tk, tv, p, G, grid, stream);
+  }
+  if (d == 64) {
+    if (paged)
+      return G > 8 ? launch_split_t<64, true, true>(tk, tv, p, G, grid, stream)
+                   : launch_split_t<64, false, true>(tk, tv, p, G, grid, stream);
+    return G > 8 ? launch_split_t<64, true, false>(tk, tv, p, G, grid, stream)
+                 : launch_split_t<64, false, false>(tk, tv, p, G, grid, stream);
+  }
   return -2;
 }
 

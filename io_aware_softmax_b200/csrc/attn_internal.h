@@ -34,6 +34,11 @@ struct DecParams {
   int num_items;      // B * Hkv * S
   float kscale;       // scale * log2(e)
   uint32_t* err;      // device error word of the library (bits, first site)
+  // Paged, variable-length caches (null / 0 for one contiguous cache of T rows each):
+  const int* block_table;   // int32 [B, max_pages]: physical page of each logical page
+  const int* seq_lens;      // int32 [B]: cache rows of each sequence
+  int page_size;            // rows per page (a multiple of the 64-row tile)
+  int max_pages;            // pages per block-table row
 };
 
 int launch_attn_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,

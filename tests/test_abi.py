@@ -156,3 +156,21 @@ def test_alibi_entry_validation(lib):
     assert a(P, P, P, P, P, 1, 2, 2, 8, 8, 96, 0.0, 1, 0, 0.0, None, 0, P, None) == -2
     assert a(None, None, None, None, None, 0, 2, 2, 8, 8, 64, 0.0, 1, 0, 0.0, None, 0, P,
              None) == 0
+
+
+def test_paged_decode_validation(lib):
+    f = lib.attn_decode_paged
+    P = ctypes.c_void_p(16)
+    I4 = ctypes.c_void_p(20)          # 4-byte aligned, not 16
+    # (q, k_pages, v_pages, table, lens, o, lse, B, Hq, Hkv, pages, page_size, max_pages, d,
+    #  scale, splits, ws, ws_bytes, stream)
+    assert f(P, P, P, I4, I4, P, P, 2, 8, 2, 10, 48, 4, 128, 0.0, 1, P, 1 << 20, None) == -2
+    assert f(P, P, P, I4, I4, P, P, 2, 8, 2, 10, 64, 4, 96, 0.0, 1, P, 1 << 20, None) == -2
+    assert f(P, P, P, I4, I4, P, P, 2, 8, 2, 10, 0, 4, 128, 0.0, 1, P, 1 << 20, None) == -1
+    assert f(P, P, P, I4, None, P, P, 2, 8, 2, 10, 64, 4, 128, 0.0, 1, P, 1 << 20, None) == -1
+    assert f(P, P, P, I4, ctypes.c_void_p(22), P, P, 2, 8, 2, 10, 64, 4, 128, 0.0, 1, P,
+             1 << 20, None) == -3
+    assert f(P, P, P, I4, I4, P, P, 2, 64, 2, 10, 64, 4, 128, 0.0, 1, P, 1 << 20, None) == -2
+    assert f(P, P, P, I4, I4, P, P, 2, 8, 2, 10, 64, 4, 128, 0.0, 2, None, 0, None) == -6
+    assert f(None, None, None, None, None, None, None, 0, 8, 2, 10, 64, 4, 128, 0.0, 1, None, 0,
+             None) == 0
