@@ -36,6 +36,9 @@ What it computes, and where that is written down (pages cited by title and secti
 * The tiled online-softmax form (normalised-O update with alpha = exp(m_old - m_new),
   beta = exp(m_local - m_new)): FlashAttention page, sections "Online Softmax와 블록 단위
   누적" and "알고리즘 의사코드".
+* Backward pass: S and P are recomputed from the saved row statistics rather than kept
+  from the forward pass: FlashAttention page, "Recomputation 전략"; the gradient formulas
+  are the calculus of the definition (``attention_backward``).
 * Split-KV decoding: each split produces partial (m, l, O) and the splits are combined by
   the same rescaling recurrence: "3.7 어텐션 II", section 3.7.4 (FlashDecoding).
 * Paged, variable-length KV caches for decode (in-flight batching with a page table,
@@ -215,6 +218,56 @@ def attention(q, k, v, scale=None, mask_kind: int = MASK_NONE, window: int = 0,
                     softcap, doc_offsets,
                     alibi_slope=0.0 if alibi_slopes is None else float(alibi_slopes[h]))
     return O, lse
+
+
+def attention_backward(q, k, v, dout, scale=None, mask_kind: int = MASK_NONE, window: int = 0,
+                       softcap: float = 0.0, doc_offsets=None, alibi_slopes=None,
+                       row_chunk: int = 256):
+    """Gradients (dQ, dK, dV) in fp64 of L with dL/dO = dout, for O = attention(q, k, v, ...).
+
+    The pages fix *how* the backward pass is organised -- S and P recomputed from the saved
+    row statistics instead of an N x N matrix kept from the forward pass (FlashAttention
+    page, "Recomputation 전략" and "FlashAttention v1: Tiling + Recomputation") -- and the
+    gradients are the calculus of the definition, written out per block of query rows:
+      dV = P^T dO;  dP = dO V^T;  D_i = sum_j P_ij dP_ij = dO_i . O_i;
+      dS = P * (dP - D)  (the softmax Jacobian);  with a soft-cap the score s = c tanh(x / c)
+      of the scaled product x contributes dx = dS (1 - tanh^2(x / c));
+      dQ = scale dX K;  dK = scale dX^T Q  (X = scale Q K^T; the ALiBi bias and the mask do
+      not depend on q, k, v).  A KV head's dK, dV sum over its query-head group.
+    Masked entries have P = 0 and so contribute nothing; rows with no visible key give 0."""
+    q = _f64(q)
+    k = _f64(k)
+    v = _f64(v)
+    dout = _f64(dout)
+    B, Hq, Nq, d = q.shape
+    Hkv, Nk = k.shape[1], k.shape[2]
+    G = Hq // Hkv
+    if scale is None or scale <= 0:
+        scale = default_scale(d)
+    dq = np.zeros_like(q)
+    dk = np.zeros_like(k)
+    dv = np.zeros_like(v)
+    for b in range(B):
+        for h in range(Hq):
+            hk = h // G
+            slope = 0.0 if alibi_slopes is None else float(alibi_slopes[h])
+            for r0 in range(0, Nq, row_chunk):
+                rows = np.arange(r0, min(Nq, r0 + row_chunk))
+                S = head_scores(q[b, h, rows], k[b, hk], scale, softcap, rows, mask_kind,
+                                window, doc_offsets, alibi_slope=slope)
+                P, _, _ = softmax_rows(S)
+                O = P @ v[b, hk]
+                dO = dout[b, h, rows]
+                dP = dO @ v[b, hk].T
+                D = (dO * O).sum(axis=1)
+                dS = P * (dP - D[:, None])
+                if softcap and softcap > 0:
+                    X = scale * (q[b, h, rows] @ k[b, hk].T)
+                    dS = dS * (1.0 - np.tanh(X / softcap) ** 2)
+                dq[b, h, rows] = scale * (dS @ k[b, hk])
+                dk[b, hk] += scale * (dS.T @ q[b, h, rows])
+                dv[b, hk] += P.T @ dO
+    return dq, dk, dv
 
 
 def attention_tiled_online(q, k, v, scale=None, block_q: int = 2, block_kv: int = 3,

@@ -565,3 +565,76 @@ def test_paged_decode_equal_scores_give_mean_of_the_first_rows():
         for h in range(q.shape[1]):
             assert np.allclose(O[b, h, 0], rows[h // G].mean(axis=0), atol=1e-14, rtol=0)
             assert abs(lse[b, h, 0] - math.log(T)) < 1e-14
+
+
+# ------------------------------------------------------------------------ backward pass
+
+def _fd_grads(q, k, v, W, eps=1e-6, **kw):
+    """Central differences of L = sum(O * W) through the forward oracle, element by element."""
+    def loss(qq, kk, vv):
+        return float((oracle.attention(qq, kk, vv, **kw)[0] * W).sum())
+    out = []
+    for x in (q, k, v):
+        g = np.zeros_like(x)
+        it = np.nditer(x, flags=["multi_index"])
+        for _ in it:
+            i = it.multi_index
+            xp, xm = x.copy(), x.copy()
+            xp[i] += eps
+            xm[i] -= eps
+            args_p = [xp if y is x else y for y in (q, k, v)]
+            args_m = [xm if y is x else y for y in (q, k, v)]
+            g[i] = (loss(*args_p) - loss(*args_m)) / (2 * eps)
+        out.append(g)
+    return out
+
+
+BWD_CASES = [dict(mask_kind=MASK_NONE), dict(mask_kind=MASK_CAUSAL),
+             dict(mask_kind=MASK_SLIDING_CAUSAL, window=2), dict(mask_kind=MASK_SLIDING, window=1),
+             dict(mask_kind=MASK_DOCUMENT_CAUSAL, doc_offsets=np.array([0, 2, 3, 6], np.int32)),
+             dict(mask_kind=MASK_CAUSAL, softcap=0.7),
+             dict(mask_kind=MASK_NONE, alibi_slopes=[0.5, 1.5, 0.25, 0.0])]
+
+
+@pytest.mark.parametrize("kw", BWD_CASES)
+def test_backward_matches_finite_differences(kw):
+    # GQA (4 query heads on 2 KV heads), N = 6, d = 3: every gradient element by central
+    # differences of the forward oracle
+    q, k, v = _rand_qkv(1, 4, 2, 6, 3, 31)
+    W = np.random.default_rng(32).standard_normal((1, 4, 6, 3))
+    kw = dict(kw, scale=0.7)
+    dq, dk, dv = oracle.attention_backward(q, k, v, W, **kw)
+    nq, nk, nv = _fd_grads(q, k, v, W, **kw)
+    for got, want in ((dq, nq), (dk, nk), (dv, nv)):
+        assert np.allclose(got, want, atol=2e-8, rtol=0), np.abs(got - want).max()
+
+
+@pytest.mark.parametrize("mask_kind,window,docs", MASKS)
+def test_backward_matches_torch_autograd_float64(mask_kind, window, docs):
+    B, Hq, Hkv, N, d = 2, 4, 2, 19, 8
+    q, k, v = _rand_qkv(B, Hq, Hkv, N, d, 33)
+    dout = np.random.default_rng(34).standard_normal((B, Hq, N, d))
+    scale = 0.3
+    dq, dk, dv = oracle.attention_backward(q, k, v, dout, scale=scale, mask_kind=mask_kind,
+                                           window=window, doc_offsets=docs)
+    tq, tk, tv = (torch.from_numpy(x).requires_grad_(True) for x in (q, k, v))
+    G = Hq // Hkv
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        tq, tk.repeat_interleave(G, dim=1), tv.repeat_interleave(G, dim=1),
+        attn_mask=_torch_mask(N, mask_kind, window, docs), scale=scale)
+    ref.backward(torch.from_numpy(dout))
+    for got, want in ((dq, tq.grad), (dk, tk.grad), (dv, tv.grad)):
+        assert np.allclose(got, want.numpy(), atol=1e-12, rtol=0)
+
+
+def test_backward_invariants():
+    # each row's dS sums to zero, so shifting every key by one vector leaves dQ unchanged;
+    # each visible row's probabilities sum to one, so the dV rows sum to the dO rows' sum
+    q, k, v = _rand_qkv(1, 2, 1, 15, 6, 35)
+    dout = np.random.default_rng(36).standard_normal((1, 2, 15, 6))
+    for kind, w in [(MASK_NONE, 0), (MASK_CAUSAL, 0), (MASK_SLIDING, 3)]:
+        dq, dk, dv = oracle.attention_backward(q, k, v, dout, mask_kind=kind, window=w)
+        dq2, _, _ = oracle.attention_backward(q, k + np.arange(6.0), v, dout, mask_kind=kind,
+                                              window=w)
+        assert np.allclose(dq, dq2, atol=1e-12, rtol=0)
+        assert np.allclose(dv.sum(axis=2)[0, 0], dout.sum(axis=(1, 2))[0], atol=1e-12, rtol=0)
