@@ -330,6 +330,8 @@ def run_ours(args, world, rank, local):
                          for x in (workloads.ALIBI_MHA, workloads.SWA_SYM_GQA)}
         out["extras"]["paged_" + workloads.DECODE.name] = bench_decode_paged(
             args, world, local, peaks, peak_src)
+        out["extras"]["backward_" + workloads.CAUSAL_MHA.name] = bench_backward(
+            workloads.CAUSAL_MHA, args, world, local, peaks, peak_src)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         tf, heads, dt = oracle_prefill_sample(w, args.cpu_budget)
         out["cpu_baseline"] = {"value": round(tf, 5), "unit": "TFLOP/s",
@@ -428,6 +430,47 @@ def bench_decode_paged(args, world, local, peaks, peak_src, page: int = 256):
                         "peak_source": f"hbm_gbs ({peak_src})", "traffic": None},
            "gpu_launches": 2 * steps, "clocks": clk.summary()}
     del q, kp, vp, o, lse, ws
+    torch.cuda.empty_cache()
+    return res
+
+
+def bench_backward(w, args, world, local, peaks, peak_src):
+    """Useful TFLOP/s of attn_bwd (dQ, dK, dV from O, LSE and dO) on a prefill workload."""
+    import torch
+    import io_aware_softmax_b200 as attn
+    dev = torch.device("cuda", torch.cuda.current_device())
+    q, k, v = workloads.make_inputs(w, device=dev)
+    dout = workloads.randn_bf16((w.B, w.Hq, w.Nq, w.d), w.seed, 3, 1.0, dev)
+    o, lse = attn.attn_fwd(q, k, v, scale=w.scale, mask=w.mask_kind, window=w.window)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = torch.empty(attn.bwd_workspace_bytes(w.B, w.Hq, w.Nq), dtype=torch.uint8, device=dev)
+    flops = accounting.backward_useful_flops(w.B, w.Hq, w.Nq, w.Nk, w.d, w.mask_kind, w.window)
+
+    def step():
+        attn.attn_bwd(q, k, v, o, lse, dout, scale=w.scale, mask=w.mask_kind, window=w.window,
+                      dq=dq, dk=dk, dv=dv, workspace=ws)
+
+    steps = max(3, min(args.steps, 20))
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        total_ms, per = time_launches(step, steps, world)
+    if attn.device_status() != 0:
+        raise RuntimeError("device status not ok after the backward pass")
+    ms = max_over_ranks(world, total_ms / steps)
+    call_ms = max_over_ranks(world, sum(per) / len(per))
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    achieved = flops / (call_ms * 1e-3) / 1e12
+    res = {"config": w.describe(), "value": round(whole_job_rate(flops, world, ms) / 1e12, 2),
+           "unit": "TFLOP/s", "ms_per_step": round(ms, 4), "steps": steps,
+           "useful_tflop_per_step": round(flops / 1e12, 4),
+           "flop_accounting": "10 d per visible pair (S, dP, dV, dQ, dK)",
+           "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak,
+                        "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                        "peak_source": f"bf16_tflops (burst, {peak_src})", "traffic": None},
+           "gpu_launches": 3 * steps, "clocks": clk.summary()}
+    del q, k, v, o, lse, dout, dq, dk, dv, ws
     torch.cuda.empty_cache()
     return res
 

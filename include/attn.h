@@ -98,6 +98,31 @@ ATTN_API int attn_fwd_alibi(const void* q, const void* k, const void* v, void* o
              const float* alibi_slopes, cudaStream_t stream);
 
 /*
+ * attn_bwd -- backward pass of attn_fwd: dQ, dK, dV from (q, k, v, o, dout, lse).
+ * Defining passages: FlashAttention page, "Recomputation 전략" (S and P are recomputed block
+ * by block from the saved row statistics instead of keeping an N x N matrix) -- here from
+ * the natural-log LSE attn_fwd returns; the gradients are those of the definition:
+ * dV = P^T dO, dP = dO V^T, dS = P (dP - rowsum(dO * O)), dQ = scale dS K,
+ * dK = scale dS^T Q, a KV head's dK and dV summing over its query-head group.
+ *
+ *   q, k, v, o, lse   as attn_fwd (o and lse: attn_fwd's outputs for these inputs)
+ *   dout         bf16 [B, Hq, Nq, d]   gradient of the loss with respect to o
+ *   dq           bf16 [B, Hq, Nq, d]   dk, dv  bf16 [B, Hkv, Nk, d]   (written)
+ *   mask_kind, window, doc_offsets, num_docs, scale   as attn_fwd; softcap must be <= 0
+ *   workspace    device, 16-byte aligned, attn_bwd_workspace_bytes(B, Hq, Nq) bytes (the
+ *                per-row rowsum(dO * O) and base-2 LSE); contents are scratch
+ * Three kernel launches on `stream`, no host synchronisation.  Rows with no visible key
+ * (LSE = -inf) contribute nothing; keys no query sees get dK = dV = 0.
+ * Errors: as attn_fwd, plus UNSUPPORTED for softcap > 0 and WORKSPACE.
+ */
+ATTN_API size_t attn_bwd_workspace_bytes(int B, int Hq, int Nq);
+ATTN_API int attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
+             const float* lse, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int Nq,
+             int Nk, int d, float scale, int mask_kind, int window, float softcap,
+             const int* doc_offsets, int num_docs, void* workspace, size_t workspace_bytes,
+             cudaStream_t stream);
+
+/*
  * attn_blockmap -- 128x128 block-sparsity map of a mask ("PyTorch FlexAttention 도입 분석",
  * section 2: BlockMask precomputed in 128 x 128 chunks so empty tiles are skipped).
  *   map  device uint8 [B, ceil(Nq/128), ceil(Nk/128)] (written): ATTN_TILE_EMPTY when no

@@ -5,11 +5,11 @@ this package is its thin Python binding.  Importing it does not load the library
 call does, and raises if the library is missing -- there is no other implementation.
 """
 from .api import (  # noqa: F401
-    MASKS, AttnError, attn_blockmap, attn_decode, attn_decode_paged, attn_fwd, attn_merge, decode_workspace_bytes,
-    default_splits, device_status,
+    MASKS, AttnError, attn_blockmap, attn_bwd, attn_decode, attn_decode_paged, attn_fwd,
+    attn_merge, bwd_workspace_bytes, decode_workspace_bytes, default_splits, device_status,
 )
 from ._lib import LIB_PATH, LibraryMissing, load as load_library  # noqa: F401
 
-__all__ = ["attn_fwd", "attn_blockmap", "attn_decode", "attn_decode_paged", "attn_merge", "decode_workspace_bytes",
-           "default_splits", "device_status", "AttnError", "LibraryMissing", "load_library",
-           "MASKS", "LIB_PATH"]
+__all__ = ["attn_fwd", "attn_bwd", "attn_blockmap", "attn_decode", "attn_decode_paged",
+           "attn_merge", "bwd_workspace_bytes", "decode_workspace_bytes", "default_splits",
+           "device_status", "AttnError", "LibraryMissing", "load_library", "MASKS", "LIB_PATH"]

@@ -27,6 +27,10 @@ SIGNATURES = {
     "attn_decode_paged": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                   c_void_p, c_int, c_int, c_int, c_int, c_int, c_int, c_int,
                                   c_float, c_int, c_void_p, c_size_t, c_void_p]),
+    "attn_bwd_workspace_bytes": (c_size_t, [c_int, c_int, c_int]),
+    "attn_bwd": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                         c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_int, c_int, c_float,
+                         c_int, c_int, c_float, c_void_p, c_int, c_void_p, c_size_t, c_void_p]),
     "attn_blockmap": (c_int, [c_int, c_int, c_int, c_int, c_int, c_void_p, c_int, c_void_p,
                               c_void_p]),
     "attn_decode_workspace_bytes": (c_size_t, [c_int, c_int, c_int, c_int]),

@@ -97,6 +97,44 @@ def attn_fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, scale: Option
     return out, lse
 
 
+def bwd_workspace_bytes(B: int, Hq: int, Nq: int) -> int:
+    return int(_lib.load().attn_bwd_workspace_bytes(B, Hq, Nq))
+
+
+def attn_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,
+             lse: torch.Tensor, dout: torch.Tensor, *, scale: Optional[float] = None,
+             mask="none", window: int = 0, doc_offsets: Optional[torch.Tensor] = None,
+             dq: Optional[torch.Tensor] = None, dk: Optional[torch.Tensor] = None,
+             dv: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+             stream=None) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+    """Backward of attn_fwd: (dq, dk, dv) from q, k, v, attn_fwd's (o, lse) and dout."""
+    lib = _lib.load()
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (dout, "dout")):
+        _need(t, n, torch.bfloat16, 4)
+    _need(lse, "lse", torch.float32, 3)
+    B, Hq, Nq, d = q.shape
+    Hkv, Nk = k.shape[1], k.shape[2]
+    if o.shape != q.shape or dout.shape != q.shape or tuple(lse.shape) != (B, Hq, Nq):
+        raise ValueError("o and dout must have q's shape and lse [B, Hq, Nq]")
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    need = bwd_workspace_bytes(B, Hq, Nq)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    num_docs = 0
+    if doc_offsets is not None:
+        _need(doc_offsets, "doc_offsets", torch.int32, 1)
+        num_docs = doc_offsets.numel() - 1
+    st = lib.attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq),
+                      _ptr(dk), _ptr(dv), B, Hq, Hkv, Nq, Nk, d, float(scale or 0.0),
+                      _mask_id(mask), int(window), 0.0, _ptr(doc_offsets), num_docs,
+                      _ptr(workspace), workspace.numel() * workspace.element_size(),
+                      _stream(q.device, stream))
+    _check(st, "attn_bwd")
+    return dq, dk, dv
+
+
 def attn_blockmap(B: int, Nq: int, Nk: int, *, mask="none", window: int = 0,
                   doc_offsets: Optional[torch.Tensor] = None, device=None,
                   out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:

@@ -378,3 +378,82 @@ extern "C" int attn_decode_paged(const void* q, const void* k_pages, const void*
              ? ATTN_OK
              : ATTN_ERR_CUDA;
 }
+
+extern "C" size_t attn_bwd_workspace_bytes(int B, int Hq, int Nq) {
+  if (B <= 0 || Hq <= 0 || Nq <= 0) return 0;
+  const size_t rows = (size_t)B * Hq * Nq;
+  return 2 * ((rows * 4 + 255) & ~(size_t)255);
+}
+
+extern "C" int attn_bwd(const void* q, const void* k, const void* v, const void* o,
+                        const void* dout, const float* lse, void* dq, void* dk, void* dv, int B,
+                        int Hq, int Hkv, int Nq, int Nk, int d, float scale, int mask_kind,
+                        int window, float softcap, const int* doc_offsets, int num_docs,
+                        void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  if (B < 0 || Hq < 0 || Hkv < 0 || Nq < 0 || Nk < 0) return ATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (Hkv == 0 && Hq > 0) return ATTN_ERR_INVALID_ARG;
+  if (Hkv > 0 && Hq % Hkv != 0) return ATTN_ERR_UNSUPPORTED;
+  int st = check_mask(mask_kind, window, doc_offsets, num_docs, Nq, Nk);
+  if (st != ATTN_OK) return st;
+  if (std::isnan(scale) || std::isnan(softcap)) return ATTN_ERR_INVALID_ARG;
+  if (softcap > 0.f) return ATTN_ERR_UNSUPPORTED;
+  if (B == 0 || Hq == 0 || (Nq == 0 && Nk == 0)) return ATTN_OK;
+  const void* ptrs[] = {q, k, v, o, dout, lse, dq, dk, dv};
+  const int needed[] = {Nq > 0, Nk > 0, Nk > 0, Nq > 0, Nq > 0, Nq > 0, Nq > 0, Nk > 0, Nk > 0};
+  for (int i = 0; i < 9; ++i) {
+    if (!needed[i]) continue;
+    if (ptrs[i] == nullptr) return ATTN_ERR_INVALID_ARG;
+    if (!aligned16(ptrs[i])) return ATTN_ERR_MISALIGNED;
+  }
+  const size_t rows = (size_t)B * Hq * Nq;
+  const size_t need = attn_bwd_workspace_bytes(B, Hq, Nq);
+  if (Nq > 0 && (workspace == nullptr || workspace_bytes < need)) return ATTN_ERR_WORKSPACE;
+  if (Nq > 0 && !aligned16(workspace)) return ATTN_ERR_MISALIGNED;
+  if ((long long)B * Hq > (1LL << 31) - 1 || (long long)B * Hkv * ((Nk + 127) / 128) > (1LL << 31) - 1 ||
+      (long long)B * Hq * ((Nq + 127) / 128) > (1LL << 31) - 1)
+    return ATTN_ERR_UNSUPPORTED;
+  if (scale <= 0.f) scale = 1.0f / std::sqrt((float)d);
+  const int dev = current_device();
+
+  BwdParams p{};
+  p.dq = dq;
+  p.dk = dk;
+  p.dv = dv;
+  p.dvec = reinterpret_cast<float*>(workspace);
+  p.l2 = reinterpret_cast<float*>(reinterpret_cast<char*>(workspace) + need / 2);
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.Nq = Nq;
+  p.Nk = Nk;
+  p.G = Hq / Hkv;
+  p.kscale = scale * kLog2e;
+  p.scale = scale;
+  p.mask = mask_params(mask_kind, window, doc_offsets, num_docs, Nq, Nk);
+  p.err = error_word_ptr(dev);
+  if (p.err == nullptr) return ATTN_ERR_CUDA;
+  if (Nq > 0 && launch_bwd_rowdot(o, dout, lse, const_cast<float*>(p.dvec),
+                                  const_cast<float*>(p.l2), (long long)rows, d, stream) != 0)
+    return ATTN_ERR_CUDA;
+
+  // With no query rows dK = dV = 0; with no keys dQ = 0 (the kernels write these too, but
+  // their maps need a non-empty tensor).
+  CUtensorMap tq, tdo, tk, tv;
+  if (Nq == 0 || Nk == 0) {
+    if (Nk > 0) {
+      if (cudaMemsetAsync(dk, 0, (size_t)B * Hkv * Nk * d * 2, stream) != cudaSuccess ||
+          cudaMemsetAsync(dv, 0, (size_t)B * Hkv * Nk * d * 2, stream) != cudaSuccess)
+        return ATTN_ERR_CUDA;
+    }
+    if (Nq > 0 && cudaMemsetAsync(dq, 0, rows * d * 2, stream) != cudaSuccess)
+      return ATTN_ERR_CUDA;
+    return ATTN_OK;
+  }
+  if (!make_map_3d(&tq, q, d, Nq, (long long)B * Hq, 128) ||
+      !make_map_3d(&tdo, dout, d, Nq, (long long)B * Hq, 128) ||
+      !make_map_3d(&tk, k, d, Nk, (long long)B * Hkv, 128) ||
+      !make_map_3d(&tv, v, d, Nk, (long long)B * Hkv, 128))
+    return ATTN_ERR_CUDA;
+  return launch_attn_bwd(tq, tdo, tk, tv, p, d, stream) == 0 ? ATTN_OK : ATTN_ERR_CUDA;
+}

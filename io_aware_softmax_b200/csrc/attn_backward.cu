@@ -1,0 +1,627 @@
+// Backward pass of the fused attention for sm_100a: dQ, dK, dV from (Q, K, V, O, dO, LSE)
+// without any N x N matrix in memory.  S and P are recomputed tile by tile from the saved
+// row log-sum-exp -- the recomputation strategy of "FlashAttention 논문 분석: IO-Aware Exact
+// Attention" (sections "FlashAttention v1: Tiling + Recomputation" and "Recomputation 전략")
+// -- and the gradients are the calculus of the definition:
+//   P = exp(scale q.k - LSE),  dP = dO V^T,  D = rowsum(dO * O),  dS = P (dP - D),
+//   dV = P^T dO,  dQ = scale dS K,  dK = scale dS^T Q   (GQA: dK, dV sum over the group).
+//
+// Three launches:
+//   * attn_bwd_rowdot_kernel: D and the base-2 LSE of every query row (one warp per row);
+//   * attn_bwd_dq_kernel: one CTA per 128-row query tile; the K/V tiles its rows can see
+//     stream through a TMA ring; per K/V tile the tensor core computes S = Q K^T and
+//     dP = dO V^T into two TMEM buffers, a warpgroup (thread r = row r) turns them into
+//     bf16 dS written back into the low half of the dP buffer, and the tensor core adds
+//     dS K (A read from TMEM, K as an MN-major operand) into the dQ accumulator in TMEM;
+//   * attn_bwd_dkdv_kernel: one CTA per 128-key tile of a KV head; the (Q, dO) tiles of
+//     every query head of its group that can see the keys stream through the ring; the
+//     tensor core computes S^T = K Q^T and dP^T = V dO^T, the warpgroup (thread r = key r)
+//     writes bf16 P^T and dS^T into the low halves of those buffers, and dV += P^T dO and
+//     dK += dS^T Q accumulate in TMEM -- dK and dV of a tile are complete in one CTA, so
+//     nothing is accumulated with atomics.
+// Warps: 0-3 the element-wise warpgroup, 4 the tcgen05 issuer (whole warp, elect.sync),
+// 5 the TMA producer.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "attn_internal.h"
+#include "mask.cuh"
+#include "sm100_ptx.cuh"
+#include "tmem_ldst.cuh"
+
+namespace attn {
+
+namespace {
+
+constexpr int kBT = 128;                 // rows of every tile (queries or keys)
+constexpr int kBwdThreads = 192;
+constexpr int kBwdMmaWarp = 4;
+constexpr int kBwdTmaWarp = 5;
+constexpr float kLog2eB = 1.44269504088896341f;
+constexpr uint32_t kTmemX = 0;           // S or S^T (fp32), then bf16 P^T in its low half
+constexpr uint32_t kTmemY = 128;         // dP or dP^T (fp32), then bf16 dS / dS^T
+constexpr uint32_t kTmemAcc0 = 256;      // dQ, or dV
+constexpr uint32_t kTmemAcc1 = 384;      // dK
+
+template <int D>
+struct BwdCfg {
+  static constexpr int kChunks = D / 64;
+  static constexpr int kChunkBytes = kBT * 128;
+  static constexpr int kTileBytes = kBT * D * 2;
+  static constexpr int kStages = (D == 128) ? 2 : 4;     // ring stages of two tiles each
+  static constexpr int kStatOff = 0;                     // two stationary tiles
+  static constexpr int kRingOff = 2 * kTileBytes;
+  static constexpr int kVecOff = kRingOff + kStages * 2 * kTileBytes;
+  static constexpr int kVecBytes = 2 * 4 * kBT * 4;      // [2 parities][lse2, D, lo, hi][128]
+  static constexpr int kBarOff = kVecOff + kVecBytes;
+  // stat, full[S], empty[S], s_ready, p_ready, acc, done
+  static constexpr int kNumBars = 5 + 2 * kStages;
+  static constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 16 + 1024;
+};
+
+enum : uint32_t {
+  kSiteBwdStat = 201, kSiteBwdFull, kSiteBwdEmpty, kSiteBwdS, kSiteBwdP, kSiteBwdAcc,
+  kSiteBwdDrain,
+};
+
+__device__ __forceinline__ float bf(uint32_t u) { return __uint_as_float(u); }
+
+// One chunk of 32 columns of the recomputed tile for one TMEM lane: s (raw q.k) and dp in
+// fp32; returns bf16 pairs of p (optional) and ds = p (dp - Dv) with p = 2^(s ks - l2).
+// vis(c) says whether column c of the chunk is a visible pair.
+template <bool kWantP, typename Vis, typename L2, typename DV>
+__device__ __forceinline__ void grad_chunk(const uint32_t (&s)[32], const uint32_t (&dp)[32],
+                                           float ks, Vis vis, L2 l2, DV dv,
+                                           uint32_t (&pk)[16], uint32_t (&dsk)[16]) {
+#pragma unroll
+  for (int c = 0; c < 32; c += 2) {
+    float p0 = ex2_approx(bf(s[c]) * ks - l2(c));
+    float p1 = ex2_approx(bf(s[c + 1]) * ks - l2(c + 1));
+    if (!vis(c)) p0 = 0.f;
+    if (!vis(c + 1)) p1 = 0.f;
+    const float d0 = p0 * (bf(dp[c]) - dv(c));
+    const float d1 = p1 * (bf(dp[c + 1]) - dv(c + 1));
+    if (kWantP) pk[c >> 1] = pack_bf16x2(p0, p1);
+    dsk[c >> 1] = pack_bf16x2(d0, d1);
+  }
+}
+
+// First / last query row whose visible key interval meets keys [k0, k1] (the intervals are
+// non-decreasing at both ends, so the rows that see the tile form one range); qa > qb when
+// no row does.
+__device__ __forceinline__ void query_range(const MaskParams& m, int Nq, int k0, int k1, int& qa,
+                                            int& qb) {
+  int lo = 0, hi = Nq;             // first row with hi(q) >= k0
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    int a, b;
+    row_interval(m, mid, a, b);
+    if (b >= k0) hi = mid; else lo = mid + 1;
+  }
+  qa = lo;
+  lo = -1;
+  hi = Nq - 1;                     // last row with lo(q) <= k1
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    int a, b;
+    row_interval(m, mid, a, b);
+    if (a <= k1) lo = mid; else hi = mid - 1;
+  }
+  qb = lo;
+}
+
+// One row of NCOL fp32 TMEM columns (read in 32-column chunks), times mul, rounded to bf16
+// and written to global memory when the row exists.
+template <int NCOL>
+__device__ __forceinline__ void store_row(uint32_t taddr, float mul, __nv_bfloat16* dst,
+                                          bool valid) {
+#pragma unroll
+  for (int cc = 0; cc < NCOL / 32; ++cc) {
+    uint32_t a[32];
+    tmem_ld_x32(taddr + 32u * cc, a);
+    uint32_t wv[16];
+#pragma unroll
+    for (int k = 0; k < 16; ++k) wv[k] = pack_bf16x2(bf(a[2 * k]) * mul, bf(a[2 * k + 1]) * mul);
+    if (valid) {
+      uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * cc);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) d4[k] = make_uint4(wv[4 * k], wv[4 * k + 1], wv[4 * k + 2],
+                                                      wv[4 * k + 3]);
+    }
+  }
+}
+
+__device__ __forceinline__ void store_zero_row(__nv_bfloat16* dst, int n, bool valid) {
+  if (!valid) return;
+  uint4* d4 = reinterpret_cast<uint4*>(dst);
+  for (int k = 0; k < n / 8; ++k) d4[k] = make_uint4(0u, 0u, 0u, 0u);
+}
+
+// D = rowsum(dO * O) and l2 = LSE * log2(e) (+inf for a row without any visible key, so
+// that 2^(x - l2) = 0) for every query row; one warp per row.
+__global__ void attn_bwd_rowdot_kernel(const __nv_bfloat16* __restrict__ o,
+                                       const __nv_bfloat16* __restrict__ dout,
+                                       const float* __restrict__ lse, float* dvec, float* l2,
+                                       long long rows, int Dh) {
+  const long long row = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  const __nv_bfloat162* a = reinterpret_cast<const __nv_bfloat162*>(o + row * Dh);
+  const __nv_bfloat162* b = reinterpret_cast<const __nv_bfloat162*>(dout + row * Dh);
+  float acc = 0.f;
+  for (int c = lane; c < Dh / 2; c += 32) {
+    const float2 x = __bfloat1622float2(a[c]);
+    const float2 y = __bfloat1622float2(b[c]);
+    acc = fmaf(x.x, y.x, fmaf(x.y, y.y, acc));
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  if (lane == 0) {
+    dvec[row] = acc;
+    const float L = lse[row];
+    l2[row] = (L == -INFINITY) ? INFINITY : L * kLog2eB;
+  }
+}
+
+// Shared pieces of the two gradient kernels: the barrier layout and the tcgen05 issue of
+// one streamed tile pair (two SS products into X and Y, then TS products from X / Y).
+template <int D>
+struct BwdSmem {
+  uint32_t stat, ring, bars;
+  uint8_t* base;
+  __device__ __forceinline__ uint32_t bar(int i) const { return bars + 8u * (uint32_t)i; }
+};
+
+template <int D>
+__device__ __forceinline__ BwdSmem<D> bwd_smem(uint8_t* smem_raw) {
+  using C = BwdCfg<D>;
+  BwdSmem<D> s;
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  s.base = smem_raw + (base - raw);
+  s.stat = base + C::kStatOff;
+  s.ring = base + C::kRingOff;
+  s.bars = base + C::kBarOff;
+  return s;
+}
+
+// X or Y = A_stat[a] (stationary tile a, K-major) times B^T (ring tile, K-major): 128 x 128.
+template <int D>
+__device__ __forceinline__ void issue_ss(uint32_t d_tmem, uint32_t a_smem, uint32_t b_smem) {
+  using C = BwdCfg<D>;
+  constexpr uint32_t idesc = idesc_bf16_f32(kBT, kBT, false);
+  const uint64_t da = smem_desc(a_smem, 16, 1024);
+  const uint64_t db = smem_desc(b_smem, 16, 1024);
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    const uint32_t off = ((kk >> 2) * C::kChunkBytes + (kk & 3) * 32) >> 4;
+    umma_ss_warp(d_tmem, da + off, db + off, idesc, kk > 0 ? 1u : 0u);
+  }
+}
+
+// acc (128 x D) += A (bf16 pairs in TMEM columns [a_col, a_col + 64)) times B (ring tile:
+// 128 rows along the contraction, D columns, MN-major).
+template <int D>
+__device__ __forceinline__ void issue_ts(uint32_t acc, uint32_t a_tmem, uint32_t b_smem,
+                                         bool first) {
+  using C = BwdCfg<D>;
+  constexpr uint32_t idesc = idesc_bf16_f32(kBT, D, true);
+  const uint64_t db = smem_desc(b_smem, C::kChunkBytes, 1024);
+#pragma unroll
+  for (int kk = 0; kk < kBT / 16; ++kk)
+    umma_ts_warp(acc, a_tmem + 8u * kk, db + ((kk * 16 * 128) >> 4), idesc,
+                 (!first || kk > 0) ? 1u : 0u);
+}
+
+// dQ of one 128-row query tile of head (b, h).
+template <int D>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO,
+                   const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                   const BwdParams p) {
+  using C = BwdCfg<D>;
+  constexpr int NS = C::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  const BwdSmem<D> sm = bwd_smem<D>(smem_raw);
+  const int BAR_STAT = 0, BAR_FULL = 1, BAR_EMPTY = 1 + NS, BAR_S = 1 + 2 * NS,
+            BAR_P = 2 + 2 * NS, BAR_ACC = 3 + 2 * NS, BAR_DONE = 4 + 2 * NS;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm.base + C::kBarOff + C::kNumBars * 8);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  const int nqt = (p.Nq + kBT - 1) / kBT;
+  const int bh = blockIdx.x / nqt, qt = blockIdx.x % nqt;
+  const int b = bh / p.Hq, h = bh % p.Hq, hk = h / p.G;
+  const int q0 = qt * kBT;
+  int lo_first, hi_first, lo_last, hi_last;
+  row_interval(p.mask, q0, lo_first, hi_first);
+  row_interval(p.mask, min(q0 + kBT, p.Nq) - 1, lo_last, hi_last);
+  int ja = 0, n = 0;                    // K/V tiles [ja, ja + n) that the tile's rows see
+  if (p.Nk > 0 && hi_last >= lo_first) {
+    ja = lo_first / kBT;
+    n = hi_last / kBT - ja + 1;
+  }
+
+  if (threadIdx.x == 0) {
+    mbar_init(sm.bar(BAR_STAT), 1);
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(sm.bar(BAR_FULL + s), 1);
+      mbar_init(sm.bar(BAR_EMPTY + s), 1);
+    }
+    mbar_init(sm.bar(BAR_S), 1);
+    mbar_init(sm.bar(BAR_P), 4);
+    mbar_init(sm.bar(BAR_ACC), 1);
+    mbar_init(sm.bar(BAR_DONE), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == kBwdMmaWarp) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == kBwdTmaWarp) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0 && n > 0) {
+      mbar_arrive_expect_tx(sm.bar(BAR_STAT), 2 * C::kTileBytes);
+#pragma unroll
+      for (int c = 0; c < C::kChunks; ++c) {
+        tma_load_3d(sm.stat + c * C::kChunkBytes, &tmQ, sm.bar(BAR_STAT), c * 64, q0, bh);
+        tma_load_3d(sm.stat + C::kTileBytes + c * C::kChunkBytes, &tmDO, sm.bar(BAR_STAT),
+                    c * 64, q0, bh);
+      }
+      const int zkv = b * p.Hkv + hk;
+      int t = 0;
+      for (; t < n; ++t) {
+        const int s = t % NS, round = t / NS;
+        if (round > 0 &&
+            !mbar_wait(sm.bar(BAR_EMPTY + s), (round - 1) & 1, abort_flag, p.err, kSiteBwdEmpty))
+          break;
+        mbar_arrive_expect_tx(sm.bar(BAR_FULL + s), 2 * C::kTileBytes);
+        const uint32_t dst = sm.ring + s * 2 * C::kTileBytes;
+#pragma unroll
+        for (int c = 0; c < C::kChunks; ++c) {
+          tma_load_3d(dst + c * C::kChunkBytes, &tmK, sm.bar(BAR_FULL + s), c * 64,
+                      (ja + t) * kBT, zkv);
+          tma_load_3d(dst + C::kTileBytes + c * C::kChunkBytes, &tmV, sm.bar(BAR_FULL + s),
+                      c * 64, (ja + t) * kBT, zkv);
+        }
+      }
+      // outstanding copies land before the CTA may exit (matters only on abort)
+      mbar_wait(sm.bar(BAR_STAT), 0, nullptr, p.err, kSiteBwdDrain);
+      for (int s = 0; s < NS && s < t; ++s) {
+        const int last = s + ((t - 1 - s) / NS) * NS;
+        mbar_wait(sm.bar(BAR_FULL + s), (last / NS) & 1, nullptr, p.err, kSiteBwdDrain);
+      }
+    }
+    __syncwarp();
+  } else if (warp == kBwdMmaWarp) {
+    // -------------------------------------------------------------- tcgen05 issuer
+    if (n > 0) {
+      bool ok = mbar_wait_warp(sm.bar(BAR_STAT), 0, abort_flag, p.err, kSiteBwdStat);
+      tc_fence_after();
+      for (int t = 0; ok && t < n; ++t) {
+        const int s = t % NS;
+        if (!mbar_wait_warp(sm.bar(BAR_FULL + s), (t / NS) & 1, abort_flag, p.err, kSiteBwdFull))
+          break;
+        tc_fence_after();
+        const uint32_t kt = sm.ring + s * 2 * C::kTileBytes;
+        issue_ss<D>(tmem + kTmemX, sm.stat, kt);                              // S = Q K^T
+        issue_ss<D>(tmem + kTmemY, sm.stat + C::kTileBytes, kt + C::kTileBytes);  // dP
+        umma_commit_warp(sm.bar(BAR_S));
+        if (!mbar_wait_warp(sm.bar(BAR_P), t & 1, abort_flag, p.err, kSiteBwdP)) break;
+        tc_fence_after();
+        issue_ts<D>(tmem + kTmemAcc0, tmem + kTmemY, kt, t == 0);            // dQ += dS K
+        umma_commit_warp(sm.bar(BAR_EMPTY + s));
+      }
+      umma_commit_warp(sm.bar(BAR_ACC));
+    }
+    umma_commit_warp(sm.bar(BAR_DONE));
+    mbar_wait_warp(sm.bar(BAR_DONE), 0, nullptr, p.err, kSiteBwdDrain);
+  } else {
+    // ------------------------------------------------------ element-wise warpgroup
+    const int wq = warp;                       // TMEM lane quarter
+    const int r = wq * 32 + lane;
+    const int row = q0 + r;
+    const bool valid = row < p.Nq;
+    const long long ridx = (long long)bh * p.Nq + row;
+    const float l2r = valid ? p.l2[ridx] : INFINITY;
+    const float dr = valid ? p.dvec[ridx] : 0.f;
+    int rlo = 1, rhi = 0;
+    if (valid) row_interval(p.mask, row, rlo, rhi);
+    const uint32_t tl = tmem + ((uint32_t)(wq * 32) << 16);
+    __nv_bfloat16* drow = reinterpret_cast<__nv_bfloat16*>(p.dq) + ridx * D;
+    bool ok = true;
+    for (int t = 0; ok && t < n; ++t) {
+      ok = __all_sync(0xffffffffu, mbar_wait(sm.bar(BAR_S), t & 1, abort_flag, p.err, kSiteBwdS));
+      if (!ok) break;
+      tc_fence_after();
+      const int k0 = (ja + t) * kBT;
+      const bool full = lo_last <= k0 && k0 + kBT - 1 <= hi_first && k0 + kBT <= p.Nk;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        uint32_t s[32], dp[32], pk[16], dsk[16];
+        tmem_ld_x32(tl + kTmemX + 32u * c, s);
+        tmem_ld_x32(tl + kTmemY + 32u * c, dp);
+        const int kc = k0 + 32 * c;
+        grad_chunk<false>(
+            s, dp, p.kscale,
+            [&](int i) { return full || (kc + i >= rlo && kc + i <= rhi); },
+            [&](int) { return l2r; }, [&](int) { return dr; }, pk, dsk);
+        tmem_st_x16(tl + kTmemY + 16u * c, dsk);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(sm.bar(BAR_P));
+    }
+    if (n == 0) {
+      store_zero_row(drow, D, valid);
+    } else if (ok) {
+      const bool okacc =
+          __all_sync(0xffffffffu, mbar_wait(sm.bar(BAR_ACC), 0, abort_flag, p.err, kSiteBwdAcc));
+      if (okacc) {
+        tc_fence_after();
+        store_row<D>(tl + kTmemAcc0, p.scale, drow, valid);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kBwdMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// dK and dV of one 128-key tile of KV head (b, hk), summed over the query heads of its group.
+template <int D>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ,
+                     const __grid_constant__ CUtensorMap tmDO,
+                     const __grid_constant__ CUtensorMap tmK,
+                     const __grid_constant__ CUtensorMap tmV, const BwdParams p) {
+  using C = BwdCfg<D>;
+  constexpr int NS = C::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  const BwdSmem<D> sm = bwd_smem<D>(smem_raw);
+  const int BAR_STAT = 0, BAR_FULL = 1, BAR_EMPTY = 1 + NS, BAR_S = 1 + 2 * NS,
+            BAR_P = 2 + 2 * NS, BAR_ACC = 3 + 2 * NS, BAR_DONE = 4 + 2 * NS;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm.base + C::kBarOff + C::kNumBars * 8);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  // per streamed query tile: base-2 LSE, D, and each query's visible key interval
+  float* vec = reinterpret_cast<float*>(sm.base + C::kVecOff);     // [2][4][128]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  const int nkt = (p.Nk + kBT - 1) / kBT;
+  const int bk = blockIdx.x / nkt, kt = blockIdx.x % nkt;
+  const int b = bk / p.Hkv, hk = bk % p.Hkv;
+  const int k0 = kt * kBT;
+  const int k1 = min(k0 + kBT, p.Nk) - 1;
+  int qa, qb;
+  query_range(p.mask, p.Nq, k0, k1, qa, qb);
+  int ia = 0, ni = 0;                 // query tiles [ia, ia + ni) of every head of the group
+  if (qa <= qb) {
+    ia = qa / kBT;
+    ni = qb / kBT - ia + 1;
+  }
+  const int n = ni * p.G;             // streamed tiles: head g of the group, query tile i
+
+  if (threadIdx.x == 0) {
+    mbar_init(sm.bar(BAR_STAT), 1);
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(sm.bar(BAR_FULL + s), 1);
+      mbar_init(sm.bar(BAR_EMPTY + s), 1);
+    }
+    mbar_init(sm.bar(BAR_S), 1);
+    mbar_init(sm.bar(BAR_P), 4);
+    mbar_init(sm.bar(BAR_ACC), 1);
+    mbar_init(sm.bar(BAR_DONE), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == kBwdMmaWarp) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == kBwdTmaWarp) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0 && n > 0) {
+      const int zkv = b * p.Hkv + hk;
+      mbar_arrive_expect_tx(sm.bar(BAR_STAT), 2 * C::kTileBytes);
+#pragma unroll
+      for (int c = 0; c < C::kChunks; ++c) {
+        tma_load_3d(sm.stat + c * C::kChunkBytes, &tmK, sm.bar(BAR_STAT), c * 64, k0, zkv);
+        tma_load_3d(sm.stat + C::kTileBytes + c * C::kChunkBytes, &tmV, sm.bar(BAR_STAT),
+                    c * 64, k0, zkv);
+      }
+      int t = 0;
+      for (; t < n; ++t) {
+        const int s = t % NS, round = t / NS;
+        if (round > 0 &&
+            !mbar_wait(sm.bar(BAR_EMPTY + s), (round - 1) & 1, abort_flag, p.err, kSiteBwdEmpty))
+          break;
+        const int h = hk * p.G + t / ni;
+        const int row = (ia + t % ni) * kBT;
+        const int zq = b * p.Hq + h;
+        mbar_arrive_expect_tx(sm.bar(BAR_FULL + s), 2 * C::kTileBytes);
+        const uint32_t dst = sm.ring + s * 2 * C::kTileBytes;
+#pragma unroll
+        for (int c = 0; c < C::kChunks; ++c) {
+          tma_load_3d(dst + c * C::kChunkBytes, &tmQ, sm.bar(BAR_FULL + s), c * 64, row, zq);
+          tma_load_3d(dst + C::kTileBytes + c * C::kChunkBytes, &tmDO, sm.bar(BAR_FULL + s),
+                      c * 64, row, zq);
+        }
+      }
+      mbar_wait(sm.bar(BAR_STAT), 0, nullptr, p.err, kSiteBwdDrain);
+      for (int s = 0; s < NS && s < t; ++s) {
+        const int last = s + ((t - 1 - s) / NS) * NS;
+        mbar_wait(sm.bar(BAR_FULL + s), (last / NS) & 1, nullptr, p.err, kSiteBwdDrain);
+      }
+    }
+    __syncwarp();
+  } else if (warp == kBwdMmaWarp) {
+    // -------------------------------------------------------------- tcgen05 issuer
+    if (n > 0) {
+      bool ok = mbar_wait_warp(sm.bar(BAR_STAT), 0, abort_flag, p.err, kSiteBwdStat);
+      tc_fence_after();
+      for (int t = 0; ok && t < n; ++t) {
+        const int s = t % NS;
+        if (!mbar_wait_warp(sm.bar(BAR_FULL + s), (t / NS) & 1, abort_flag, p.err, kSiteBwdFull))
+          break;
+        tc_fence_after();
+        const uint32_t qt = sm.ring + s * 2 * C::kTileBytes;
+        issue_ss<D>(tmem + kTmemX, sm.stat, qt);                              // S^T = K Q^T
+        issue_ss<D>(tmem + kTmemY, sm.stat + C::kTileBytes, qt + C::kTileBytes);  // dP^T
+        umma_commit_warp(sm.bar(BAR_S));
+        if (!mbar_wait_warp(sm.bar(BAR_P), t & 1, abort_flag, p.err, kSiteBwdP)) break;
+        tc_fence_after();
+        issue_ts<D>(tmem + kTmemAcc0, tmem + kTmemX, qt + C::kTileBytes, t == 0);  // dV
+        issue_ts<D>(tmem + kTmemAcc1, tmem + kTmemY, qt, t == 0);                 // dK
+        umma_commit_warp(sm.bar(BAR_EMPTY + s));
+      }
+      umma_commit_warp(sm.bar(BAR_ACC));
+    }
+    umma_commit_warp(sm.bar(BAR_DONE));
+    mbar_wait_warp(sm.bar(BAR_DONE), 0, nullptr, p.err, kSiteBwdDrain);
+  } else {
+    // ------------------------------------------------------ element-wise warpgroup
+    const int wq = warp;
+    const int r = wq * 32 + lane;
+    const int key = k0 + r;
+    const bool kvalid = key < p.Nk;
+    const uint32_t tl = tmem + ((uint32_t)(wq * 32) << 16);
+    const long long kidx = ((long long)b * p.Hkv + hk) * p.Nk + key;
+    bool ok = true;
+    for (int t = 0; t < n; ++t) {
+      // this tile's query vectors; the barrier also makes the four warps agree to go on
+      const int par = t & 1;
+      const int h = hk * p.G + t / ni;
+      const int q0 = (ia + t % ni) * kBT;
+      {
+        const int q = q0 + r;
+        float l2q = INFINITY, dq = 0.f;
+        int lo = 1, hi = 0;
+        if (q < p.Nq) {
+          const long long qi = ((long long)b * p.Hq + h) * p.Nq + q;
+          l2q = p.l2[qi];
+          dq = p.dvec[qi];
+          row_interval(p.mask, q, lo, hi);
+        }
+        vec[(par * 4 + 0) * kBT + r] = l2q;
+        vec[(par * 4 + 1) * kBT + r] = dq;
+        vec[(par * 4 + 2) * kBT + r] = __int_as_float(lo);
+        vec[(par * 4 + 3) * kBT + r] = __int_as_float(hi);
+      }
+      uint32_t all_ok;
+      asm volatile("{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
+                   "bar.red.and.pred q, 1, 128, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+                   : "=r"(all_ok) : "r"(ok ? 1u : 0u) : "memory");
+      if (!all_ok) { ok = false; break; }
+      ok = __all_sync(0xffffffffu, mbar_wait(sm.bar(BAR_S), t & 1, abort_flag, p.err, kSiteBwdS));
+      if (!ok) continue;      // the next barrier ends the loop for all four warps
+      tc_fence_after();
+      const float* l2v = vec + (par * 4 + 0) * kBT;
+      const float* dv = vec + (par * 4 + 1) * kBT;
+      const int* lov = reinterpret_cast<const int*>(vec + (par * 4 + 2) * kBT);
+      const int* hiv = reinterpret_cast<const int*>(vec + (par * 4 + 3) * kBT);
+      const int qlast = min(q0 + kBT, p.Nq) - 1 - q0;
+      const bool full = q0 + kBT <= p.Nq && k0 + kBT <= p.Nk && lov[qlast] <= k0 &&
+                        k1 <= hiv[0];
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        uint32_t s[32], dp[32], pk[16], dsk[16];
+        tmem_ld_x32(tl + kTmemX + 32u * c, s);
+        tmem_ld_x32(tl + kTmemY + 32u * c, dp);
+        const int qc = 32 * c;
+        grad_chunk<true>(
+            s, dp, p.kscale,
+            [&](int i) {
+              return full || (kvalid && lov[qc + i] <= key && key <= hiv[qc + i]);
+            },
+            [&](int i) { return l2v[qc + i]; }, [&](int i) { return dv[qc + i]; }, pk, dsk);
+        tmem_st_x16(tl + kTmemX + 16u * c, pk);
+        tmem_st_x16(tl + kTmemY + 16u * c, dsk);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(sm.bar(BAR_P));
+    }
+    __nv_bfloat16* dvrow = reinterpret_cast<__nv_bfloat16*>(p.dv) + kidx * D;
+    __nv_bfloat16* dkrow = reinterpret_cast<__nv_bfloat16*>(p.dk) + kidx * D;
+    if (n == 0) {
+      store_zero_row(dvrow, D, kvalid);
+      store_zero_row(dkrow, D, kvalid);
+    } else if (ok) {
+      const bool okacc =
+          __all_sync(0xffffffffu, mbar_wait(sm.bar(BAR_ACC), 0, abort_flag, p.err, kSiteBwdAcc));
+      if (okacc) {
+        tc_fence_after();
+        store_row<D>(tl + kTmemAcc0, 1.f, dvrow, kvalid);
+        store_row<D>(tl + kTmemAcc1, p.scale, dkrow, kvalid);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kBwdMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+template <int D>
+int launch_bwd_t(const CUtensorMap& tq, const CUtensorMap& tdo, const CUtensorMap& tk,
+                 const CUtensorMap& tv, const BwdParams& p, cudaStream_t stream) {
+  using C = BwdCfg<D>;
+  static_assert(C::kSmemBytes <= 227 * 1024, "shared memory budget");
+  if (cudaFuncSetAttribute(attn_bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           C::kSmemBytes) != cudaSuccess ||
+      cudaFuncSetAttribute(attn_bwd_dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           C::kSmemBytes) != cudaSuccess)
+    return -4;
+  const long long nq = (long long)p.B * p.Hq * ((p.Nq + kBT - 1) / kBT);
+  const long long nk = (long long)p.B * p.Hkv * ((p.Nk + kBT - 1) / kBT);
+  if (nk > 0)
+    attn_bwd_dkdv_kernel<D><<<(unsigned)nk, kBwdThreads, C::kSmemBytes, stream>>>(tq, tdo, tk,
+                                                                                 tv, p);
+  if (nq > 0)
+    attn_bwd_dq_kernel<D><<<(unsigned)nq, kBwdThreads, C::kSmemBytes, stream>>>(tq, tdo, tk,
+                                                                               tv, p);
+  return cudaGetLastError() == cudaSuccess ? 0 : -4;
+}
+
+}  // namespace
+
+int launch_bwd_rowdot(const void* o, const void* dout, const float* lse, float* dvec, float* l2,
+                      long long rows, int d, cudaStream_t stream) {
+  if (rows <= 0) return 0;
+  const int warps = 8;
+  const long long blocks = (rows + warps - 1) / warps;
+  attn_bwd_rowdot_kernel<<<(unsigned)blocks, warps * 32, 0, stream>>>(
+      reinterpret_cast<const __nv_bfloat16*>(o), reinterpret_cast<const __nv_bfloat16*>(dout),
+      lse, dvec, l2, rows, d);
+  return cudaGetLastError() == cudaSuccess ? 0 : -4;
+}
+
+int launch_attn_bwd(const CUtensorMap& tq, const CUtensorMap& tdo, const CUtensorMap& tk,
+                    const CUtensorMap& tv, const BwdParams& p, int d, cudaStream_t stream) {
+  if (d == 128) return launch_bwd_t<128>(tq, tdo, tk, tv, p, stream);
+  if (d == 64) return launch_bwd_t<64>(tq, tdo, tk, tv, p, stream);
+  return -2;
+}
+
+}  // namespace attn

@@ -41,6 +41,20 @@ struct DecParams {
   int max_pages;            // pages per block-table row
 };
 
+struct BwdParams {
+  void* dq;           // bf16 [B, Hq, Nq, d]  (written)
+  void* dk;           // bf16 [B, Hkv, Nk, d] (written)
+  void* dv;           // bf16 [B, Hkv, Nk, d] (written)
+  const float* dvec;  // fp32 [B, Hq, Nq]: rowsum(dO * O)
+  const float* l2;    // fp32 [B, Hq, Nq]: LSE * log2(e), +inf for rows without a key
+  int B, Hq, Hkv, Nq, Nk;
+  int G;              // Hq / Hkv
+  float kscale;       // scale * log2(e)
+  float scale;
+  MaskParams mask;
+  uint32_t* err;      // device error word of the library (bits, first site)
+};
+
 int launch_attn_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                     const FwdParams& p, int d, cudaStream_t stream);
 int launch_fill_empty(void* o, float* lse, size_t rows, int d, cudaStream_t stream);
@@ -49,6 +63,10 @@ int launch_blockmap(const MaskParams& m, int B, int Nq, int Nk, uint8_t* map,
 int launch_decode_split(const CUtensorMap& tk, const CUtensorMap& tv, const DecParams& p,
                         int d, int G, int grid, cudaStream_t stream);
 int decode_ctas_per_sm(int d, int G);
+int launch_bwd_rowdot(const void* o, const void* dout, const float* lse, float* dvec, float* l2,
+                      long long rows, int d, cudaStream_t stream);
+int launch_attn_bwd(const CUtensorMap& tq, const CUtensorMap& tdo, const CUtensorMap& tk,
+                    const CUtensorMap& tv, const BwdParams& p, int d, cudaStream_t stream);
 int launch_merge(const float* o_part, const float* lse_part, void* o, float* lse, long long rows,
                  int S, int d, cudaStream_t stream);
 

@@ -38,6 +38,13 @@ def prefill_useful_flops(B: int, Hq: int, Nq: int, Nk: int, d: int, mask_kind: i
     return 4 * d * visible_pairs(Nq, Nk, mask_kind, window, doc_offsets) * B * Hq
 
 
+def backward_useful_flops(B: int, Hq: int, Nq: int, Nk: int, d: int, mask_kind: int,
+                          window: int = 0, doc_offsets=None) -> int:
+    """Useful FLOPs of the backward pass: five products per visible pair (S recomputed,
+    dP = dO V^T, dV = P^T dO, dQ = dS K, dK = dS^T Q), 2 d flops each."""
+    return 10 * d * visible_pairs(Nq, Nk, mask_kind, window, doc_offsets) * B * Hq
+
+
 def decode_kv_bytes(B: int, Hkv: int, T: int, d: int, elem_bytes: int = 2) -> int:
     """Bytes of K plus V read by one decode step (each cache byte read once)."""
     return 2 * B * Hkv * T * d * elem_bytes
