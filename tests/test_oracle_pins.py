@@ -638,3 +638,71 @@ def test_backward_invariants():
                                               window=w)
         assert np.allclose(dq, dq2, atol=1e-12, rtol=0)
         assert np.allclose(dv.sum(axis=2)[0, 0], dout.sum(axis=(1, 2))[0], atol=1e-12, rtol=0)
+
+
+# ------------------------------------------------------------------------ FP8 inputs
+
+from oracle import fp8 as ofp8  # noqa: E402
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_rotation_is_orthogonal_and_keeps_the_scores(d):
+    H = ofp8.hadamard(d)
+    assert np.array_equal(H @ H.T, d * np.eye(d))
+    assert set(np.unique(H)) == {-1.0, 1.0}
+    rng = np.random.default_rng(d)
+    signs = rng.choice([-1.0, 1.0], size=d)
+    q = rng.standard_normal((7, d))
+    k = rng.standard_normal((9, d))
+    assert np.allclose(ofp8.rotate(q, signs) @ ofp8.rotate(k, signs).T, q @ k.T, atol=1e-12)
+    # an outlier column is spread over all columns (incoherence): max |x| drops by sqrt(d)
+    x = np.zeros((1, d))
+    x[0, 3] = 10.0
+    assert np.allclose(np.abs(ofp8.rotate(x, signs)), 10.0 / np.sqrt(d))
+
+
+def test_e4m3_grid_points_and_error_bounds():
+    # the largest finite E4M3 value is 448; 1 + 2^-3 is a grid point, 1 + 2^-4 a tie that
+    # rounds to even (1); normal values round within 2^-4 relative, subnormals (below 2^-6)
+    # within half their spacing 2^-9
+    vals = ofp8.to_e4m3(np.array([448.0, 1.125, 1.0625, 1.1875, -3.0, 2 ** -9, 2 ** -6]))
+    assert list(vals) == [448.0, 1.125, 1.0, 1.25, -3.0, 2 ** -9, 2 ** -6]
+    x = np.random.default_rng(3).standard_normal(100000) * 50
+    r = ofp8.to_e4m3(x)
+    normal = np.abs(x) >= 2 ** -6
+    assert np.all(np.abs(r - x)[normal] <= 2 ** -4 * np.abs(x)[normal] + 1e-12)
+    assert np.all(np.abs(r - x)[~normal] <= 2 ** -10 + 1e-12)
+
+
+def test_block_quantization_uses_the_full_range_per_block():
+    rng = np.random.default_rng(4)
+    x = rng.standard_normal((2, 3, 300, 16)) * np.array([1.0, 100.0, 0.01])[None, :, None, None]
+    x[1, 2, 128:256] = 0.0                                   # an all-zero block
+    codes, scales = ofp8.quantize_blocks(x, 128)
+    assert scales.shape == (2, 3, 3) and scales[1, 2, 1] == 1.0
+    assert np.all(codes[1, 2, 128:256] == 0.0)
+    for b in range(2):
+        for h in range(3):
+            for i in range(3):
+                blk = codes[b, h, i * 128:(i + 1) * 128]
+                if scales[b, h, i] != 1.0 or np.any(blk):
+                    assert np.abs(blk).max() == 448.0        # the block's amax maps to 448
+    deq = ofp8.dequantize_blocks(codes, scales, 128)
+    rep = np.repeat(scales, 128, axis=2)[:, :, :300, None]
+    assert np.all(np.abs(deq - x) <= 2 ** -4 * np.abs(x) + rep * 2 ** -10 + 1e-12)
+
+
+def test_fp8_attention_is_attention_of_the_dequantized_values():
+    rng = np.random.default_rng(5)
+    q, k, v = (rng.standard_normal((1, 2, 200, 16)) for _ in range(3))
+    qc, qs = ofp8.quantize_blocks(q, 128)
+    kc, ks = ofp8.quantize_blocks(k, 128)
+    vc, vs = ofp8.quantize_blocks(v, 200)                    # one scale per head
+    O, lse = ofp8.attention_fp8(qc, qs, kc, ks, vc, vs[:, :, 0], scale=0.25, mask_kind=1)
+    O2, lse2 = oracle.attention(ofp8.dequantize_blocks(qc, qs, 128),
+                                ofp8.dequantize_blocks(kc, ks, 128),
+                                ofp8.dequantize_blocks(vc, vs, 200), scale=0.25, mask_kind=1)
+    assert np.array_equal(O, O2) and np.array_equal(lse, lse2)
+    # causal row 0 sees only key 0: O = the dequantized v_0, within E4M3 rounding of v_0
+    assert np.all(np.abs(O[0, :, 0] - v[0, :, 0]) <= 2 ** -4 * np.abs(v[0, :, 0])
+                  + vs[0, :, 0, None] * 2 ** -10 + 1e-12)
