@@ -332,6 +332,8 @@ def run_ours(args, world, rank, local):
             args, world, local, peaks, peak_src)
         out["extras"]["backward_" + workloads.CAUSAL_MHA.name] = bench_backward(
             workloads.CAUSAL_MHA, args, world, local, peaks, peak_src)
+        out["extras"]["fp8_" + workloads.CAUSAL_MHA.name] = bench_fp8(
+            workloads.CAUSAL_MHA, args, world, local, peaks, peak_src)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         tf, heads, dt = oracle_prefill_sample(w, args.cpu_budget)
         out["cpu_baseline"] = {"value": round(tf, 5), "unit": "TFLOP/s",
@@ -471,6 +473,64 @@ def bench_backward(w, args, world, local, peaks, peak_src):
                         "peak_source": f"bf16_tflops (burst, {peak_src})", "traffic": None},
            "gpu_launches": 3 * steps, "clocks": clk.summary()}
     del q, k, v, o, lse, dout, dq, dk, dv, ws
+    torch.cuda.empty_cache()
+    return res
+
+
+def bench_fp8(w, args, world, local, peaks, peak_src):
+    """Useful TFLOP/s of attn_fwd_fp8 on a prefill workload: Q and K quantized per 128-row
+    block after the seeded random-sign Hadamard rotation, V per head and transposed; the
+    quantization runs before the timed region and is timed on its own."""
+    import torch
+    import io_aware_softmax_b200 as attn
+    dev = torch.device("cuda", torch.cuda.current_device())
+    q, k, v = workloads.make_inputs(w, device=dev)
+    signs = torch.from_numpy(np.random.default_rng(w.seed).choice([-1.0, 1.0], w.d)
+                             .astype(np.float32)).to(dev)
+
+    def quant():
+        q8, qs = attn.quantize_fp8(q, block_rows=128, signs=signs)
+        k8, ks = attn.quantize_fp8(k, block_rows=128, signs=signs)
+        vt8, vs = attn.quantize_fp8(v, block_rows=w.Nk, transpose=True)
+        return q8, qs, k8, ks, vt8, vs[:, :, 0].contiguous()
+
+    for _ in range(2):
+        inputs = quant()
+    torch.cuda.synchronize()
+    qt_ms, _ = time_launches(quant, 3, world)
+    q8, qs, k8, ks, vt8, vs = inputs
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.Hq, w.Nq), dtype=torch.float32, device=dev)
+    flops = accounting.prefill_useful_flops(w.B, w.Hq, w.Nq, w.Nk, w.d, w.mask_kind, w.window)
+
+    def step():
+        attn.attn_fwd_fp8(q8, qs, k8, ks, vt8, vs, scale=w.scale, mask=w.mask_kind,
+                          window=w.window, out=o, lse=lse)
+
+    steps = max(3, min(args.steps, 30))
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        total_ms, per = time_launches(step, steps, world)
+    if attn.device_status() != 0:
+        raise RuntimeError("device status not ok after the FP8 prefill")
+    ms = max_over_ranks(world, total_ms / steps)
+    call_ms = max_over_ranks(world, sum(per) / len(per))
+    peak = 2.0 * float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    achieved = flops / (call_ms * 1e-3) / 1e12
+    res = {"config": {**w.describe(), "dtype": "e4m3 (P e4m3), bf16 O",
+                      "scales": "Q, K per 128 rows after Hadamard rotation; V per head"},
+           "value": round(whole_job_rate(flops, world, ms) / 1e12, 2), "unit": "TFLOP/s",
+           "ms_per_step": round(ms, 4), "steps": steps,
+           "quantize_ms": round(max_over_ranks(world, qt_ms / 3), 4),
+           "useful_tflop_per_step": round(flops / 1e12, 4),
+           "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak,
+                        "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                        "peak_source": f"2 x bf16_tflops (burst, {peak_src}): the nominal "
+                                       "fp8 / bf16 ratio", "traffic": None},
+           "gpu_launches": steps, "clocks": clk.summary()}
+    del q, k, v, q8, k8, vt8, o, lse
     torch.cuda.empty_cache()
     return res
 

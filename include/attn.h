@@ -123,6 +123,43 @@ ATTN_API int attn_bwd(const void* q, const void* k, const void* v, const void* o
              cudaStream_t stream);
 
 /*
+ * attn_quantize_fp8 -- block quantization to E4M3 ("FlashAttention 논문 분석", section
+ * "FP8 지원과 정확도 유지": an independent scale per block; Q and K optionally multiplied by a
+ * random orthogonal matrix first, which leaves Q K^T unchanged).
+ *   x        bf16 [B, H, N, d], d in {64, 128}
+ *   signs    NULL, or device fp32 [d] of +-1: rows become (x * signs) H / sqrt(d), H the
+ *            Sylvester Hadamard matrix (use the same signs for Q and K)
+ *   block_rows  rows per scale; scales fp32 [B, H, ceil(N / block_rows)] (written):
+ *            amax / 448 of the (rotated) block, 1 for an all-zero block
+ *   out      E4M3 codes (written) of x * (448 / amax), round to nearest even, saturating:
+ *            transpose = 0: [B, H, N, d]; transpose = 1: [B, H, d, n_pad] with columns
+ *            [N, n_pad) zero (the layout attn_fwd_fp8 takes for V)
+ * Errors: INVALID_ARG, UNSUPPORTED (d), MISALIGNED (x 16 bytes; scales, signs and a
+ * row-major out 4 bytes), CUDA.
+ */
+ATTN_API int attn_quantize_fp8(const void* x, void* out, float* scales, int B, int H, int N, int d,
+                      int block_rows, int transpose, int n_pad, const float* signs,
+                      cudaStream_t stream);
+
+/*
+ * attn_fwd_fp8 -- attn_fwd on E4M3 inputs (the FP8 tensor-core path of "FlashAttention 논문
+ * 분석", sections "FP8 텐서 코어" and "FP8 지원과 정확도 유지").  The result is attention of
+ * the dequantized values: Q = q8 * q_scales (per 128-row block), K = k8 * k_scales (per
+ * 128-row block), V = vt8^T * v_scales (per head).  Both products run on E4M3 operands;
+ * P is rounded to E4M3 (as 64 P, the lazy-rescale bound being 2^2).
+ *   q8       E4M3 [B, Hq, Nq, 128]            q_scales  fp32 [B, Hq, ceil(Nq / 128)]
+ *   k8       E4M3 [B, Hkv, Nk, 128]           k_scales  fp32 [B, Hkv, ceil(Nk / 128)]
+ *   vt8      E4M3 [B, Hkv, 128, nk_pad] (V transposed; nk_pad >= Nk, a multiple of 16)
+ *   v_scales fp32 [B, Hkv]
+ *   o, lse, scale, masks as attn_fwd (no soft-cap); d must be 128.
+ * Errors: as attn_fwd; UNSUPPORTED for d != 128.
+ */
+ATTN_API int attn_fwd_fp8(const void* q8, const void* k8, const void* vt8, const float* q_scales,
+                 const float* k_scales, const float* v_scales, void* o, float* lse, int B,
+                 int Hq, int Hkv, int Nq, int Nk, int nk_pad, int d, float scale, int mask_kind,
+                 int window, const int* doc_offsets, int num_docs, cudaStream_t stream);
+
+/*
  * attn_blockmap -- 128x128 block-sparsity map of a mask ("PyTorch FlexAttention 도입 분석",
  * section 2: BlockMask precomputed in 128 x 128 chunks so empty tiles are skipped).
  *   map  device uint8 [B, ceil(Nq/128), ceil(Nk/128)] (written): ATTN_TILE_EMPTY when no

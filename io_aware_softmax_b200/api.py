@@ -135,6 +135,62 @@ def attn_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,
     return dq, dk, dv
 
 
+def quantize_fp8(x: torch.Tensor, *, block_rows: int = 128, transpose: bool = False,
+                 n_pad: Optional[int] = None, signs: Optional[torch.Tensor] = None,
+                 stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """E4M3 block quantization of x [B,H,N,d] bf16 -> (codes float8_e4m3fn, scales fp32
+    [B,H,ceil(N/block_rows)]); codes are [B,H,N,d], or [B,H,d,n_pad] when transposed (V)."""
+    lib = _lib.load()
+    _need(x, "x", torch.bfloat16, 4)
+    B, H, N, d = x.shape
+    if signs is not None:
+        _need(signs, "signs", torch.float32, 1)
+    if transpose:
+        n_pad = -(-N // 16) * 16 if n_pad is None else int(n_pad)
+        out = torch.empty((B, H, d, n_pad), dtype=torch.float8_e4m3fn, device=x.device)
+    else:
+        n_pad = 0
+        out = torch.empty((B, H, N, d), dtype=torch.float8_e4m3fn, device=x.device)
+    scales = torch.empty((B, H, -(-N // block_rows)), dtype=torch.float32, device=x.device)
+    st = lib.attn_quantize_fp8(_ptr(x), _ptr(out), _ptr(scales), B, H, N, d, int(block_rows),
+                               int(bool(transpose)), n_pad, _ptr(signs), _stream(x.device, stream))
+    _check(st, "attn_quantize_fp8")
+    return out, scales
+
+
+def attn_fwd_fp8(q8: torch.Tensor, q_scales: torch.Tensor, k8: torch.Tensor,
+                 k_scales: torch.Tensor, vt8: torch.Tensor, v_scales: torch.Tensor, *,
+                 scale: Optional[float] = None, mask="none", window: int = 0,
+                 doc_offsets: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
+                 lse: Optional[torch.Tensor] = None, stream=None
+                 ) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Prefill on E4M3 inputs: q8 [B,Hq,Nq,d], k8 [B,Hkv,Nk,d], vt8 [B,Hkv,d,nk_pad] with
+    per-block scales (q, k: [.., ceil(N/128)]) and per-head V scales [B,Hkv] -> (O, LSE)."""
+    lib = _lib.load()
+    for t, n in ((q8, "q8"), (k8, "k8"), (vt8, "vt8")):
+        _need(t, n, torch.float8_e4m3fn, 4)
+    B, Hq, Nq, d = q8.shape
+    Hkv, Nk = k8.shape[1], k8.shape[2]
+    nk_pad = vt8.shape[3]
+    for t, n, dims in ((q_scales, "q_scales", 3), (k_scales, "k_scales", 3),
+                       (v_scales, "v_scales", 2)):
+        _need(t, n, torch.float32, dims)
+    if out is None:
+        out = torch.empty((B, Hq, Nq, d), dtype=torch.bfloat16, device=q8.device)
+    if lse is None:
+        lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q8.device)
+    num_docs = 0
+    if doc_offsets is not None:
+        _need(doc_offsets, "doc_offsets", torch.int32, 1)
+        num_docs = doc_offsets.numel() - 1
+    st = lib.attn_fwd_fp8(_ptr(q8), _ptr(k8), _ptr(vt8), _ptr(q_scales), _ptr(k_scales),
+                          _ptr(v_scales), _ptr(out), _ptr(lse), B, Hq, Hkv, Nq, Nk, nk_pad, d,
+                          float(scale or 0.0), _mask_id(mask), int(window), _ptr(doc_offsets),
+                          num_docs, _stream(q8.device, stream))
+    _check(st, "attn_fwd_fp8")
+    return out, lse
+
+
 def attn_blockmap(B: int, Nq: int, Nk: int, *, mask="none", window: int = 0,
                   doc_offsets: Optional[torch.Tensor] = None, device=None,
                   out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:

@@ -38,6 +38,23 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
+// 3-D tensor map of bytes over [z, rows, inner] (inner = `extent` valid bytes of each
+// `stride`-byte row) with a (128 x box_rows x 1) box and 128-byte swizzle; bytes past the
+// extent read as zero.
+bool make_map_3d_u8(CUtensorMap* map, const void* ptr, long long extent, long long stride,
+                    long long rows, long long z, int box_rows) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)extent, (cuuint64_t)rows, (cuuint64_t)z};
+  cuuint64_t strides[2] = {(cuuint64_t)stride, (cuuint64_t)stride * (cuuint64_t)rows};
+  cuuint32_t box[3] = {128, (cuuint32_t)box_rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(ptr), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // 3-D bf16 tensor map over [z, rows, d] (d innermost) with a (64 x box_rows x 1) box and
 // 128-byte swizzle: one box fills `box_rows` rows of 128 bytes in shared memory.
 bool make_map_3d(CUtensorMap* map, const void* ptr, int d, long long rows, long long z,
@@ -159,7 +176,7 @@ extern "C" int attn_fwd_alibi(const void* q, const void* k, const void* v, void*
   if ((long long)B * Hq > (1LL << 31) - 1) return ATTN_ERR_UNSUPPORTED;
 
   if (scale <= 0.f) scale = 1.0f / std::sqrt((float)d);
-  FwdParams p;
+  FwdParams p{};
   p.o = o;
   p.lse = lse;
   p.B = B;
@@ -456,4 +473,78 @@ extern "C" int attn_bwd(const void* q, const void* k, const void* v, const void*
       !make_map_3d(&tv, v, d, Nk, (long long)B * Hkv, 128))
     return ATTN_ERR_CUDA;
   return launch_attn_bwd(tq, tdo, tk, tv, p, d, stream) == 0 ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+extern "C" int attn_quantize_fp8(const void* x, void* out, float* scales, int B, int H, int N,
+                                 int d, int block_rows, int transpose, int n_pad,
+                                 const float* signs, cudaStream_t stream) {
+  if (B < 0 || H < 0 || N < 0 || block_rows <= 0) return ATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (transpose && n_pad < N) return ATTN_ERR_INVALID_ARG;
+  if (B == 0 || H == 0 || N == 0) return ATTN_OK;
+  if (!x || !out || !scales) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(x) || (reinterpret_cast<uintptr_t>(scales) & 3u) ||
+      (reinterpret_cast<uintptr_t>(signs) & 3u))
+    return ATTN_ERR_MISALIGNED;
+  if (!transpose && (reinterpret_cast<uintptr_t>(out) & 3u)) return ATTN_ERR_MISALIGNED;
+  return launch_quantize_e4m3(x, out, scales, B, H, N, d, block_rows, transpose, n_pad, signs,
+                              stream) == 0
+             ? ATTN_OK
+             : ATTN_ERR_CUDA;
+}
+
+extern "C" int attn_fwd_fp8(const void* q8, const void* k8, const void* vt8,
+                            const float* q_scales, const float* k_scales, const float* v_scales,
+                            void* o, float* lse, int B, int Hq, int Hkv, int Nq, int Nk,
+                            int nk_pad, int d, float scale, int mask_kind, int window,
+                            const int* doc_offsets, int num_docs, cudaStream_t stream) {
+  if (B < 0 || Hq < 0 || Hkv < 0 || Nq < 0 || Nk < 0) return ATTN_ERR_INVALID_ARG;
+  if (d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (Hkv == 0 && Hq > 0) return ATTN_ERR_INVALID_ARG;
+  if (Hkv > 0 && Hq % Hkv != 0) return ATTN_ERR_UNSUPPORTED;
+  int st = check_mask(mask_kind, window, doc_offsets, num_docs, Nq, Nk);
+  if (st != ATTN_OK) return st;
+  if (std::isnan(scale)) return ATTN_ERR_INVALID_ARG;
+  if (nk_pad < Nk || (nk_pad & 15)) return ATTN_ERR_INVALID_ARG;
+  if (B == 0 || Hq == 0 || Nq == 0) return ATTN_OK;
+  if (!o || !lse || !q8 || !q_scales) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(o) || !aligned16(lse) || !aligned16(q8)) return ATTN_ERR_MISALIGNED;
+  const long long rows = (long long)B * Hq * Nq;
+  if (Nk == 0) return launch_fill_empty(o, lse, (size_t)rows, d, stream) == 0 ? ATTN_OK : ATTN_ERR_CUDA;
+  if (!k8 || !vt8 || !k_scales || !v_scales) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(k8) || !aligned16(vt8)) return ATTN_ERR_MISALIGNED;
+  if ((reinterpret_cast<uintptr_t>(q_scales) | reinterpret_cast<uintptr_t>(k_scales) |
+       reinterpret_cast<uintptr_t>(v_scales)) & 3u)
+    return ATTN_ERR_MISALIGNED;
+  if ((long long)B * Hq > (1LL << 31) - 1) return ATTN_ERR_UNSUPPORTED;
+
+  if (scale <= 0.f) scale = 1.0f / std::sqrt((float)d);
+  FwdParams p{};
+  p.o = o;
+  p.lse = lse;
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.Nq = Nq;
+  p.Nk = Nk;
+  p.G = Hq / Hkv;
+  p.num_pairs = (Nq + 255) / 256;
+  p.num_sms = sm_count(current_device());
+  p.kscale = scale * kLog2e;
+  p.mask = mask_params(mask_kind, window, doc_offsets, num_docs, Nq, Nk);
+  p.q_scales = q_scales;
+  p.k_scales = k_scales;
+  p.v_scales = v_scales;
+  p.nqt = (Nq + 127) / 128;
+  p.nkt = (Nk + 127) / 128;
+  if ((long long)p.num_pairs * B * Hq > (1LL << 31) - 1) return ATTN_ERR_UNSUPPORTED;
+  p.err = error_word_ptr(current_device());
+  if (p.err == nullptr) return ATTN_ERR_CUDA;
+
+  CUtensorMap tq, tk, tv;
+  if (!make_map_3d_u8(&tq, q8, d, d, Nq, (long long)B * Hq, 128) ||
+      !make_map_3d_u8(&tk, k8, d, d, Nk, (long long)B * Hkv, 128) ||
+      !make_map_3d_u8(&tv, vt8, Nk, nk_pad, d, (long long)B * Hkv, d))
+    return ATTN_ERR_CUDA;
+  return launch_attn_fwd(tq, tk, tv, p, d, stream) == 0 ? ATTN_OK : ATTN_ERR_CUDA;
 }

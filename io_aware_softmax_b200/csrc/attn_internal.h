@@ -23,6 +23,11 @@ struct FwdParams {
   float cap_log2;     // softcap * log2(e)
   MaskParams mask;
   const float* alibi; // fp32 [Hq] ALiBi slopes (natural-log units per key of distance) or null
+  // FP8 (E4M3) inputs, null otherwise: per 128-row block scales of Q and K, per head of V
+  const float* q_scales;  // fp32 [B, Hq, nqt]
+  const float* k_scales;  // fp32 [B, Hkv, nkt]
+  const float* v_scales;  // fp32 [B, Hkv]
+  int nqt, nkt;           // ceil(Nq / 128), ceil(Nk / 128)
   uint32_t* err;      // device error word of the library (bits, first site)
 };
 
@@ -67,6 +72,9 @@ int launch_bwd_rowdot(const void* o, const void* dout, const float* lse, float* 
                       long long rows, int d, cudaStream_t stream);
 int launch_attn_bwd(const CUtensorMap& tq, const CUtensorMap& tdo, const CUtensorMap& tk,
                     const CUtensorMap& tv, const BwdParams& p, int d, cudaStream_t stream);
+int launch_quantize_e4m3(const void* x, void* out, float* scales, int B, int H, int N, int d,
+                         int block_rows, int transpose, int n_pad, const float* signs,
+                         cudaStream_t stream);
 int launch_merge(const float* o_part, const float* lse_part, void* o, float* lse, long long rows,
                  int S, int d, cudaStream_t stream);
 

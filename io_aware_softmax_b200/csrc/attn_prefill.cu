@@ -57,12 +57,13 @@ constexpr float kLn2 = 0.69314718055994531f;
 constexpr float kLog2eF = 1.44269504088896341f;
 constexpr uint32_t kNegInfBits = 0xff800000u;
 
-template <int D>
+template <int D, bool kFp8 = false>
 struct Cfg {
-  static constexpr int kChunks = D / 64;            // 128-byte swizzle atoms along d
+  static constexpr int kElem = kFp8 ? 1 : 2;        // bytes per element (E4M3 or bf16)
+  static constexpr int kChunks = D * kElem / 128;   // 128-byte swizzle atoms along d
   static constexpr int kChunkBytes = kBM * 128;     // 128 rows x 128 bytes
-  static constexpr int kTileBytes = kBM * D * 2;    // one Q, K or V tile (bf16)
-  static constexpr int kStages = (D == 128) ? 4 : 8;
+  static constexpr int kTileBytes = kBM * D * kElem;  // one Q, K or V tile
+  static constexpr int kStages = (kTileBytes >= 32768) ? 4 : 8;
   static constexpr int kQOff = 0;
   static constexpr int kRingOff = 2 * kTileBytes;
   static constexpr int kBarOff = kRingOff + kStages * kTileBytes;
@@ -129,6 +130,33 @@ __device__ __forceinline__ void alibi_row(uint32_t (&s)[128], const FwdParams& p
     s[c] = __float_as_uint(t0);
     s[c + 1] = __float_as_uint(t1);
   }
+}
+
+// FP8 path: 2^(x - m_use + 6) = 64 P for one 64-column half of a tile row, packed four
+// per TMEM column as E4M3 (key 4c + i in byte i of column c); returns the half's fp32 sum
+// of P (the sum of 64 P divided by 64, exact).
+__device__ __forceinline__ float tile_row_exp_half_e4m3(const uint32_t (&s)[128], int base,
+                                                        float ks, float m_use,
+                                                        uint32_t (&pk)[16]) {
+  const float mu = m_use - 6.0f;
+  float a0 = 0.f, a1 = 0.f, b0 = 0.f, b1 = 0.f;
+#pragma unroll
+  for (int c = 0; c < 64; c += 4) {
+    float x0, x1, x2, x3;
+    ffma2(x0, x1, f32(s[base + c]), f32(s[base + c + 1]), ks, ks, -mu, -mu);
+    ffma2(x2, x3, f32(s[base + c + 2]), f32(s[base + c + 3]), ks, ks, -mu, -mu);
+    const float e0 = ex2_approx(x0), e1 = ex2_approx(x1);
+    const float e2 = ex2_approx(x2), e3 = ex2_approx(x3);
+    if ((c >> 2) & 1) {
+      add2(b0, b1, e0, e1);
+      add2(b0, b1, e2, e3);
+    } else {
+      add2(a0, a1, e0, e1);
+      add2(a0, a1, e2, e3);
+    }
+    pk[c >> 2] = pack_e4m3x4(e0, e1, e2, e3);
+  }
+  return (((a0 + a1) + (b0 + b1)) * (1.0f / 64.0f));
 }
 
 // P = 2^(x - m_use) for one 64-column half of a tile row, packed as bf16 pairs; returns
@@ -226,13 +254,18 @@ __device__ __forceinline__ void for_each_pair(const FwdParams& p, F&& f) {
   }
 }
 
-template <int D, bool kAlibi>
+template <int D, bool kAlibi, bool kFp8>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
                       const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
-  using C = Cfg<D>;
+  using C = Cfg<D, kFp8>;
   constexpr int NS = C::kStages;
+  static_assert(!(kFp8 && (kAlibi || D != 128)), "FP8 path: d = 128, no bias");
+  // FP8: the lazy-rescale bound is 2^2 and P is stored as E4M3 of 64 P (<= 256 < 448), so
+  // probabilities down to 2^-12 of the reference stay in E4M3's normal range.
+  constexpr float kThreshold = kFp8 ? 2.0f : kRescaleThreshold;
+  constexpr float kPScale = 64.0f;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_u32 = smem_u32(smem_raw);
   const uint32_t base_u32 = (raw_u32 + 1023u) & ~1023u;
@@ -297,10 +330,15 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
           mbar_arrive_expect_tx(bar(BAR_FULL + s), C::kTileBytes);
           const int row = (w.jt0 + (i >> 1)) * kBN;
           const CUtensorMap* m = (i & 1) ? &tmV : &tmK;
+          if (kFp8 && (i & 1)) {
+            // FP8 V is stored transposed ([d][keys] per head): one box of d rows x 128 keys
+            tma_load_3d(sRing + s * C::kTileBytes, m, bar(BAR_FULL + s), row, 0, zkv);
+          } else {
 #pragma unroll
-          for (int c = 0; c < C::kChunks; ++c)
-            tma_load_3d(sRing + s * C::kTileBytes + c * C::kChunkBytes, m, bar(BAR_FULL + s),
-                        c * 64, row, zkv);
+            for (int c = 0; c < C::kChunks; ++c)
+              tma_load_3d(sRing + s * C::kTileBytes + c * C::kChunkBytes, m, bar(BAR_FULL + s),
+                          c * (128 / C::kElem), row, zkv);
+          }
           ++issued;
         }
         return true;
@@ -329,7 +367,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
 #pragma unroll
           for (int c = 0; c < C::kChunks; ++c)
             tma_load_3d(sQ + t * C::kTileBytes + c * C::kChunkBytes, &tmQ, bar(BAR_Q + t),
-                        c * 64, w.q_first + t * kBM, w.b * p.Hq + w.h);
+                        c * (128 / C::kElem), w.q_first + t * kBM, w.b * p.Hq + w.h);
         }
         ++pairs;
         return true;
@@ -344,34 +382,51 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
     // The whole warp runs this role with warp-uniform values and one elected lane issues
     // each tensor-core operation, so descriptors stay in the uniform datapath.
     {
-      constexpr uint32_t idesc_qk = idesc_bf16_f32(kBM, kBN, false);
-      constexpr uint32_t idesc_pv = idesc_bf16_f32(kBM, D, true);
+      constexpr uint32_t idesc_qk =
+          kFp8 ? idesc_e4m3_f32(kBM, kBN) : idesc_bf16_f32(kBM, kBN, false);
+      constexpr uint32_t idesc_pv = kFp8 ? idesc_e4m3_f32(kBM, D) : idesc_bf16_f32(kBM, D, true);
       // Descriptors differ only in their start-address field (address >> 4, 14 bits; the
       // CTA's shared memory stays below 2^18 bytes, so adding an offset never carries out
       // of it): keep three base descriptors and add offsets in 16-byte units.
       const uint64_t dQ = smem_desc(sQ, 16, 1024);
       const uint64_t dK = smem_desc(sRing, 16, 1024);
-      const uint64_t dV = smem_desc(sRing, C::kChunkBytes, 1024);
+      // bf16 V is MN-major (d along the 128-byte rows); FP8 V^T is K-major like K
+      const uint64_t dV = kFp8 ? smem_desc(sRing, 16, 1024) : smem_desc(sRing, C::kChunkBytes, 1024);
       auto issue_qk = [&](int t, int sk) {
         const uint32_t d_tmem = tmem + 128u * t;
         const uint32_t q_off = (uint32_t)(t * C::kTileBytes) >> 4;
         const uint32_t k_off = (uint32_t)(sk * C::kTileBytes) >> 4;
+        // one k-step reads 32 bytes of every row: 16 bf16 or 32 E4M3 values
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
+        for (int kk = 0; kk < D * C::kElem / 32; ++kk) {
           const uint32_t off = ((kk >> 2) * C::kChunkBytes + (kk & 3) * 32) >> 4;
-          umma_ss_warp(d_tmem, dQ + q_off + off, dK + k_off + off, idesc_qk, kk > 0 ? 1u : 0u);
+          if constexpr (kFp8)
+            umma_ss_f8_warp(d_tmem, dQ + q_off + off, dK + k_off + off, idesc_qk, kk > 0 ? 1u : 0u);
+          else
+            umma_ss_warp(d_tmem, dQ + q_off + off, dK + k_off + off, idesc_qk, kk > 0 ? 1u : 0u);
         }
       };
       // O_t += P_t[:, 64h : 64h + 64] V_j[64h : 64h + 64]: key half h of the PV product.
       auto issue_pv_half = [&](int t, int sv, int h, bool first) {
         const uint32_t d_tmem = tmem + 256u + 128u * t;
-        const uint32_t a_tmem = tmem + 128u * t + 64u;
         const uint32_t v_off = (uint32_t)(sv * C::kTileBytes) >> 4;
+        if constexpr (kFp8) {
+          // E4M3 P: four keys per TMEM column in S columns [96, 128); a k-step is 32 keys
+          const uint32_t a_tmem = tmem + 128u * t + 96u;
 #pragma unroll
-        for (int k = 0; k < kBN / 32; ++k) {
-          const int kk = h * (kBN / 32) + k;
-          umma_ts_warp(d_tmem, a_tmem + 8u * kk, dV + v_off + ((kk * 16 * 128) >> 4), idesc_pv,
-                       (!first || kk > 0) ? 1u : 0u);
+          for (int k = 0; k < kBN / 64; ++k) {
+            const int kk = h * (kBN / 64) + k;
+            umma_ts_f8_warp(d_tmem, a_tmem + 8u * kk, dV + v_off + ((kk * 32) >> 4), idesc_pv,
+                            (!first || kk > 0) ? 1u : 0u);
+          }
+        } else {
+          const uint32_t a_tmem = tmem + 128u * t + 64u;
+#pragma unroll
+          for (int k = 0; k < kBN / 32; ++k) {
+            const int kk = h * (kBN / 32) + k;
+            umma_ts_warp(d_tmem, a_tmem + 8u * kk, dV + v_off + ((kk * 16 * 128) >> 4), idesc_pv,
+                         (!first || kk > 0) ? 1u : 0u);
+          }
         }
       };
       int pairs = 0;        // pairs started
@@ -477,6 +532,11 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
       row_interval(p.mask, row, row_lo, row_hi);
       // ALiBi slope of this head in base-2 units (0: no bias).
       const float slope2 = kAlibi ? __ldg(p.alibi + w.h) * kLog2eF : 0.f;
+      // FP8: the block scale of this query tile; a K tile's scale joins it per tile.
+      const float qs = (kFp8 && tq0 < p.Nq)
+                           ? __ldg(p.q_scales + (size_t)(w.b * p.Hq + w.h) * p.nqt + tq0 / kBM)
+                           : 1.f;
+      const float* ksc = kFp8 ? p.k_scales + (size_t)(w.b * p.Hkv + w.hk) * p.nkt : nullptr;
       // Tile-level bounds: a K/V tile needs no mask when every valid row of this query
       // tile sees every key of it and it lies inside Nk.
       int lo_last = 0, hi_first = 0;
@@ -500,7 +560,12 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
         const bool masked =
             !(lo_last <= k0 && k0 + kBN - 1 <= hi_first && k0 + kBN <= p.Nk);
         float mx;
-        if constexpr (!kAlibi) {
+        const float ks_eff = kFp8 ? p.kscale * qs * __ldg(ksc + k0 / kBN) : p.kscale;
+        if constexpr (kFp8) {
+          const float mx_raw = masked ? tile_row_max<true>(s, row_lo - k0, row_hi - k0)
+                                      : tile_row_max<false>(s, 0, 0);
+          mx = mx_raw * ks_eff;
+        } else if constexpr (!kAlibi) {
           const float mx_raw = masked ? tile_row_max<true>(s, row_lo - k0, row_hi - k0)
                                       : tile_row_max<false>(s, 0, 0);
           mx = (p.softcap > 0.f) ? scaled_score<true>(mx_raw, p)
@@ -513,7 +578,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
           mx = tile_row_max<false>(s, 0, 0);
         }
         const float m_new = fmaxf(m_ref, mx);
-        const bool need = m_new > m_ref + kRescaleThreshold;
+        const bool need = m_new > m_ref + kThreshold;
         float alpha = 1.f;
         if (need) {
           alpha = ex2_approx(m_ref - m_new);
@@ -539,15 +604,21 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
         float sum = 0.f;
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
-          uint32_t pk[32];
-          if constexpr (kAlibi) {
-            sum += tile_row_exp_half<false>(s, 64 * half, p, 1.f, m_use, pk);
-          } else if (p.softcap > 0.f) {
-            sum += tile_row_exp_half<true>(s, 64 * half, p, p.kscale, m_use, pk);
+          if constexpr (kFp8) {
+            uint32_t pk[16];
+            sum += tile_row_exp_half_e4m3(s, 64 * half, ks_eff, m_use, pk);
+            tmem_st_x16(tS + 96u + 16u * half, pk);
           } else {
-            sum += tile_row_exp_half<false>(s, 64 * half, p, p.kscale, m_use, pk);
+            uint32_t pk[32];
+            if constexpr (kAlibi) {
+              sum += tile_row_exp_half<false>(s, 64 * half, p, 1.f, m_use, pk);
+            } else if (p.softcap > 0.f) {
+              sum += tile_row_exp_half<true>(s, 64 * half, p, p.kscale, m_use, pk);
+            } else {
+              sum += tile_row_exp_half<false>(s, 64 * half, p, p.kscale, m_use, pk);
+            }
+            tmem_st_x32(tP + 32u * half, pk);
           }
-          tmem_st_x32(tP + 32u * half, pk);
           tmem_wait_st();
           tc_fence_before();
           __syncwarp();
@@ -565,7 +636,9 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
       ++ocount;
       tc_fence_after();
       const bool valid = row < p.Nq;
-      const float inv_l = (l > 0.f) ? 1.0f / l : 0.f;
+      // FP8: O holds 64 P V_codes; the V scale of the head and the 64 come out here
+      const float o_mul = kFp8 ? __ldg(p.v_scales + w.b * p.Hkv + w.hk) / kPScale : 1.f;
+      const float inv_l = (l > 0.f) ? o_mul / l : 0.f;
       const float lse = (l > 0.f) ? (m_ref + log2f(l)) * kLn2 : -INFINITY;
       const size_t row_index = (size_t)(w.b * p.Hq + w.h) * (size_t)p.Nq + (size_t)row;
       __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.o) + row_index * D;
@@ -606,18 +679,18 @@ __global__ void attn_fill_empty_kernel(__nv_bfloat16* o, float* lse, size_t rows
   if (i < rows) lse[i] = -INFINITY;
 }
 
-template <int D, bool kAlibi>
+template <int D, bool kAlibi, bool kFp8 = false>
 int launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                const FwdParams& p, cudaStream_t stream) {
-  using C = Cfg<D>;
+  using C = Cfg<D, kFp8>;
   static_assert(C::kSmemBytes <= 227 * 1024, "shared memory budget");
-  cudaError_t e = cudaFuncSetAttribute(attn_fwd_sm100_kernel<D, kAlibi>,
+  cudaError_t e = cudaFuncSetAttribute(attn_fwd_sm100_kernel<D, kAlibi, kFp8>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        C::kSmemBytes);
   if (e != cudaSuccess) return -4;
   const long long units = (long long)((p.num_pairs + 1) / 2) * p.B * p.Hq;
   const long long grid = units < p.num_sms ? units : p.num_sms;
-  attn_fwd_sm100_kernel<D, kAlibi>
+  attn_fwd_sm100_kernel<D, kAlibi, kFp8>
       <<<(unsigned)grid, kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, p);
   return cudaGetLastError() == cudaSuccess ? 0 : -4;
 }
@@ -627,6 +700,7 @@ int launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& 
 int launch_attn_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                     const FwdParams& p, int d, cudaStream_t stream) {
   const bool alibi = p.alibi != nullptr;
+  if (p.q_scales != nullptr) return d == 128 ? launch_fwd<128, false, true>(tq, tk, tv, p, stream) : -2;
   if (d == 128) return alibi ? launch_fwd<128, true>(tq, tk, tv, p, stream)
                              : launch_fwd<128, false>(tq, tk, tv, p, stream);
   if (d == 64) return alibi ? launch_fwd<64, true>(tq, tk, tv, p, stream)

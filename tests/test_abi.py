@@ -190,3 +190,21 @@ def test_backward_validation(lib):
     assert f(*args(wsb=10)) == -6
     assert lib.attn_bwd_workspace_bytes(2, 4, 100) == 2 * ((2 * 4 * 100 * 4 + 255) // 256 * 256)
     assert lib.attn_bwd_workspace_bytes(0, 4, 100) == 0
+
+
+def test_fp8_entry_validation(lib):
+    f = lib.attn_fwd_fp8
+    P = ctypes.c_void_p(16)
+    # (q8, k8, vt8, qs, ks, vs, o, lse, B, Hq, Hkv, Nq, Nk, nk_pad, d, scale, mask, window,
+    #  docs, num_docs, stream)
+    assert f(P, P, P, P, P, P, P, P, 1, 2, 2, 64, 64, 64, 64, 0.0, 1, 0, None, 0, None) == -2
+    assert f(P, P, P, P, P, P, P, P, 1, 2, 2, 64, 64, 60, 128, 0.0, 1, 0, None, 0, None) == -1
+    assert f(P, P, P, P, P, P, P, P, 1, 2, 2, 64, 64, 72, 128, 0.0, 1, 0, None, 0, None) == -1
+    assert f(P, P, P, P, P, P, P, P, 1, 3, 2, 64, 64, 64, 128, 0.0, 1, 0, None, 0, None) == -2
+    assert f(None, None, None, None, None, None, None, None, 0, 2, 2, 64, 64, 64, 128, 0.0, 1, 0,
+             None, 0, None) == 0
+    q = lib.attn_quantize_fp8
+    assert q(P, P, P, 1, 1, 8, 96, 128, 0, 0, None, None) == -2
+    assert q(P, P, P, 1, 1, 8, 128, 0, 0, 0, None, None) == -1
+    assert q(P, P, P, 1, 1, 8, 128, 128, 1, 4, None, None) == -1      # n_pad < N
+    assert q(ctypes.c_void_p(24), P, P, 1, 1, 8, 128, 128, 0, 0, None, None) == -3

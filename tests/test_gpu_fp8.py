@@ -1,0 +1,135 @@
+"""FP8 (E4M3) path: the block quantizer and attn_fwd_fp8 against the oracle (fp8 module).
+
+The attention oracle is exact attention of the dequantized codes the quantizer produced, so
+the kernel's remaining error is P rounded to E4M3 before the P V product (at most 2^-4
+relative per element in E4M3's normal range, which the 64 P scaling keeps probabilities
+down to 2^-12 of the row max in) and O rounded to bf16.  Bounds: the maximum O error at most
+2^-4 of max |V| (each output is a convex combination of V rows, each weight off by at most
+2^-4 relative), the mean O error 2^-7 of the mean |V| (round-to-nearest leaves 2^-5 relative
+on average per weight, and the signs of those errors vary over the visible keys of a row;
+measured at most 4.7e-3), and LSE within 1e-3 (it comes from the fp32 P, not the rounded
+one; measured at most 2.6e-6)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+from io_aware_softmax_b200 import attn_fwd_fp8, device_status, quantize_fp8
+from oracle import fp8 as ofp8
+from tests.gpu_common import f64
+
+pytestmark = pytest.mark.gpu
+
+MASK_ID = {"none": 0, "causal": 1, "sliding_causal": 2, "document_causal": 3, "sliding": 4}
+TOL_MEAN_O = 2.0 ** -7
+
+
+def _codes(t):
+    return t.float().cpu().numpy().astype(np.float64)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("N", [1, 127, 300])
+def test_quantizer_is_bit_exact_without_rotation(d, N):
+    x = (workloads.randn_bf16((2, 3, N, d), N + d, 0).float()
+         * torch.tensor([1.0, 30.0, 0.02]).view(1, 3, 1, 1)).to(torch.bfloat16)
+    x[1, 2, :min(N, 128)] = 0                               # an all-zero first block
+    codes, scales = quantize_fp8(x.cuda(), block_rows=128)
+    assert device_status() == 0
+    want_c, want_s = ofp8.quantize_blocks(x.float().numpy(), 128)
+    assert np.array_equal(_codes(codes), want_c)
+    assert np.allclose(scales.cpu().numpy(), want_s, rtol=1e-6, atol=0)
+
+
+@pytest.mark.parametrize("N,n_pad", [(300, 304), (128, 144), (5, 16)])
+def test_quantizer_transposed_per_head(N, n_pad):
+    x = workloads.randn_bf16((2, 2, N, 128), N, 1)
+    codes, scales = quantize_fp8(x.cuda(), block_rows=N, transpose=True, n_pad=n_pad)
+    assert device_status() == 0
+    assert codes.shape == (2, 2, 128, n_pad) and scales.shape == (2, 2, 1)
+    want_c, want_s = ofp8.quantize_blocks(x.float().numpy(), N)
+    got = _codes(codes)
+    assert np.array_equal(got[..., :N], np.swapaxes(want_c, 2, 3))
+    assert np.all(got[..., N:] == 0.0)
+    assert np.allclose(scales.cpu().numpy(), want_s, rtol=1e-6, atol=0)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_quantizer_rotation_within_e4m3_rounding(d):
+    x = workloads.randn_bf16((1, 2, 260, d), d, 2)
+    x[0, 0, :, 5] *= 40                                     # an outlier column
+    signs = torch.from_numpy(np.random.default_rng(d).choice([-1.0, 1.0], d).astype(np.float32))
+    codes, scales = quantize_fp8(x.cuda(), block_rows=128, signs=signs.cuda())
+    assert device_status() == 0
+    rot = ofp8.rotate(x.float().numpy(), signs.numpy())
+    deq = ofp8.dequantize_blocks(_codes(codes), scales.cpu().numpy(), 128)
+    rep = np.repeat(scales.cpu().numpy(), 128, axis=2)[:, :, :260, None]
+    assert np.all(np.abs(deq - rot) <= 2 ** -4 * np.abs(rot) + rep * 2 ** -10 + 1e-5 * np.abs(rot).max())
+    # the rotation spread the outlier: the head's scale is far below the unrotated one
+    _, s_plain = quantize_fp8(x.cuda(), block_rows=128)
+    assert float(scales[0, 0, 0]) < 0.4 * float(s_plain[0, 0, 0])
+
+
+def _fp8_case(B, Hq, Hkv, N, mask="none", window=0, docs=None, seed=0, rotate=True, std=1.0):
+    d = 128
+    q = workloads.randn_bf16((B, Hq, N, d), seed, 0, std).cuda()
+    k = workloads.randn_bf16((B, Hkv, N, d), seed, 1, std).cuda()
+    v = workloads.randn_bf16((B, Hkv, N, d), seed, 2, std).cuda()
+    signs = None
+    if rotate:
+        rng = np.random.default_rng(seed)
+        signs = torch.from_numpy(rng.choice([-1.0, 1.0], d).astype(np.float32)).cuda()
+    q8, qs = quantize_fp8(q, block_rows=128, signs=signs)
+    k8, ks = quantize_fp8(k, block_rows=128, signs=signs)
+    vt8, vs = quantize_fp8(v, block_rows=N, transpose=True)
+    doc_t = None if docs is None else torch.tensor(docs, dtype=torch.int32, device="cuda")
+    o, lse = attn_fwd_fp8(q8, qs, k8, ks, vt8, vs[:, :, 0], mask=mask, window=window,
+                          doc_offsets=doc_t)
+    assert device_status() == 0
+    vcodes = np.swapaxes(_codes(vt8)[..., :N], 2, 3)
+    O_ref, L_ref = ofp8.attention_fp8(_codes(q8), qs.cpu().numpy(), _codes(k8),
+                                      ks.cpu().numpy(), vcodes, vs.cpu().numpy()[:, :, 0],
+                                      mask_kind=MASK_ID[mask], window=window, doc_offsets=docs)
+    O = f64(o)
+    vmax = float(np.abs(vcodes * vs.cpu().numpy()[:, :, 0][:, :, None, None]).max())
+    vmean = float(np.abs(vcodes * vs.cpu().numpy()[:, :, 0][:, :, None, None]).mean())
+    err = np.abs(O - O_ref)
+    lerr = np.abs(f64(lse) - L_ref)
+    tag = f"fp8 {B}x{Hq}/{Hkv}x{N} {mask} w{window} rot{rotate}"
+    print(f"{tag}: O max {err.max() / vmax:.2e} of max|V|, mean {err.mean() / vmean:.2e} of "
+          f"mean|V|, LSE max {lerr.max():.2e}")
+    assert np.all(np.isfinite(O))
+    assert err.max() <= 2 ** -4 * vmax, tag
+    assert err.mean() <= TOL_MEAN_O * vmean, tag
+    assert lerr.max() <= 1e-3, tag
+
+
+@pytest.mark.parametrize("N", [1, 129, 300, 777])
+@pytest.mark.parametrize("mask", ["none", "causal"])
+def test_fp8_attention_ragged(N, mask):
+    _fp8_case(1, 2, 2, N, mask=mask, seed=N)
+
+
+def test_fp8_attention_gqa_and_no_rotation():
+    _fp8_case(2, 8, 2, 600, mask="causal", seed=3)
+    _fp8_case(1, 4, 1, 600, mask="causal", seed=4, rotate=False)
+
+
+@pytest.mark.parametrize("mask,window,docs", [("sliding_causal", 100, None), ("sliding", 70, None),
+                                              ("document_causal", 0, [0, 100, 101, 700, 900])])
+def test_fp8_attention_masks(mask, window, docs):
+    _fp8_case(1, 2, 1, 900, mask=mask, window=window, docs=docs, seed=window + 11)
+
+
+def test_fp8_attention_large_scores():
+    _fp8_case(1, 2, 2, 500, mask="causal", seed=12, std=2.5)
+
+
+def test_fp8_head_dim_64_is_unsupported():
+    q8 = torch.zeros((1, 1, 8, 64), dtype=torch.float8_e4m3fn, device="cuda")
+    vt8 = torch.zeros((1, 1, 64, 16), dtype=torch.float8_e4m3fn, device="cuda")
+    s = torch.ones((1, 1, 1), dtype=torch.float32, device="cuda")
+    with pytest.raises(Exception) as e:
+        attn_fwd_fp8(q8, s, q8, s, vt8, s[:, :, 0])
+    assert "unsupported" in str(e.value).lower()
