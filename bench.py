@@ -275,6 +275,8 @@ def run_ours(args, world, rank, local):
     peaks, peak_src = load_peaks()
     if args.only == "decode":
         return bench_decode(args, world, local, peaks, peak_src)
+    if args.only == "extras":
+        return {"extras": bench_extras(args, world, local, peaks, peak_src)}
     w = workloads.CAUSAL_MHA
     dev = torch.device("cuda", torch.cuda.current_device())
     q, k, v = workloads.make_inputs(w, device=dev)
@@ -326,14 +328,7 @@ def run_ours(args, world, rank, local):
         torch.cuda.empty_cache()
         out["decode"] = bench_decode(args, world, local, peaks, peak_src)
     if not args.no_extras and args.only == "all":
-        out["extras"] = {x.name: bench_prefill_variant(x, args, world, local, peaks, peak_src)
-                         for x in (workloads.ALIBI_MHA, workloads.SWA_SYM_GQA)}
-        out["extras"]["paged_" + workloads.DECODE.name] = bench_decode_paged(
-            args, world, local, peaks, peak_src)
-        out["extras"]["backward_" + workloads.CAUSAL_MHA.name] = bench_backward(
-            workloads.CAUSAL_MHA, args, world, local, peaks, peak_src)
-        out["extras"]["fp8_" + workloads.CAUSAL_MHA.name] = bench_fp8(
-            workloads.CAUSAL_MHA, args, world, local, peaks, peak_src)
+        out["extras"] = bench_extras(args, world, local, peaks, peak_src)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         tf, heads, dt = oracle_prefill_sample(w, args.cpu_budget)
         out["cpu_baseline"] = {"value": round(tf, 5), "unit": "TFLOP/s",
@@ -341,6 +336,31 @@ def run_ours(args, world, rank, local):
                                "sample": f"{heads} whole heads (4096 query rows each, all keys) "
                                          f"of {w.name}, fp64, {dt:.1f} s"}
     return out
+
+
+def bench_extras(args, world, local, peaks, peak_src):
+    """The rows beyond the headline: ALiBi and symmetric-window prefill, paged decode, the
+    backward pass and the FP8 prefill, one line each."""
+    ex = {x.name: bench_prefill_variant(x, args, world, local, peaks, peak_src)
+          for x in (workloads.ALIBI_MHA, workloads.SWA_SYM_GQA)}
+    paged = bench_decode_paged(args, world, local, peaks, peak_src)
+    ex["paged_" + paged["config"]["workload"]] = paged
+    ex["backward_" + workloads.CAUSAL_MHA.name] = bench_backward(
+        workloads.CAUSAL_MHA, args, world, local, peaks, peak_src)
+    ex["fp8_" + workloads.CAUSAL_MHA.name] = bench_fp8(
+        workloads.CAUSAL_MHA, args, world, local, peaks, peak_src)
+    return ex
+
+
+def decode_workload(args):
+    """The decode workload, with the batch overridden by --decode-batch (smaller caches for
+    profiler captures)."""
+    import dataclasses
+    w = workloads.DECODE
+    if args.decode_batch:
+        w = dataclasses.replace(w, B=args.decode_batch, name=w.name.replace(
+            f"b{w.B}_", f"b{args.decode_batch}_"))
+    return w
 
 
 def bench_prefill_variant(w, args, world, local, peaks, peak_src):
@@ -377,7 +397,9 @@ def bench_prefill_variant(w, args, world, local, peaks, peak_src):
            "useful_tflop_per_step": round(flops / 1e12, 4),
            "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak,
                         "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
-                        "peak_source": f"bf16_tflops (burst, {peak_src})", "traffic": None},
+                        "peak_source": f"bf16_tflops (burst, {peak_src})",
+                        "kernel": "attn_fwd_sm100_kernel<128>" + (" (ALiBi)" if w.alibi else ""),
+                        "traffic": recorded_traffic("prefill_" + w.name)},
            "gpu_launches": steps, "clocks": clk.summary()}
     del q, k, v, o, lse
     torch.cuda.empty_cache()
@@ -389,7 +411,7 @@ def bench_decode_paged(args, world, local, peaks, peak_src, page: int = 256):
     every sequence at full length (the same KV bytes as the contiguous line)."""
     import torch
     import io_aware_softmax_b200 as attn
-    w = workloads.DECODE
+    w = decode_workload(args)
     dev = torch.device("cuda", torch.cuda.current_device())
     max_pages = w.Nk // page
     num_pages = w.B * max_pages
@@ -429,7 +451,10 @@ def bench_decode_paged(args, world, local, peaks, peak_src, page: int = 256):
            "roofline": {"bound": "hbm", "achieved": round(io / (call_ms * 1e-3) / 1e9, 1),
                         "peak": peak, "unit": "GB/s",
                         "frac": round(io / (call_ms * 1e-3) / 1e9 / peak, 4),
-                        "peak_source": f"hbm_gbs ({peak_src})", "traffic": None},
+                        "peak_source": f"hbm_gbs ({peak_src})",
+                        "kernel": "attn_decode_split_kernel (paged) + attn_merge_kernel "
+                                  "(one call)",
+                        "traffic": recorded_traffic("paged_decode")},
            "gpu_launches": 2 * steps, "clocks": clk.summary()}
     del q, kp, vp, o, lse, ws
     torch.cuda.empty_cache()
@@ -470,7 +495,9 @@ def bench_backward(w, args, world, local, peaks, peak_src):
            "flop_accounting": "10 d per visible pair (S, dP, dV, dQ, dK)",
            "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak,
                         "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
-                        "peak_source": f"bf16_tflops (burst, {peak_src})", "traffic": None},
+                        "peak_source": f"bf16_tflops (burst, {peak_src})",
+                        "kernel": "attn_bwd_rowdot + attn_bwd_dq + attn_bwd_dkdv (one call)",
+                        "traffic": recorded_traffic("backward")},
            "gpu_launches": 3 * steps, "clocks": clk.summary()}
     del q, k, v, o, lse, dout, dq, dk, dv, ws
     torch.cuda.empty_cache()
@@ -528,7 +555,9 @@ def bench_fp8(w, args, world, local, peaks, peak_src):
            "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak,
                         "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
                         "peak_source": f"2 x bf16_tflops (burst, {peak_src}): the nominal "
-                                       "fp8 / bf16 ratio", "traffic": None},
+                                       "fp8 / bf16 ratio",
+                        "kernel": "attn_fwd_sm100_kernel<128> (E4M3)",
+                        "traffic": recorded_traffic("fp8")},
            "gpu_launches": steps, "clocks": clk.summary()}
     del q, k, v, q8, k8, vt8, o, lse
     torch.cuda.empty_cache()
@@ -568,12 +597,8 @@ def e2e_prefill(w, args, world, q, k, v):
 
 def bench_decode(args, world, local, peaks, peak_src):
     import torch
-    import dataclasses
     import io_aware_softmax_b200 as attn
-    w = workloads.DECODE
-    if args.decode_batch:
-        w = dataclasses.replace(w, B=args.decode_batch, name=w.name.replace(
-            f"b{w.B}_", f"b{args.decode_batch}_"))
+    w = decode_workload(args)
     dev = torch.device("cuda", torch.cuda.current_device())
     q, kc, vc = workloads.make_inputs(w, device=dev)
     S = attn.default_splits(w.B, w.Hkv, w.Nk, dev.index)
@@ -682,7 +707,7 @@ def main(argv=None):
                     help="skip the ALiBi and symmetric-window prefill lines")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle time")
-    ap.add_argument("--only", choices=["all", "prefill", "decode"], default="all",
+    ap.add_argument("--only", choices=["all", "prefill", "decode", "extras"], default="all",
                     help="run one part only (profiling runs)")
     ap.add_argument("--decode-batch", type=int, default=None,
                     help="decode batch size override (smaller caches for ncu captures)")

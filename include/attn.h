@@ -184,7 +184,9 @@ ATTN_API int attn_blockmap(int B, int Nq, int Nk, int mask_kind, int window, con
  *   o        bf16 [B, Hq, 1, d] (written) lse fp32 [B, Hq, 1] natural log (written)
  *   scale    <= 0 selects 1/sqrt(d); num_splits <= 0 selects attn_decode_default_splits
  *   workspace, workspace_bytes  caller-owned device scratch, >= attn_decode_workspace_bytes,
- *            16-byte aligned; its contents on return are the per-split partials.
+ *            16-byte aligned; its contents on return are the per-split partials.  Split s
+ *            covers the 64-row tiles [s n / S, (s + 1) n / S) of the n = ceil(T / 64) tiles
+ *            (rows past T excluded), so no tile is read by two splits.
  *   No mask (every cached key is visible).  Hq / Hkv <= 16, d in {64, 128}.
  * Errors: INVALID_ARG, UNSUPPORTED, MISALIGNED, WORKSPACE, CUDA.  T == 0 writes O = 0 and
  * LSE = -inf.

@@ -24,27 +24,34 @@ SOURCES = ["attn_api.cu", "attn_prefill.cu", "attn_decode.cu", "attn_blockmap.cu
 HEADERS = ["attn_internal.h", "mask.cuh", "sm100_ptx.cuh", "tmem_ldst.cuh"]
 ARCH_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
-# The prefill kernel splits its launch registers between warpgroups with setmaxnreg
-# (two softmax warpgroups, one warpgroup of MMA/TMA warps, 384 threads).  The split must fit
-# in what the CTA is launched with, or the increase would wait forever: check the count
-# ptxas chose against the split constants read from the kernel source.
-PREFILL_KERNEL = "attn_fwd_sm100_kernel"
-PREFILL_THREADS = 384
+# Kernels that split their launch registers between warpgroups with setmaxnreg (two
+# element-wise / softmax warpgroups and one warpgroup of MMA/TMA warps, 384 threads).  A split
+# must fit in what the CTA is launched with, or the increase would wait forever: the build
+# checks the count ptxas chose against the split constants read from each kernel's source.
+# (kernel name fragment, source, constant of the two big warpgroups, constant of the third)
+SPLIT_KERNELS = [
+    ("attn_fwd_sm100_kernel", "attn_prefill.cu", "kRegsSoftmax", "kRegsOther"),
+    ("attn_bwd_dq_kernel", "attn_backward.cu", "kBwdRegsElem", "kBwdRegsOther"),
+    ("attn_bwd_dkdv_kernel", "attn_backward.cu", "kBwdRegsElem", "kBwdRegsOther"),
+]
+SPLIT_THREADS = 384
+PREFILL_KERNEL = SPLIT_KERNELS[0][0]
+PREFILL_THREADS = SPLIT_THREADS
 
 
-def _prefill_split_regs() -> int:
-    src = open(os.path.join(CSRC, "attn_prefill.cu"), encoding="utf-8").read()
-    soft = int(re.search(r"kRegsSoftmax\s*=\s*(\d+)", src).group(1))
-    other = int(re.search(r"kRegsOther\s*=\s*(\d+)", src).group(1))
-    return 2 * 128 * soft + 128 * other
+def split_regs(source: str, big: str, other: str) -> int:
+    src = open(os.path.join(CSRC, source), encoding="utf-8").read()
+    n_big = int(re.search(big + r"\s*=\s*(\d+)", src).group(1))
+    n_other = int(re.search(other + r"\s*=\s*(\d+)", src).group(1))
+    return 2 * 128 * n_big + 128 * n_other
 
 
-PREFILL_SPLIT_REGS = _prefill_split_regs()
+PREFILL_SPLIT_REGS = split_regs(*SPLIT_KERNELS[0][1:])
 
 
 def check_register_budget(ptxas_log: str) -> dict:
-    """Launch register counts of the prefill kernels from ``-Xptxas -v`` output; raises if
-    the setmaxnreg split would not fit."""
+    """Launch register counts of the kernels that split registers, from ``-Xptxas -v``
+    output; raises if a split would not fit or a kernel is missing."""
     counts = {}
     current = None
     for line in ptxas_log.splitlines():
@@ -56,13 +63,17 @@ def check_register_budget(ptxas_log: str) -> dict:
         if m and current is not None:
             counts[current] = int(m.group(1))
             current = None
-    found = {k: v for k, v in counts.items() if PREFILL_KERNEL in k}
-    if not found:
-        raise RuntimeError("ptxas output lists no prefill kernel; cannot check registers")
-    for name, regs in found.items():
-        if regs * PREFILL_THREADS < PREFILL_SPLIT_REGS:
-            raise RuntimeError(f"{name}: launched with {regs} registers/thread, the warpgroup "
-                               f"split needs {PREFILL_SPLIT_REGS / PREFILL_THREADS:.1f}")
+    found = {}
+    for frag, source, big, other in SPLIT_KERNELS:
+        need = split_regs(source, big, other)
+        hits = {k: v for k, v in counts.items() if frag in k}
+        if not hits:
+            raise RuntimeError(f"ptxas output lists no {frag}; cannot check registers")
+        for name, regs in hits.items():
+            if regs * SPLIT_THREADS < need:
+                raise RuntimeError(f"{name}: launched with {regs} registers/thread, the "
+                                   f"warpgroup split needs {need / SPLIT_THREADS:.1f}")
+        found.update(hits)
     return found
 
 

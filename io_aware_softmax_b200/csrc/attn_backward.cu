@@ -19,8 +19,10 @@
 //     writes bf16 P^T and dS^T into the low halves of those buffers, and dV += P^T dO and
 //     dK += dS^T Q accumulate in TMEM -- dK and dV of a tile are complete in one CTA, so
 //     nothing is accumulated with atomics.
-// Warps: 0-3 the element-wise warpgroup, 4 the tcgen05 issuer (whole warp, elect.sync),
-// 5 the TMA producer.
+// Warps: 0-7 two element-wise warpgroups (group g owns the tile's columns [64g, 64g + 64)
+// in every TMEM lane), 8 the tcgen05 issuer (whole warp, elect.sync), 9 the TMA producer,
+// 10-11 the per-query vectors of the streamed tiles (key-tile kernel; idle in the query-tile
+// kernel).  Warps 8-11 give registers to the element-wise groups with setmaxnreg.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -35,12 +37,19 @@ namespace attn {
 namespace {
 
 constexpr int kBT = 128;                 // rows of every tile (queries or keys)
-constexpr int kBwdThreads = 192;
-constexpr int kBwdMmaWarp = 4;
-constexpr int kBwdTmaWarp = 5;
+constexpr int kBwdThreads = 384;
+constexpr int kBwdMmaWarp = 8;
+constexpr int kBwdTmaWarp = 9;
+// setmaxnreg split of the 384 x 168 launch registers: 2 x 128 x 200 + 128 x 104 = 64512
+constexpr uint32_t kBwdRegsElem = 200;
+constexpr uint32_t kBwdRegsOther = 104;
 constexpr float kLog2eB = 1.44269504088896341f;
-constexpr uint32_t kTmemX = 0;           // S or S^T (fp32), then bf16 P^T in its low half
+constexpr uint32_t kTmemX = 0;           // S or S^T (fp32), then bf16 P^T (see below)
 constexpr uint32_t kTmemY = 128;         // dP or dP^T (fp32), then bf16 dS / dS^T
+// The bf16 result of fp32 columns [64g, 64g + 64) goes to columns [64g, 64g + 32) of the same
+// buffer: each warpgroup overwrites only columns it has already read itself, so the two
+// groups never wait for each other.  Contraction step kk (16 columns) then sits at TMEM
+// column 8 kk, plus 32 for the second group's half.
 constexpr uint32_t kTmemAcc0 = 256;      // dQ, or dV
 constexpr uint32_t kTmemAcc1 = 384;      // dK
 
@@ -55,35 +64,50 @@ struct BwdCfg {
   static constexpr int kVecOff = kRingOff + kStages * 2 * kTileBytes;
   static constexpr int kVecBytes = 2 * 4 * kBT * 4;      // [2 parities][lse2, D, lo, hi][128]
   static constexpr int kBarOff = kVecOff + kVecBytes;
-  // stat, full[S], empty[S], s_ready, p_ready, acc, done
-  static constexpr int kNumBars = 5 + 2 * kStages;
+  // stat, full[S], empty[S], s_ready, p_ready, acc, done, vec_full[2], vec_empty[2]
+  static constexpr int kNumBars = 9 + 2 * kStages;
   static constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 16 + 1024;
 };
 
 enum : uint32_t {
   kSiteBwdStat = 201, kSiteBwdFull, kSiteBwdEmpty, kSiteBwdS, kSiteBwdP, kSiteBwdAcc,
-  kSiteBwdDrain,
+  kSiteBwdDrain, kSiteBwdVecFull, kSiteBwdVecEmpty,
 };
 
 __device__ __forceinline__ float bf(uint32_t u) { return __uint_as_float(u); }
 
-// One chunk of 32 columns of the recomputed tile for one TMEM lane: s (raw q.k) and dp in
-// fp32; returns bf16 pairs of p (optional) and ds = p (dp - Dv) with p = 2^(s ks - l2).
-// vis(c) says whether column c of the chunk is a visible pair.
-template <bool kWantP, typename Vis, typename L2, typename DV>
-__device__ __forceinline__ void grad_chunk(const uint32_t (&s)[32], const uint32_t (&dp)[32],
-                                           float ks, Vis vis, L2 l2, DV dv,
+// Columns [OFF, OFF + 32) of the N (32 or 64) loaded columns of the recomputed tile for one
+// TMEM lane: s (raw q.k) and dp in fp32; returns bf16 pairs of p (optional) and ds = p (dp - Dv)
+// with p = 2^(s ks - l2).  Four columns at a time: l2(j) and dv(j) give the values of
+// columns OFF + 4j .. OFF + 4j + 3, vis(j) a 4-bit mask of which of them are visible pairs.
+template <bool kWantP, int OFF, int N, typename L2, typename DV, typename Vis>
+__device__ __forceinline__ void grad_chunk(const uint32_t (&s)[N], const uint32_t (&dp)[N],
+                                           float ks, L2 l2, DV dv, Vis vis,
                                            uint32_t (&pk)[16], uint32_t (&dsk)[16]) {
 #pragma unroll
-  for (int c = 0; c < 32; c += 2) {
-    float p0 = ex2_approx(bf(s[c]) * ks - l2(c));
-    float p1 = ex2_approx(bf(s[c + 1]) * ks - l2(c + 1));
-    if (!vis(c)) p0 = 0.f;
-    if (!vis(c + 1)) p1 = 0.f;
-    const float d0 = p0 * (bf(dp[c]) - dv(c));
-    const float d1 = p1 * (bf(dp[c + 1]) - dv(c + 1));
-    if (kWantP) pk[c >> 1] = pack_bf16x2(p0, p1);
-    dsk[c >> 1] = pack_bf16x2(d0, d1);
+  for (int j = 0; j < 8; ++j) {
+    const float4 l = l2(j);
+    const float4 d = dv(j);
+    const unsigned m = vis(j);
+    const int c = OFF + 4 * j;
+    float x0, x1, x2, x3;
+    ffma2(x0, x1, bf(s[c]), bf(s[c + 1]), ks, ks, -l.x, -l.y);
+    ffma2(x2, x3, bf(s[c + 2]), bf(s[c + 3]), ks, ks, -l.z, -l.w);
+    float p0 = ex2_approx(x0), p1 = ex2_approx(x1), p2 = ex2_approx(x2), p3 = ex2_approx(x3);
+    if (!(m & 1u)) p0 = 0.f;
+    if (!(m & 2u)) p1 = 0.f;
+    if (!(m & 4u)) p2 = 0.f;
+    if (!(m & 8u)) p3 = 0.f;
+    const float d0 = p0 * (bf(dp[c]) - d.x);
+    const float d1 = p1 * (bf(dp[c + 1]) - d.y);
+    const float d2 = p2 * (bf(dp[c + 2]) - d.z);
+    const float d3 = p3 * (bf(dp[c + 3]) - d.w);
+    if (kWantP) {
+      pk[2 * j] = pack_bf16x2(p0, p1);
+      pk[2 * j + 1] = pack_bf16x2(p2, p3);
+    }
+    dsk[2 * j] = pack_bf16x2(d0, d1);
+    dsk[2 * j + 1] = pack_bf16x2(d2, d3);
   }
 }
 
@@ -200,8 +224,9 @@ __device__ __forceinline__ void issue_ss(uint32_t d_tmem, uint32_t a_smem, uint3
   }
 }
 
-// acc (128 x D) += A (bf16 pairs in TMEM columns [a_col, a_col + 64)) times B (ring tile:
-// 128 rows along the contraction, D columns, MN-major).
+// acc (128 x D) += A (bf16 pairs in TMEM: contraction step kk at column 8 kk, plus 32 for
+// kk >= 4, the second warpgroup's half) times B (ring tile: 128 rows along the contraction,
+// D columns, MN-major).
 template <int D>
 __device__ __forceinline__ void issue_ts(uint32_t acc, uint32_t a_tmem, uint32_t b_smem,
                                          bool first) {
@@ -210,8 +235,8 @@ __device__ __forceinline__ void issue_ts(uint32_t acc, uint32_t a_tmem, uint32_t
   const uint64_t db = smem_desc(b_smem, C::kChunkBytes, 1024);
 #pragma unroll
   for (int kk = 0; kk < kBT / 16; ++kk)
-    umma_ts_warp(acc, a_tmem + 8u * kk, db + ((kk * 16 * 128) >> 4), idesc,
-                 (!first || kk > 0) ? 1u : 0u);
+    umma_ts_warp(acc, a_tmem + 8u * kk + (kk >= 4 ? 32u : 0u), db + ((kk * 16 * 128) >> 4),
+                 idesc, (!first || kk > 0) ? 1u : 0u);
 }
 
 // dQ of one 128-row query tile of head (b, h).
@@ -250,7 +275,7 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       mbar_init(sm.bar(BAR_EMPTY + s), 1);
     }
     mbar_init(sm.bar(BAR_S), 1);
-    mbar_init(sm.bar(BAR_P), 4);
+    mbar_init(sm.bar(BAR_P), 8);
     mbar_init(sm.bar(BAR_ACC), 1);
     mbar_init(sm.bar(BAR_DONE), 1);
     *abort_flag = 0;
@@ -265,7 +290,9 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == kBwdTmaWarp) {
+  if (warp >= kBwdMmaWarp) {
+   regs_decrease<kBwdRegsOther>();
+   if (warp == kBwdTmaWarp) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0 && n > 0) {
       mbar_arrive_expect_tx(sm.bar(BAR_STAT), 2 * C::kTileBytes);
@@ -300,7 +327,7 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       }
     }
     __syncwarp();
-  } else if (warp == kBwdMmaWarp) {
+   } else if (warp == kBwdMmaWarp) {
     // -------------------------------------------------------------- tcgen05 issuer
     if (n > 0) {
       bool ok = mbar_wait_warp(sm.bar(BAR_STAT), 0, abort_flag, p.err, kSiteBwdStat);
@@ -323,18 +350,24 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     }
     umma_commit_warp(sm.bar(BAR_DONE));
     mbar_wait_warp(sm.bar(BAR_DONE), 0, nullptr, p.err, kSiteBwdDrain);
+   }
   } else {
-    // ------------------------------------------------------ element-wise warpgroup
-    const int wq = warp;                       // TMEM lane quarter
+    regs_increase<kBwdRegsElem>();
+    // ----------------------------------------------------- element-wise warpgroups
+    const int g = warp >> 2;                   // key columns [64g, 64g + 64) of each tile
+    const int wq = warp & 3;                   // TMEM lane quarter
     const int r = wq * 32 + lane;
     const int row = q0 + r;
     const bool valid = row < p.Nq;
     const long long ridx = (long long)bh * p.Nq + row;
     const float l2r = valid ? p.l2[ridx] : INFINITY;
     const float dr = valid ? p.dvec[ridx] : 0.f;
+    const float4 l2r4 = make_float4(l2r, l2r, l2r, l2r);
+    const float4 dr4 = make_float4(dr, dr, dr, dr);
     int rlo = 1, rhi = 0;
     if (valid) row_interval(p.mask, row, rlo, rhi);
     const uint32_t tl = tmem + ((uint32_t)(wq * 32) << 16);
+    const uint32_t col = 64u * (uint32_t)g;
     __nv_bfloat16* drow = reinterpret_cast<__nv_bfloat16*>(p.dq) + ridx * D;
     bool ok = true;
     for (int t = 0; ok && t < n; ++t) {
@@ -343,31 +376,48 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       tc_fence_after();
       const int k0 = (ja + t) * kBT;
       const bool full = lo_last <= k0 && k0 + kBT - 1 <= hi_first && k0 + kBT <= p.Nk;
-#pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        uint32_t s[32], dp[32], pk[16], dsk[16];
-        tmem_ld_x32(tl + kTmemX + 32u * c, s);
-        tmem_ld_x32(tl + kTmemY + 32u * c, dp);
-        const int kc = k0 + 32 * c;
-        grad_chunk<false>(
-            s, dp, p.kscale,
-            [&](int i) { return full || (kc + i >= rlo && kc + i <= rhi); },
-            [&](int) { return l2r; }, [&](int) { return dr; }, pk, dsk);
-        tmem_st_x16(tl + kTmemY + 16u * c, dsk);
+      const int kc = k0 + (int)col;
+      uint32_t s[64], dp[64];
+      tmem_ld_x64_async(tl + kTmemX + col, s);
+      tmem_ld_x64_async(tl + kTmemY + col, dp);
+      tmem_ld_wait_x64(s);
+      tmem_ld_wait_x64(dp);
+      auto vis = [&](int c) -> unsigned {      // columns kc + c .. kc + c + 3
+        if (full) return 0xFu;
+        unsigned m = 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) m |= (kc + c + i >= rlo && kc + c + i <= rhi) ? (1u << i) : 0u;
+        return m;
+      };
+      {
+        uint32_t pk[16], dsk[16];
+        grad_chunk<false, 0, 64>(s, dp, p.kscale, [&](int) { return l2r4; },
+                             [&](int) { return dr4; }, [&](int j) { return vis(4 * j); }, pk,
+                             dsk);
+        tmem_st_x16(tl + kTmemY + col, dsk);
+      }
+      {
+        uint32_t pk[16], dsk[16];
+        grad_chunk<false, 32, 64>(s, dp, p.kscale, [&](int) { return l2r4; },
+                              [&](int) { return dr4; }, [&](int j) { return vis(32 + 4 * j); },
+                              pk, dsk);
+        tmem_st_x16(tl + kTmemY + col + 16u, dsk);
       }
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(sm.bar(BAR_P));
     }
+    // group g writes dQ columns [g D / 2, (g + 1) D / 2) of its row
     if (n == 0) {
-      store_zero_row(drow, D, valid);
+      store_zero_row(drow + g * (D / 2), D / 2, valid);
     } else if (ok) {
       const bool okacc =
           __all_sync(0xffffffffu, mbar_wait(sm.bar(BAR_ACC), 0, abort_flag, p.err, kSiteBwdAcc));
       if (okacc) {
         tc_fence_after();
-        store_row<D>(tl + kTmemAcc0, p.scale, drow, valid);
+        store_row<D / 2>(tl + kTmemAcc0 + (uint32_t)(g * (D / 2)), p.scale, drow + g * (D / 2),
+                         valid);
       }
     }
   }
@@ -392,7 +442,8 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ,
   extern __shared__ uint8_t smem_raw[];
   const BwdSmem<D> sm = bwd_smem<D>(smem_raw);
   const int BAR_STAT = 0, BAR_FULL = 1, BAR_EMPTY = 1 + NS, BAR_S = 1 + 2 * NS,
-            BAR_P = 2 + 2 * NS, BAR_ACC = 3 + 2 * NS, BAR_DONE = 4 + 2 * NS;
+            BAR_P = 2 + 2 * NS, BAR_ACC = 3 + 2 * NS, BAR_DONE = 4 + 2 * NS,
+            BAR_VF = 5 + 2 * NS, BAR_VE = 7 + 2 * NS;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm.base + C::kBarOff + C::kNumBars * 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   // per streamed query tile: base-2 LSE, D, and each query's visible key interval
@@ -420,9 +471,13 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ,
       mbar_init(sm.bar(BAR_EMPTY + s), 1);
     }
     mbar_init(sm.bar(BAR_S), 1);
-    mbar_init(sm.bar(BAR_P), 4);
+    mbar_init(sm.bar(BAR_P), 8);
     mbar_init(sm.bar(BAR_ACC), 1);
     mbar_init(sm.bar(BAR_DONE), 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(sm.bar(BAR_VF + i), 64);     // every thread of warps 10-11
+      mbar_init(sm.bar(BAR_VE + i), 8);      // every element-wise warp
+    }
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -435,7 +490,39 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ,
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == kBwdTmaWarp) {
+  if (warp >= kBwdMmaWarp) {
+   regs_decrease<kBwdRegsOther>();
+   if (warp > kBwdTmaWarp) {
+    // ------------------------------------------------- per-query vectors of each tile
+    // l2 = LSE log2(e), D and the visible key interval of the tile's 128 queries, into the
+    // parity buffer of the tile, ahead of the element-wise groups.
+    const int i = (warp - kBwdTmaWarp - 1) * 32 + lane;     // 0..63
+    for (int t = 0; t < n; ++t) {
+      const int par = t & 1;
+      if (t >= 2 && !mbar_wait(sm.bar(BAR_VE + par), ((t >> 1) - 1) & 1, abort_flag, p.err,
+                               kSiteBwdVecEmpty))
+        break;
+      const int h = hk * p.G + t / ni;
+      const int q0 = (ia + t % ni) * kBT;
+#pragma unroll
+      for (int e = i; e < kBT; e += 64) {
+        const int q = q0 + e;
+        float l2q = INFINITY, dq = 0.f;
+        int lo = 1, hi = 0;
+        if (q < p.Nq) {
+          const long long qi = ((long long)b * p.Hq + h) * p.Nq + q;
+          l2q = p.l2[qi];
+          dq = p.dvec[qi];
+          row_interval(p.mask, q, lo, hi);
+        }
+        vec[(par * 4 + 0) * kBT + e] = l2q;
+        vec[(par * 4 + 1) * kBT + e] = dq;
+        vec[(par * 4 + 2) * kBT + e] = __int_as_float(lo);
+        vec[(par * 4 + 3) * kBT + e] = __int_as_float(hi);
+      }
+      mbar_arrive(sm.bar(BAR_VF + par));
+    }
+   } else if (warp == kBwdTmaWarp) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0 && n > 0) {
       const int zkv = b * p.Hkv + hk;
@@ -471,7 +558,7 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ,
       }
     }
     __syncwarp();
-  } else if (warp == kBwdMmaWarp) {
+   } else if (warp == kBwdMmaWarp) {
     // -------------------------------------------------------------- tcgen05 issuer
     if (n > 0) {
       bool ok = mbar_wait_warp(sm.bar(BAR_STAT), 0, abort_flag, p.err, kSiteBwdStat);
@@ -495,82 +582,89 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ,
     }
     umma_commit_warp(sm.bar(BAR_DONE));
     mbar_wait_warp(sm.bar(BAR_DONE), 0, nullptr, p.err, kSiteBwdDrain);
+   }
   } else {
-    // ------------------------------------------------------ element-wise warpgroup
-    const int wq = warp;
+    regs_increase<kBwdRegsElem>();
+    // ----------------------------------------------------- element-wise warpgroups
+    const int g = warp >> 2;         // query columns [64g, 64g + 64) of each streamed tile
+    const int wq = warp & 3;
     const int r = wq * 32 + lane;
     const int key = k0 + r;
     const bool kvalid = key < p.Nk;
     const uint32_t tl = tmem + ((uint32_t)(wq * 32) << 16);
+    const uint32_t col = 64u * (uint32_t)g;
     const long long kidx = ((long long)b * p.Hkv + hk) * p.Nk + key;
     bool ok = true;
     for (int t = 0; t < n; ++t) {
-      // this tile's query vectors; the barrier also makes the four warps agree to go on
+      // this tile's query vectors, written ahead by warps 10-11
       const int par = t & 1;
-      const int h = hk * p.G + t / ni;
       const int q0 = (ia + t % ni) * kBT;
-      {
-        const int q = q0 + r;
-        float l2q = INFINITY, dq = 0.f;
-        int lo = 1, hi = 0;
-        if (q < p.Nq) {
-          const long long qi = ((long long)b * p.Hq + h) * p.Nq + q;
-          l2q = p.l2[qi];
-          dq = p.dvec[qi];
-          row_interval(p.mask, q, lo, hi);
-        }
-        vec[(par * 4 + 0) * kBT + r] = l2q;
-        vec[(par * 4 + 1) * kBT + r] = dq;
-        vec[(par * 4 + 2) * kBT + r] = __int_as_float(lo);
-        vec[(par * 4 + 3) * kBT + r] = __int_as_float(hi);
-      }
-      uint32_t all_ok;
-      asm volatile("{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
-                   "bar.red.and.pred q, 1, 128, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
-                   : "=r"(all_ok) : "r"(ok ? 1u : 0u) : "memory");
-      if (!all_ok) { ok = false; break; }
+      ok = __all_sync(0xffffffffu, mbar_wait(sm.bar(BAR_VF + par), (t >> 1) & 1, abort_flag,
+                                             p.err, kSiteBwdVecFull));
+      if (!ok) break;
       ok = __all_sync(0xffffffffu, mbar_wait(sm.bar(BAR_S), t & 1, abort_flag, p.err, kSiteBwdS));
-      if (!ok) continue;      // the next barrier ends the loop for all four warps
+      if (!ok) break;
       tc_fence_after();
-      const float* l2v = vec + (par * 4 + 0) * kBT;
-      const float* dv = vec + (par * 4 + 1) * kBT;
-      const int* lov = reinterpret_cast<const int*>(vec + (par * 4 + 2) * kBT);
-      const int* hiv = reinterpret_cast<const int*>(vec + (par * 4 + 3) * kBT);
-      const int qlast = min(q0 + kBT, p.Nq) - 1 - q0;
-      const bool full = q0 + kBT <= p.Nq && k0 + kBT <= p.Nk && lov[qlast] <= k0 &&
+      const float* l2v = vec + (par * 4 + 0) * kBT + col;
+      const float* dv = vec + (par * 4 + 1) * kBT + col;
+      const int* lov = reinterpret_cast<const int*>(vec + (par * 4 + 2) * kBT + col);
+      const int* hiv = reinterpret_cast<const int*>(vec + (par * 4 + 3) * kBT + col);
+      // Every query of the group's 64 sees every key of the CTA's tile (the intervals are
+      // non-decreasing at both ends, so the last query's start and the first query's end
+      // decide): no per-pair test.
+      const bool full = q0 + (int)col + 64 <= p.Nq && k0 + kBT <= p.Nk && lov[63] <= k0 &&
                         k1 <= hiv[0];
-#pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
+      auto vis = [&](int c) -> unsigned {      // group columns c .. c + 3
+        if (full) return 0xFu;
+        const int4 lo = *reinterpret_cast<const int4*>(lov + c);
+        const int4 hi = *reinterpret_cast<const int4*>(hiv + c);
+        unsigned m = 0;
+        if (kvalid) {
+          m |= (lo.x <= key && key <= hi.x) ? 1u : 0u;
+          m |= (lo.y <= key && key <= hi.y) ? 2u : 0u;
+          m |= (lo.z <= key && key <= hi.z) ? 4u : 0u;
+          m |= (lo.w <= key && key <= hi.w) ? 8u : 0u;
+        }
+        return m;
+      };
+      auto l2f = [&](int c) { return *reinterpret_cast<const float4*>(l2v + c); };
+      auto dvf = [&](int c) { return *reinterpret_cast<const float4*>(dv + c); };
+      // two halves of 32 columns, one after the other (P^T and dS^T of a half land in
+      // columns the group has already read)
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) {
         uint32_t s[32], dp[32], pk[16], dsk[16];
-        tmem_ld_x32(tl + kTmemX + 32u * c, s);
-        tmem_ld_x32(tl + kTmemY + 32u * c, dp);
-        const int qc = 32 * c;
-        grad_chunk<true>(
-            s, dp, p.kscale,
-            [&](int i) {
-              return full || (kvalid && lov[qc + i] <= key && key <= hiv[qc + i]);
-            },
-            [&](int i) { return l2v[qc + i]; }, [&](int i) { return dv[qc + i]; }, pk, dsk);
-        tmem_st_x16(tl + kTmemX + 16u * c, pk);
-        tmem_st_x16(tl + kTmemY + 16u * c, dsk);
+        tmem_ld_x32_async(tl + kTmemX + col + 32u * hf, s);
+        tmem_ld_x32_async(tl + kTmemY + col + 32u * hf, dp);
+        tmem_ld_wait_x32(s);
+        tmem_ld_wait_x32(dp);
+        grad_chunk<true, 0, 32>(s, dp, p.kscale, [&](int j) { return l2f(32 * hf + 4 * j); },
+                                [&](int j) { return dvf(32 * hf + 4 * j); },
+                                [&](int j) { return vis(32 * hf + 4 * j); }, pk, dsk);
+        tmem_st_x16(tl + kTmemX + col + 16u * hf, pk);
+        tmem_st_x16(tl + kTmemY + col + 16u * hf, dsk);
       }
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(sm.bar(BAR_P));
+      if (lane == 0) {
+        mbar_arrive(sm.bar(BAR_P));
+        mbar_arrive(sm.bar(BAR_VE + par));    // this warp has read the tile's vectors
+      }
     }
-    __nv_bfloat16* dvrow = reinterpret_cast<__nv_bfloat16*>(p.dv) + kidx * D;
-    __nv_bfloat16* dkrow = reinterpret_cast<__nv_bfloat16*>(p.dk) + kidx * D;
+    // group 0 writes the dV row, group 1 the dK row
+    __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(g == 0 ? p.dv : p.dk) + kidx * D;
     if (n == 0) {
-      store_zero_row(dvrow, D, kvalid);
-      store_zero_row(dkrow, D, kvalid);
+      store_zero_row(dst, D, kvalid);
     } else if (ok) {
       const bool okacc =
           __all_sync(0xffffffffu, mbar_wait(sm.bar(BAR_ACC), 0, abort_flag, p.err, kSiteBwdAcc));
       if (okacc) {
         tc_fence_after();
-        store_row<D>(tl + kTmemAcc0, 1.f, dvrow, kvalid);
-        store_row<D>(tl + kTmemAcc1, p.scale, dkrow, kvalid);
+        if (g == 0)
+          store_row<D>(tl + kTmemAcc0, 1.f, dst, kvalid);
+        else
+          store_row<D>(tl + kTmemAcc1, p.scale, dst, kvalid);
       }
     }
   }

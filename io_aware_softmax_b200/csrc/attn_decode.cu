@@ -80,9 +80,11 @@ __device__ __forceinline__ uint32_t swz_off(int tok, int d) {
   return (uint32_t)((d >> 6) * (kTok * 128) + tok * 128 + ((((d & 63) >> 3) ^ (tok & 7)) << 4));
 }
 
-// Item = (batch b, KV head hk, split s) and its rows [t0, t1).  Contiguous caches cut the
-// T rows evenly; paged caches cut the sequence's own length at 64-row tile boundaries, so
-// no tile straddles two pages (page_size is a multiple of the tile).
+// Item = (batch b, KV head hk, split s) and its rows [t0, t1).  The splits cut the rows at
+// 64-row tile boundaries, as evenly as whole tiles allow: every tile is loaded by exactly
+// one split (an uneven cut would load the tile across a boundary twice), and in a paged
+// cache no tile straddles two pages (page_size is a multiple of the tile).  A paged
+// sequence is cut at its own length.
 template <bool kPaged>
 __device__ __forceinline__ void item_coords(const DecParams& p, int item, int& b, int& hk, int& s,
                                             int& t0, int& t1) {
@@ -90,17 +92,15 @@ __device__ __forceinline__ void item_coords(const DecParams& p, int item, int& b
   s = item % p.S;
   b = bk / p.Hkv;
   hk = bk % p.Hkv;
-  if (!kPaged) {
-    t0 = (int)(((long long)s * p.T) / p.S);
-    t1 = (int)(((long long)(s + 1) * p.T) / p.S);
-  } else {
+  int T = p.T;
+  if (kPaged) {
     const long long cap = (long long)p.max_pages * p.page_size;
-    const int T = (int)min(max((long long)__ldg(p.seq_lens + b), 0LL), cap);
-    const long long tiles = (T + kTok - 1) / kTok;
-    t0 = (int)((s * tiles) / p.S) * kTok;
-    t1 = (int)min((long long)T, (((s + 1) * tiles) / p.S) * kTok);
-    if (t1 < t0) t1 = t0;
+    T = (int)min(max((long long)__ldg(p.seq_lens + b), 0LL), cap);
   }
+  const long long tiles = (T + kTok - 1) / kTok;
+  t0 = (int)((s * tiles) / p.S) * kTok;
+  t1 = (int)min((long long)T, (((s + 1) * tiles) / p.S) * kTok);
+  if (t1 < t0) t1 = t0;
 }
 
 template <int D, bool kUpper, bool kPaged>

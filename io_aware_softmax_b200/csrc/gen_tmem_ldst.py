@@ -59,6 +59,6 @@ hdr = '''// TMEM <-> register moves in the 32x32b shape: every thread of a warp 
 namespace attn {
 
 '''
-body = (ld(16) + "\n" + ld(32) + "\n" + ld(64) + "\n" + ld(128) + "\n" + ld_nowait(64) + "\n" +
-        ld_wait(64) + "\n" + st(16) + "\n" + st(32))
+body = (ld(16) + "\n" + ld(32) + "\n" + ld(64) + "\n" + ld(128) + "\n" + ld_nowait(32) + "\n" +
+        ld_wait(32) + "\n" + ld_nowait(64) + "\n" + ld_wait(64) + "\n" + st(16) + "\n" + st(32))
 open(os.path.join(os.path.dirname(os.path.abspath(__file__)), "tmem_ldst.cuh"), "w").write(hdr + body + "\n}  // namespace attn\n")

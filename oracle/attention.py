@@ -352,12 +352,17 @@ def merge_partials(o_parts, lse_parts):
     return O, lse
 
 
-def split_bounds(T: int, num_splits: int):
-    """Even split of T keys into num_splits contiguous slices (sizes differ by <= 1)."""
-    return [(s * T // num_splits, (s + 1) * T // num_splits) for s in range(num_splits)]
+def split_bounds(T: int, num_splits: int, tile: int = 1):
+    """Split of T keys into num_splits contiguous slices that cut only at multiples of
+    `tile` (the last slice ends at T): slice s holds tiles [s n / S, (s + 1) n / S) of the
+    n = ceil(T / tile) tiles, so sizes differ by at most one tile (tile = 1: an even split of
+    the keys).  Which slices FlashDecoding uses is free; merging is exact for any of them."""
+    n = -(-T // tile)
+    return [(min(T, (s * n // num_splits) * tile), min(T, ((s + 1) * n // num_splits) * tile))
+            for s in range(num_splits)]
 
 
-def decode_splitkv(q, k_cache, v_cache, num_splits: int, scale=None):
+def decode_splitkv(q, k_cache, v_cache, num_splits: int, scale=None, tile: int = 1):
     """FlashDecoding reference ("3.7 어텐션 II", 3.7.4): q [B,Hq,1,d] against a
     contiguous cache [B,Hkv,T,d]; every split is attended separately (plain definition on
     its slice) and the partials are merged with ``merge_partials``.
@@ -377,7 +382,7 @@ def decode_splitkv(q, k_cache, v_cache, num_splits: int, scale=None):
     for b in range(B):
         for h in range(Hq):
             hk = h // G
-            for s, (t0, t1) in enumerate(split_bounds(T, S)):
+            for s, (t0, t1) in enumerate(split_bounds(T, S, tile)):
                 if t1 <= t0:
                     continue
                 o, l = attention_head(q[b, h], np.arange(Nq), k_cache[b, hk, t0:t1],

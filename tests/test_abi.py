@@ -47,7 +47,10 @@ def test_built_for_sm100a_only():
     assert "for 'sm_100a'" in log
     assert re.search(r"for 'sm_(?!100a)", log) is None
     regs = build.check_register_budget(log)
-    assert regs and all(r * build.PREFILL_THREADS >= build.PREFILL_SPLIT_REGS for r in regs.values())
+    for frag, source, big, other in build.SPLIT_KERNELS:
+        hits = [r for k, r in regs.items() if frag in k]
+        need = build.split_regs(source, big, other)
+        assert hits and all(r * build.SPLIT_THREADS >= need for r in hits), frag
 
 
 def _spills_by_kernel(log):

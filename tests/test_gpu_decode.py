@@ -56,8 +56,8 @@ def test_workspace_holds_split_partials_that_merge_to_the_output():
     o_bytes = ((rows * d * 4 + 255) // 256) * 256
     o_part = ws[:rows * d * 4].view(torch.float32).view(B, Hq, S, d)
     lse_part = ws[o_bytes:o_bytes + rows * 4].view(torch.float32).view(B, Hq, S)
-    # the partials are the oracle's per-split results (split boundaries s*T//S)
-    _, _, O_parts, L_parts = oracle.decode_splitkv(f64(q), f64(kc), f64(vc), S)
+    # the partials are the oracle's per-split results; the kernel cuts at 64-row tiles
+    _, _, O_parts, L_parts = oracle.decode_splitkv(f64(q), f64(kc), f64(vc), S, tile=64)
     compare(o_part, lse_part, O_parts[:, :, 0], L_parts[:, :, 0], "split partials")
 
 

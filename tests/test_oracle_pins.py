@@ -265,17 +265,31 @@ def test_tiled_online_softmax_equals_full(mask_kind, window, docs, bq, bk):
     assert np.allclose(lse, lt, atol=1e-12, rtol=0)
 
 
-@pytest.mark.parametrize("splits", [1, 2, 3, 8, 37])
-def test_split_kv_merge_equals_unsplit(splits):
-    B, Hq, Hkv, T, d = 2, 8, 2, 37, 16
+@pytest.mark.parametrize("splits,T,tile", [(1, 37, 1), (2, 37, 1), (3, 37, 1), (8, 37, 1),
+                                            (37, 37, 1), (3, 200, 64), (5, 200, 64),
+                                            (6, 2000, 64)])
+def test_split_kv_merge_equals_unsplit(splits, T, tile):
+    B, Hq, Hkv, d = 2, 8, 2, 16
     rng = np.random.default_rng(8)
     q = rng.standard_normal((B, Hq, 1, d))
     kc = rng.standard_normal((B, Hkv, T, d))
     vc = rng.standard_normal((B, Hkv, T, d))
-    O, lse, _, _ = oracle.decode_splitkv(q, kc, vc, splits)
+    O, lse, _, _ = oracle.decode_splitkv(q, kc, vc, splits, tile=tile)
     Ou, lu = oracle.attention(q, kc, vc)
     assert np.allclose(O, Ou, atol=1e-12, rtol=0)
     assert np.allclose(lse, lu, atol=1e-12, rtol=0)
+
+
+@pytest.mark.parametrize("T,S,tile", [(37, 8, 1), (2000, 6, 64), (200, 5, 64), (64, 3, 64),
+                                      (32768, 15, 64), (1, 4, 64)])
+def test_split_bounds_tile_the_keys(T, S, tile):
+    b = oracle.split_bounds(T, S, tile)
+    assert len(b) == S and b[0][0] == 0 and b[-1][1] == T
+    assert all(b[i][1] == b[i + 1][0] for i in range(S - 1))       # contiguous, no overlap
+    assert all(t0 <= t1 for t0, t1 in b)
+    assert all(t1 % tile == 0 for t0, t1 in b[:-1])                 # cuts only at tile ends
+    tiles = [-(-(t1 - t0) // tile) for t0, t1 in b]
+    assert max(tiles) - min(tiles) <= 1                             # balanced by whole tiles
 
 
 def test_merge_with_fully_masked_splits():
