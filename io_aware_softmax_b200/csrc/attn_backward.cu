@@ -64,8 +64,9 @@ struct BwdCfg {
   static constexpr int kVecOff = kRingOff + kStages * 2 * kTileBytes;
   static constexpr int kVecBytes = 2 * 4 * kBT * 4;      // [2 parities][lse2, D, lo, hi][128]
   static constexpr int kBarOff = kVecOff + kVecBytes;
-  // stat, full[S], empty[S], s_ready, p_ready, acc, done, vec_full[2], vec_empty[2]
-  static constexpr int kNumBars = 9 + 2 * kStages;
+  // stat, full[S], empty[S], s_ready, dp_ready, p_ready (or x_free), ds_ready, acc, done,
+  // vec_full[2], vec_empty[2]
+  static constexpr int kNumBars = 11 + 2 * kStages;
   static constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 16 + 1024;
 };
 
@@ -76,32 +77,43 @@ enum : uint32_t {
 
 __device__ __forceinline__ float bf(uint32_t u) { return __uint_as_float(u); }
 
-// Columns [OFF, OFF + 32) of the N (32 or 64) loaded columns of the recomputed tile for one
-// TMEM lane: s (raw q.k) and dp in fp32; returns bf16 pairs of p (optional) and ds = p (dp - Dv)
-// with p = 2^(s ks - l2).  Four columns at a time: l2(j) and dv(j) give the values of
-// columns OFF + 4j .. OFF + 4j + 3, vis(j) a 4-bit mask of which of them are visible pairs.
-template <bool kWantP, int OFF, int N, typename L2, typename DV, typename Vis>
-__device__ __forceinline__ void grad_chunk(const uint32_t (&s)[N], const uint32_t (&dp)[N],
-                                           float ks, L2 l2, DV dv, Vis vis,
-                                           uint32_t (&pk)[16], uint32_t (&dsk)[16]) {
+// The two element-wise steps of the recomputed tile for one TMEM lane, four columns at a
+// time (column groups j = 0 .. N/4 - 1 of the loaded run):
+//   probs: s (raw q.k, fp32 bits) becomes p = 2^(s ks - l2), 0 where vis(j) has no bit;
+//   grads: ds = p (dp - Dv) and bf16 pairs of ds (and of p, optionally) for the 32 columns
+//          [OFF, OFF + 32).
+// l2(j) and dv(j) give the four columns' values, vis(j) a 4-bit mask of visible pairs.
+template <int N, typename L2, typename Vis>
+__device__ __forceinline__ void probs(uint32_t (&s)[N], float ks, L2 l2, Vis vis) {
 #pragma unroll
-  for (int j = 0; j < 8; ++j) {
+  for (int j = 0; j < N / 4; ++j) {
     const float4 l = l2(j);
-    const float4 d = dv(j);
     const unsigned m = vis(j);
-    const int c = OFF + 4 * j;
+    const int c = 4 * j;
     float x0, x1, x2, x3;
     ffma2(x0, x1, bf(s[c]), bf(s[c + 1]), ks, ks, -l.x, -l.y);
     ffma2(x2, x3, bf(s[c + 2]), bf(s[c + 3]), ks, ks, -l.z, -l.w);
-    float p0 = ex2_approx(x0), p1 = ex2_approx(x1), p2 = ex2_approx(x2), p3 = ex2_approx(x3);
-    if (!(m & 1u)) p0 = 0.f;
-    if (!(m & 2u)) p1 = 0.f;
-    if (!(m & 4u)) p2 = 0.f;
-    if (!(m & 8u)) p3 = 0.f;
-    const float d0 = p0 * (bf(dp[c]) - d.x);
-    const float d1 = p1 * (bf(dp[c + 1]) - d.y);
-    const float d2 = p2 * (bf(dp[c + 2]) - d.z);
-    const float d3 = p3 * (bf(dp[c + 3]) - d.w);
+    s[c] = __float_as_uint((m & 1u) ? ex2_approx(x0) : 0.f);
+    s[c + 1] = __float_as_uint((m & 2u) ? ex2_approx(x1) : 0.f);
+    s[c + 2] = __float_as_uint((m & 4u) ? ex2_approx(x2) : 0.f);
+    s[c + 3] = __float_as_uint((m & 8u) ? ex2_approx(x3) : 0.f);
+  }
+}
+
+template <bool kWantP, int OFF, int N, int ND, typename DV>
+__device__ __forceinline__ void grads(const uint32_t (&pr)[N], const uint32_t (&dp)[ND], DV dv,
+                                      uint32_t (&pk)[16], uint32_t (&dsk)[16]) {
+  static_assert(ND == 32 || ND == N, "dp holds these 32 columns or all N");
+  constexpr int DOFF = (ND == 32) ? 0 : OFF;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const float4 d = dv(j);
+    const int c = OFF + 4 * j, e = DOFF + 4 * j;
+    const float p0 = bf(pr[c]), p1 = bf(pr[c + 1]), p2 = bf(pr[c + 2]), p3 = bf(pr[c + 3]);
+    const float d0 = p0 * (bf(dp[e]) - d.x);
+    const float d1 = p1 * (bf(dp[e + 1]) - d.y);
+    const float d2 = p2 * (bf(dp[e + 2]) - d.z);
+    const float d3 = p3 * (bf(dp[e + 3]) - d.w);
     if (kWantP) {
       pk[2 * j] = pack_bf16x2(p0, p1);
       pk[2 * j + 1] = pack_bf16x2(p2, p3);
@@ -109,6 +121,12 @@ __device__ __forceinline__ void grad_chunk(const uint32_t (&s)[N], const uint32_
     dsk[2 * j] = pack_bf16x2(d0, d1);
     dsk[2 * j + 1] = pack_bf16x2(d2, d3);
   }
+}
+
+// bf16 pairs of 32 fp32 values.
+__device__ __forceinline__ void pack_pairs(const uint32_t (&v)[32], uint32_t (&pk)[16]) {
+#pragma unroll
+  for (int k = 0; k < 16; ++k) pk[k] = pack_bf16x2(bf(v[2 * k]), bf(v[2 * k + 1]));
 }
 
 // First / last query row whose visible key interval meets keys [k0, k1] (the intervals are
@@ -249,8 +267,10 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   constexpr int NS = C::kStages;
   extern __shared__ uint8_t smem_raw[];
   const BwdSmem<D> sm = bwd_smem<D>(smem_raw);
+  // S ready, dP ready, X free (S loaded into registers), dS ready
   const int BAR_STAT = 0, BAR_FULL = 1, BAR_EMPTY = 1 + NS, BAR_S = 1 + 2 * NS,
-            BAR_P = 2 + 2 * NS, BAR_ACC = 3 + 2 * NS, BAR_DONE = 4 + 2 * NS;
+            BAR_DP = 2 + 2 * NS, BAR_XF = 3 + 2 * NS, BAR_DS = 4 + 2 * NS,
+            BAR_ACC = 5 + 2 * NS, BAR_DONE = 6 + 2 * NS;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm.base + C::kBarOff + C::kNumBars * 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -275,7 +295,9 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       mbar_init(sm.bar(BAR_EMPTY + s), 1);
     }
     mbar_init(sm.bar(BAR_S), 1);
-    mbar_init(sm.bar(BAR_P), 8);
+    mbar_init(sm.bar(BAR_DP), 1);
+    mbar_init(sm.bar(BAR_XF), 8);
+    mbar_init(sm.bar(BAR_DS), 8);
     mbar_init(sm.bar(BAR_ACC), 1);
     mbar_init(sm.bar(BAR_DONE), 1);
     *abort_flag = 0;
@@ -332,19 +354,41 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     if (n > 0) {
       bool ok = mbar_wait_warp(sm.bar(BAR_STAT), 0, abort_flag, p.err, kSiteBwdStat);
       tc_fence_after();
-      for (int t = 0; ok && t < n; ++t) {
-        const int s = t % NS;
-        if (!mbar_wait_warp(sm.bar(BAR_FULL + s), (t / NS) & 1, abort_flag, p.err, kSiteBwdFull))
-          break;
+      // Order: S_0, dP_0, then per tile t: S_{t+1} as soon as the element-wise groups hold
+      // S_t in registers, dQ += dS_t K_t once dS_t is written, dP_{t+1} behind it (dP_{t+1}
+      // overwrites Y, which dQ reads first: the tensor pipe runs in order).  The products of
+      // the next tile overlap the element-wise work of this one.
+      auto stage = [&](int t) { return sm.ring + (t % NS) * 2 * C::kTileBytes; };
+      auto full = [&](int t) {
+        const bool f = mbar_wait_warp(sm.bar(BAR_FULL + t % NS), (t / NS) & 1, abort_flag,
+                                      p.err, kSiteBwdFull);
         tc_fence_after();
-        const uint32_t kt = sm.ring + s * 2 * C::kTileBytes;
-        issue_ss<D>(tmem + kTmemX, sm.stat, kt);                              // S = Q K^T
-        issue_ss<D>(tmem + kTmemY, sm.stat + C::kTileBytes, kt + C::kTileBytes);  // dP
+        return f;
+      };
+      if (ok && full(0)) {
+        issue_ss<D>(tmem + kTmemX, sm.stat, stage(0));                              // S_0
         umma_commit_warp(sm.bar(BAR_S));
-        if (!mbar_wait_warp(sm.bar(BAR_P), t & 1, abort_flag, p.err, kSiteBwdP)) break;
+        issue_ss<D>(tmem + kTmemY, sm.stat + C::kTileBytes, stage(0) + C::kTileBytes);  // dP_0
+        umma_commit_warp(sm.bar(BAR_DP));
+      } else {
+        ok = false;
+      }
+      for (int t = 0; ok && t < n; ++t) {
+        const uint32_t kt = stage(t);
+        if (t + 1 < n) {
+          if (!mbar_wait_warp(sm.bar(BAR_XF), t & 1, abort_flag, p.err, kSiteBwdP) || !full(t + 1))
+            break;
+          issue_ss<D>(tmem + kTmemX, sm.stat, stage(t + 1));                      // S_{t+1}
+          umma_commit_warp(sm.bar(BAR_S));
+        }
+        if (!mbar_wait_warp(sm.bar(BAR_DS), t & 1, abort_flag, p.err, kSiteBwdP)) break;
         tc_fence_after();
         issue_ts<D>(tmem + kTmemAcc0, tmem + kTmemY, kt, t == 0);            // dQ += dS K
-        umma_commit_warp(sm.bar(BAR_EMPTY + s));
+        umma_commit_warp(sm.bar(BAR_EMPTY + t % NS));
+        if (t + 1 < n) {
+          issue_ss<D>(tmem + kTmemY, sm.stat + C::kTileBytes, stage(t + 1) + C::kTileBytes);
+          umma_commit_warp(sm.bar(BAR_DP));                                    // dP_{t+1}
+        }
       }
       umma_commit_warp(sm.bar(BAR_ACC));
     }
@@ -377,11 +421,6 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       const int k0 = (ja + t) * kBT;
       const bool full = lo_last <= k0 && k0 + kBT - 1 <= hi_first && k0 + kBT <= p.Nk;
       const int kc = k0 + (int)col;
-      uint32_t s[64], dp[64];
-      tmem_ld_x64_async(tl + kTmemX + col, s);
-      tmem_ld_x64_async(tl + kTmemY + col, dp);
-      tmem_ld_wait_x64(s);
-      tmem_ld_wait_x64(dp);
       auto vis = [&](int c) -> unsigned {      // columns kc + c .. kc + c + 3
         if (full) return 0xFu;
         unsigned m = 0;
@@ -389,24 +428,34 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         for (int i = 0; i < 4; ++i) m |= (kc + c + i >= rlo && kc + c + i <= rhi) ? (1u << i) : 0u;
         return m;
       };
+      uint32_t s[64];
+      tmem_ld_x64_async(tl + kTmemX + col, s);
+      tmem_ld_wait_x64(s);
+      // S_t is in registers: X may take S_{t+1}
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(sm.bar(BAR_XF));
+      probs<64>(s, p.kscale, [&](int) { return l2r4; }, [&](int j) { return vis(4 * j); });
+      ok = __all_sync(0xffffffffu, mbar_wait(sm.bar(BAR_DP), t & 1, abort_flag, p.err, kSiteBwdS));
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t dp[64];
+      tmem_ld_x64_async(tl + kTmemY + col, dp);
+      tmem_ld_wait_x64(dp);
       {
         uint32_t pk[16], dsk[16];
-        grad_chunk<false, 0, 64>(s, dp, p.kscale, [&](int) { return l2r4; },
-                             [&](int) { return dr4; }, [&](int j) { return vis(4 * j); }, pk,
-                             dsk);
+        grads<false, 0, 64, 64>(s, dp, [&](int) { return dr4; }, pk, dsk);
         tmem_st_x16(tl + kTmemY + col, dsk);
       }
       {
         uint32_t pk[16], dsk[16];
-        grad_chunk<false, 32, 64>(s, dp, p.kscale, [&](int) { return l2r4; },
-                              [&](int) { return dr4; }, [&](int j) { return vis(32 + 4 * j); },
-                              pk, dsk);
+        grads<false, 32, 64, 64>(s, dp, [&](int) { return dr4; }, pk, dsk);
         tmem_st_x16(tl + kTmemY + col + 16u, dsk);
       }
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(sm.bar(BAR_P));
+      if (lane == 0) mbar_arrive(sm.bar(BAR_DS));
     }
     // group g writes dQ columns [g D / 2, (g + 1) D / 2) of its row
     if (n == 0) {
@@ -441,9 +490,11 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ,
   constexpr int NS = C::kStages;
   extern __shared__ uint8_t smem_raw[];
   const BwdSmem<D> sm = bwd_smem<D>(smem_raw);
+  // S^T ready, dP^T ready, P^T written, dS^T written
   const int BAR_STAT = 0, BAR_FULL = 1, BAR_EMPTY = 1 + NS, BAR_S = 1 + 2 * NS,
-            BAR_P = 2 + 2 * NS, BAR_ACC = 3 + 2 * NS, BAR_DONE = 4 + 2 * NS,
-            BAR_VF = 5 + 2 * NS, BAR_VE = 7 + 2 * NS;
+            BAR_DP = 2 + 2 * NS, BAR_P = 3 + 2 * NS, BAR_DS = 4 + 2 * NS,
+            BAR_ACC = 5 + 2 * NS, BAR_DONE = 6 + 2 * NS, BAR_VF = 7 + 2 * NS,
+            BAR_VE = 9 + 2 * NS;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm.base + C::kBarOff + C::kNumBars * 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   // per streamed query tile: base-2 LSE, D, and each query's visible key interval
@@ -471,7 +522,9 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ,
       mbar_init(sm.bar(BAR_EMPTY + s), 1);
     }
     mbar_init(sm.bar(BAR_S), 1);
+    mbar_init(sm.bar(BAR_DP), 1);
     mbar_init(sm.bar(BAR_P), 8);
+    mbar_init(sm.bar(BAR_DS), 8);
     mbar_init(sm.bar(BAR_ACC), 1);
     mbar_init(sm.bar(BAR_DONE), 1);
     for (int i = 0; i < 2; ++i) {
@@ -563,20 +616,43 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ,
     if (n > 0) {
       bool ok = mbar_wait_warp(sm.bar(BAR_STAT), 0, abort_flag, p.err, kSiteBwdStat);
       tc_fence_after();
-      for (int t = 0; ok && t < n; ++t) {
-        const int s = t % NS;
-        if (!mbar_wait_warp(sm.bar(BAR_FULL + s), (t / NS) & 1, abort_flag, p.err, kSiteBwdFull))
-          break;
+      // Order: S^T_0, dP^T_0, then per tile t: dV += P^T_t dO_t once P^T_t is written,
+      // S^T_{t+1} behind it (it overwrites X, which dV reads first: the tensor pipe runs in
+      // order), dK += dS^T_t Q_t once dS^T_t is written, dP^T_{t+1} behind it.  Each pair of
+      // products overlaps one of the two element-wise steps.
+      auto stage = [&](int t) { return sm.ring + (t % NS) * 2 * C::kTileBytes; };
+      auto full = [&](int t) {
+        const bool f = mbar_wait_warp(sm.bar(BAR_FULL + t % NS), (t / NS) & 1, abort_flag,
+                                      p.err, kSiteBwdFull);
         tc_fence_after();
-        const uint32_t qt = sm.ring + s * 2 * C::kTileBytes;
-        issue_ss<D>(tmem + kTmemX, sm.stat, qt);                              // S^T = K Q^T
-        issue_ss<D>(tmem + kTmemY, sm.stat + C::kTileBytes, qt + C::kTileBytes);  // dP^T
+        return f;
+      };
+      if (ok && full(0)) {
+        issue_ss<D>(tmem + kTmemX, sm.stat, stage(0));                              // S^T_0
         umma_commit_warp(sm.bar(BAR_S));
+        issue_ss<D>(tmem + kTmemY, sm.stat + C::kTileBytes, stage(0) + C::kTileBytes);  // dP^T_0
+        umma_commit_warp(sm.bar(BAR_DP));
+      } else {
+        ok = false;
+      }
+      for (int t = 0; ok && t < n; ++t) {
+        const uint32_t qt = stage(t);
         if (!mbar_wait_warp(sm.bar(BAR_P), t & 1, abort_flag, p.err, kSiteBwdP)) break;
         tc_fence_after();
         issue_ts<D>(tmem + kTmemAcc0, tmem + kTmemX, qt + C::kTileBytes, t == 0);  // dV
+        if (t + 1 < n) {
+          if (!full(t + 1)) break;
+          issue_ss<D>(tmem + kTmemX, sm.stat, stage(t + 1));                      // S^T_{t+1}
+          umma_commit_warp(sm.bar(BAR_S));
+        }
+        if (!mbar_wait_warp(sm.bar(BAR_DS), t & 1, abort_flag, p.err, kSiteBwdP)) break;
+        tc_fence_after();
         issue_ts<D>(tmem + kTmemAcc1, tmem + kTmemY, qt, t == 0);                 // dK
-        umma_commit_warp(sm.bar(BAR_EMPTY + s));
+        umma_commit_warp(sm.bar(BAR_EMPTY + t % NS));
+        if (t + 1 < n) {
+          issue_ss<D>(tmem + kTmemY, sm.stat + C::kTileBytes, stage(t + 1) + C::kTileBytes);
+          umma_commit_warp(sm.bar(BAR_DP));                                    // dP^T_{t+1}
+        }
       }
       umma_commit_warp(sm.bar(BAR_ACC));
     }
@@ -629,26 +705,47 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ,
       };
       auto l2f = [&](int c) { return *reinterpret_cast<const float4*>(l2v + c); };
       auto dvf = [&](int c) { return *reinterpret_cast<const float4*>(dv + c); };
-      // two halves of 32 columns, one after the other (P^T and dS^T of a half land in
-      // columns the group has already read)
-#pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {
-        uint32_t s[32], dp[32], pk[16], dsk[16];
-        tmem_ld_x32_async(tl + kTmemX + col + 32u * hf, s);
-        tmem_ld_x32_async(tl + kTmemY + col + 32u * hf, dp);
-        tmem_ld_wait_x32(s);
-        tmem_ld_wait_x32(dp);
-        grad_chunk<true, 0, 32>(s, dp, p.kscale, [&](int j) { return l2f(32 * hf + 4 * j); },
-                                [&](int j) { return dvf(32 * hf + 4 * j); },
-                                [&](int j) { return vis(32 * hf + 4 * j); }, pk, dsk);
-        tmem_st_x16(tl + kTmemX + col + 16u * hf, pk);
-        tmem_st_x16(tl + kTmemY + col + 16u * hf, dsk);
+      // Step 1 (S^T ready): P^T of the group's 64 columns, in two halves of 32; the bf16
+      // P^T of a half lands in columns the group has already read.
+      uint32_t pr0[32], pr1[32];
+      {
+        uint32_t pk[16];
+        tmem_ld_x32_async(tl + kTmemX + col, pr0);
+        tmem_ld_wait_x32(pr0);
+        probs<32>(pr0, p.kscale, [&](int j) { return l2f(4 * j); }, [&](int j) { return vis(4 * j); });
+        pack_pairs(pr0, pk);
+        tmem_st_x16(tl + kTmemX + col, pk);
+        tmem_ld_x32_async(tl + kTmemX + col + 32u, pr1);
+        tmem_ld_wait_x32(pr1);
+        probs<32>(pr1, p.kscale, [&](int j) { return l2f(32 + 4 * j); },
+                  [&](int j) { return vis(32 + 4 * j); });
+        pack_pairs(pr1, pk);
+        tmem_st_x16(tl + kTmemX + col + 16u, pk);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(sm.bar(BAR_P));
+      // Step 2 (dP^T ready): dS^T = P^T (dP^T - D), into the low half of Y likewise.
+      ok = __all_sync(0xffffffffu, mbar_wait(sm.bar(BAR_DP), t & 1, abort_flag, p.err, kSiteBwdS));
+      if (!ok) break;
+      tc_fence_after();
+      {
+        uint32_t dph[32], pk[16], dsk[16];
+        tmem_ld_x32_async(tl + kTmemY + col, dph);
+        tmem_ld_wait_x32(dph);
+        grads<false, 0, 32, 32>(pr0, dph, [&](int j) { return dvf(4 * j); }, pk, dsk);
+        tmem_st_x16(tl + kTmemY + col, dsk);
+        tmem_ld_x32_async(tl + kTmemY + col + 32u, dph);
+        tmem_ld_wait_x32(dph);
+        grads<false, 0, 32, 32>(pr1, dph, [&](int j) { return dvf(32 + 4 * j); }, pk, dsk);
+        tmem_st_x16(tl + kTmemY + col + 16u, dsk);
       }
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
-        mbar_arrive(sm.bar(BAR_P));
+        mbar_arrive(sm.bar(BAR_DS));
         mbar_arrive(sm.bar(BAR_VE + par));    // this warp has read the tile's vectors
       }
     }
