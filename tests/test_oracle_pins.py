@@ -387,6 +387,19 @@ def test_visible_pair_closed_forms_match_element_counts():
     assert accounting.visible_pairs(16384, 16384, MASK_SLIDING_CAUSAL, 1024) == 16268800
 
 
+def test_executed_tiles_are_the_non_empty_tiles_of_the_brute_force_map():
+    # every key tile a query tile walks holds a visible pair (the row intervals are
+    # monotone), so the kernel's executed tiles are exactly the map's non-empty tiles
+    docs = workloads.doc_offsets_for(1000, 100, 400, seed=5)
+    for (kind, w, dd) in [(MASK_NONE, 0, None), (MASK_CAUSAL, 0, None),
+                          (MASK_SLIDING_CAUSAL, 200, None), (MASK_DOCUMENT_CAUSAL, 0, docs),
+                          (MASK_SLIDING, 130, None), (MASK_SLIDING, 0, None)]:
+        tm = oracle.tile_map(1, 1000, 1000, kind, w, dd)
+        assert accounting.executed_tiles(1000, 1000, kind, w, dd) == int((tm != 0).sum()), kind
+    assert accounting.executed_tiles(4096, 4096, MASK_CAUSAL) == 528
+    assert accounting.executed_tiles(16384, 16384, MASK_SLIDING_CAUSAL, 1024) == 868 + 248
+
+
 def test_document_generator():
     lens = workloads.doc_lengths(32768, 512, 4096, seed=0)
     assert sum(lens) == 32768 and all(512 <= x <= 4096 for x in lens[:-1])

@@ -38,6 +38,45 @@ def prefill_useful_flops(B: int, Hq: int, Nq: int, Nk: int, d: int, mask_kind: i
     return 4 * d * visible_pairs(Nq, Nk, mask_kind, window, doc_offsets) * B * Hq
 
 
+def _row_interval(q: int, Nk: int, mask_kind: int, window: int, doc_offsets) -> tuple:
+    """Visible keys [lo, hi] of query row q (lo > hi: none); the intervals are non-decreasing
+    in q at both ends for every mask kind."""
+    last = Nk - 1
+    if mask_kind == MASK_NONE:
+        return 0, last
+    if mask_kind == MASK_CAUSAL:
+        return 0, min(q, last)
+    if mask_kind == MASK_SLIDING_CAUSAL:
+        return max(0, q - window), min(q, last)
+    if mask_kind == MASK_SLIDING:
+        return max(0, q - window), min(q + window, last)
+    if mask_kind == MASK_DOCUMENT_CAUSAL:
+        offs = [int(x) for x in doc_offsets]
+        start = max([o for o in offs[:-1] if o <= q], default=0)
+        return start, min(q, last)
+    raise ValueError(mask_kind)
+
+
+def executed_tiles(Nq: int, Nk: int, mask_kind: int, window: int = 0, doc_offsets=None,
+                   tile: int = 128) -> int:
+    """(query tile, key tile) pairs the prefill kernel runs for one head: each query tile
+    walks the key tiles from its first row's first visible key to its last row's last one."""
+    n = 0
+    for q0 in range(0, Nq, tile):
+        lo, _ = _row_interval(q0, Nk, mask_kind, window, doc_offsets)
+        _, hi = _row_interval(min(q0 + tile, Nq) - 1, Nk, mask_kind, window, doc_offsets)
+        if hi >= lo:
+            n += hi // tile - lo // tile + 1
+    return n
+
+
+def prefill_executed_flops(B: int, Hq: int, Nq: int, Nk: int, d: int, mask_kind: int,
+                           window: int = 0, doc_offsets=None, tile: int = 128) -> int:
+    """FLOPs the tensor cores execute: full tile products for every executed tile pair."""
+    return 4 * d * tile * tile * executed_tiles(Nq, Nk, mask_kind, window, doc_offsets,
+                                                tile) * B * Hq
+
+
 def backward_useful_flops(B: int, Hq: int, Nq: int, Nk: int, d: int, mask_kind: int,
                           window: int = 0, doc_offsets=None) -> int:
     """Useful FLOPs of the backward pass: five products per visible pair (S recomputed,
