@@ -56,6 +56,29 @@ def test_quantizer_transposed_per_head(N, n_pad):
 
 
 @pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("N,block_rows,transpose", [(700, 300, False), (700, 700, False),
+                                                    (300, 64, True), (130, 7, True),
+                                                    (100, 3, False)])
+def test_quantizer_chunked_blocks_are_bit_exact(d, N, block_rows, transpose):
+    # blocks longer than 128 rows, several blocks per chunk, and transposed outputs with
+    # several blocks per head go through the chunked amax / codes / finalize launches
+    x = (workloads.randn_bf16((2, 2, N, d), N + block_rows, 3).float()
+         * torch.tensor([1.0, 7.0]).view(1, 2, 1, 1)).to(torch.bfloat16)
+    n_pad = -(-N // 16) * 16
+    codes, scales = quantize_fp8(x.cuda(), block_rows=block_rows, transpose=transpose,
+                                 n_pad=n_pad if transpose else None)
+    assert device_status() == 0
+    want_c, want_s = ofp8.quantize_blocks(x.float().numpy(), block_rows)
+    got = _codes(codes)
+    if transpose:
+        assert np.array_equal(got[..., :N], np.swapaxes(want_c, 2, 3))
+        assert np.all(got[..., N:] == 0.0)
+    else:
+        assert np.array_equal(got, want_c)
+    assert np.allclose(scales.cpu().numpy(), want_s, rtol=1e-6, atol=0)
+
+
+@pytest.mark.parametrize("d", [64, 128])
 def test_quantizer_rotation_within_e4m3_rounding(d):
     x = workloads.randn_bf16((1, 2, 260, d), d, 2)
     x[0, 0, :, 5] *= 40                                     # an outlier column
