@@ -70,6 +70,25 @@ struct BwdCfg {
   static constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 16 + 1024;
 };
 
+// The query-tile kernel streams K and V through separate rings: a K tile is read by S = Q K^T
+// (issued as soon as the previous S is in registers) and by dQ += dS K at the end of its
+// step, so it lives about two steps and gets three slots; a V tile is read only by
+// dP = dO V^T and gets two.  The early S of the next tile then never waits for its K.
+template <int D>
+struct DqCfg {
+  static constexpr int kTileBytes = BwdCfg<D>::kTileBytes;
+  static constexpr int kSlotsK = 3, kSlotsV = 2;
+  static constexpr int kStatOff = 0;                     // Q and dO of the CTA's query tile
+  static constexpr int kKOff = 2 * kTileBytes;
+  static constexpr int kVOff = kKOff + kSlotsK * kTileBytes;
+  static constexpr int kBarOff = kVOff + kSlotsV * kTileBytes;
+  // stat, fullK[3], emptyK[3], fullV[2], emptyV[2], s, dp, x_free, ds, acc, done
+  static constexpr int kFullK = 1, kEmptyK = 1 + kSlotsK, kFullV = 1 + 2 * kSlotsK,
+                       kEmptyV = 1 + 2 * kSlotsK + kSlotsV, kOwn = 1 + 2 * (kSlotsK + kSlotsV);
+  static constexpr int kNumBars = kOwn + 6;
+  static constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 16 + 1024;
+};
+
 enum : uint32_t {
   kSiteBwdStat = 201, kSiteBwdFull, kSiteBwdEmpty, kSiteBwdS, kSiteBwdP, kSiteBwdAcc,
   kSiteBwdDrain, kSiteBwdVecFull, kSiteBwdVecEmpty,
@@ -263,15 +282,21 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO,
                    const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                    const BwdParams p) {
-  using C = BwdCfg<D>;
-  constexpr int NS = C::kStages;
+  using C = DqCfg<D>;
+  using CB = BwdCfg<D>;
+  constexpr int SK = C::kSlotsK, SV = C::kSlotsV;
   extern __shared__ uint8_t smem_raw[];
-  const BwdSmem<D> sm = bwd_smem<D>(smem_raw);
+  const uint32_t raw_u32 = smem_u32(smem_raw);
+  const uint32_t base_u32 = (raw_u32 + 1023u) & ~1023u;
+  uint8_t* base = smem_raw + (base_u32 - raw_u32);
+  const uint32_t sStat = base_u32 + C::kStatOff;
+  auto k_tile = [&](int t) { return base_u32 + C::kKOff + (uint32_t)(t % SK) * C::kTileBytes; };
+  auto v_tile = [&](int t) { return base_u32 + C::kVOff + (uint32_t)(t % SV) * C::kTileBytes; };
+  auto bar = [&](int i) { return base_u32 + C::kBarOff + 8u * (uint32_t)i; };
   // S ready, dP ready, X free (S loaded into registers), dS ready
-  const int BAR_STAT = 0, BAR_FULL = 1, BAR_EMPTY = 1 + NS, BAR_S = 1 + 2 * NS,
-            BAR_DP = 2 + 2 * NS, BAR_XF = 3 + 2 * NS, BAR_DS = 4 + 2 * NS,
-            BAR_ACC = 5 + 2 * NS, BAR_DONE = 6 + 2 * NS;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm.base + C::kBarOff + C::kNumBars * 8);
+  const int BAR_STAT = 0, BAR_S = C::kOwn, BAR_DP = C::kOwn + 1, BAR_XF = C::kOwn + 2,
+            BAR_DS = C::kOwn + 3, BAR_ACC = C::kOwn + 4, BAR_DONE = C::kOwn + 5;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base + C::kBarOff + C::kNumBars * 8);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -289,17 +314,13 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   }
 
   if (threadIdx.x == 0) {
-    mbar_init(sm.bar(BAR_STAT), 1);
-    for (int s = 0; s < NS; ++s) {
-      mbar_init(sm.bar(BAR_FULL + s), 1);
-      mbar_init(sm.bar(BAR_EMPTY + s), 1);
-    }
-    mbar_init(sm.bar(BAR_S), 1);
-    mbar_init(sm.bar(BAR_DP), 1);
-    mbar_init(sm.bar(BAR_XF), 8);
-    mbar_init(sm.bar(BAR_DS), 8);
-    mbar_init(sm.bar(BAR_ACC), 1);
-    mbar_init(sm.bar(BAR_DONE), 1);
+    for (int i = 0; i < C::kOwn; ++i) mbar_init(bar(i), 1);   // stat, both rings
+    mbar_init(bar(BAR_S), 1);
+    mbar_init(bar(BAR_DP), 1);
+    mbar_init(bar(BAR_XF), 8);
+    mbar_init(bar(BAR_DS), 8);
+    mbar_init(bar(BAR_ACC), 1);
+    mbar_init(bar(BAR_DONE), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -317,83 +338,101 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
    if (warp == kBwdTmaWarp) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0 && n > 0) {
-      mbar_arrive_expect_tx(sm.bar(BAR_STAT), 2 * C::kTileBytes);
+      mbar_arrive_expect_tx(bar(BAR_STAT), 2 * C::kTileBytes);
 #pragma unroll
-      for (int c = 0; c < C::kChunks; ++c) {
-        tma_load_3d(sm.stat + c * C::kChunkBytes, &tmQ, sm.bar(BAR_STAT), c * 64, q0, bh);
-        tma_load_3d(sm.stat + C::kTileBytes + c * C::kChunkBytes, &tmDO, sm.bar(BAR_STAT),
-                    c * 64, q0, bh);
+      for (int c = 0; c < CB::kChunks; ++c) {
+        tma_load_3d(sStat + c * CB::kChunkBytes, &tmQ, bar(BAR_STAT), c * 64, q0, bh);
+        tma_load_3d(sStat + C::kTileBytes + c * CB::kChunkBytes, &tmDO, bar(BAR_STAT), c * 64,
+                    q0, bh);
       }
       const int zkv = b * p.Hkv + hk;
-      int t = 0;
-      for (; t < n; ++t) {
-        const int s = t % NS, round = t / NS;
-        if (round > 0 &&
-            !mbar_wait(sm.bar(BAR_EMPTY + s), (round - 1) & 1, abort_flag, p.err, kSiteBwdEmpty))
+      int tk = 0, tv = 0;                    // tiles issued into the K and V rings
+      for (int t = 0; t < n; ++t) {
+        const int row = (ja + t) * kBT;
+        if (t >= SK && !mbar_wait(bar(C::kEmptyK + t % SK), (t / SK - 1) & 1, abort_flag, p.err,
+                                  kSiteBwdEmpty))
           break;
-        mbar_arrive_expect_tx(sm.bar(BAR_FULL + s), 2 * C::kTileBytes);
-        const uint32_t dst = sm.ring + s * 2 * C::kTileBytes;
+        mbar_arrive_expect_tx(bar(C::kFullK + t % SK), C::kTileBytes);
 #pragma unroll
-        for (int c = 0; c < C::kChunks; ++c) {
-          tma_load_3d(dst + c * C::kChunkBytes, &tmK, sm.bar(BAR_FULL + s), c * 64,
-                      (ja + t) * kBT, zkv);
-          tma_load_3d(dst + C::kTileBytes + c * C::kChunkBytes, &tmV, sm.bar(BAR_FULL + s),
-                      c * 64, (ja + t) * kBT, zkv);
-        }
+        for (int c = 0; c < CB::kChunks; ++c)
+          tma_load_3d(k_tile(t) + c * CB::kChunkBytes, &tmK, bar(C::kFullK + t % SK), c * 64,
+                      row, zkv);
+        ++tk;
+        if (t >= SV && !mbar_wait(bar(C::kEmptyV + t % SV), (t / SV - 1) & 1, abort_flag, p.err,
+                                  kSiteBwdEmpty))
+          break;
+        mbar_arrive_expect_tx(bar(C::kFullV + t % SV), C::kTileBytes);
+#pragma unroll
+        for (int c = 0; c < CB::kChunks; ++c)
+          tma_load_3d(v_tile(t) + c * CB::kChunkBytes, &tmV, bar(C::kFullV + t % SV), c * 64,
+                      row, zkv);
+        ++tv;
       }
       // outstanding copies land before the CTA may exit (matters only on abort)
-      mbar_wait(sm.bar(BAR_STAT), 0, nullptr, p.err, kSiteBwdDrain);
-      for (int s = 0; s < NS && s < t; ++s) {
-        const int last = s + ((t - 1 - s) / NS) * NS;
-        mbar_wait(sm.bar(BAR_FULL + s), (last / NS) & 1, nullptr, p.err, kSiteBwdDrain);
+      mbar_wait(bar(BAR_STAT), 0, nullptr, p.err, kSiteBwdDrain);
+      for (int s = 0; s < SK && s < tk; ++s) {
+        const int last = s + ((tk - 1 - s) / SK) * SK;
+        mbar_wait(bar(C::kFullK + s), (last / SK) & 1, nullptr, p.err, kSiteBwdDrain);
+      }
+      for (int s = 0; s < SV && s < tv; ++s) {
+        const int last = s + ((tv - 1 - s) / SV) * SV;
+        mbar_wait(bar(C::kFullV + s), (last / SV) & 1, nullptr, p.err, kSiteBwdDrain);
       }
     }
     __syncwarp();
    } else if (warp == kBwdMmaWarp) {
     // -------------------------------------------------------------- tcgen05 issuer
     if (n > 0) {
-      bool ok = mbar_wait_warp(sm.bar(BAR_STAT), 0, abort_flag, p.err, kSiteBwdStat);
+      bool ok = mbar_wait_warp(bar(BAR_STAT), 0, abort_flag, p.err, kSiteBwdStat);
       tc_fence_after();
       // Order: S_0, dP_0, then per tile t: S_{t+1} as soon as the element-wise groups hold
       // S_t in registers, dQ += dS_t K_t once dS_t is written, dP_{t+1} behind it (dP_{t+1}
       // overwrites Y, which dQ reads first: the tensor pipe runs in order).  The products of
-      // the next tile overlap the element-wise work of this one.
-      auto stage = [&](int t) { return sm.ring + (t % NS) * 2 * C::kTileBytes; };
-      auto full = [&](int t) {
-        const bool f = mbar_wait_warp(sm.bar(BAR_FULL + t % NS), (t / NS) & 1, abort_flag,
-                                      p.err, kSiteBwdFull);
+      // the next tile overlap the element-wise work of this one.  A K tile is released after
+      // its dQ product, a V tile after its dP product.
+      auto full_k = [&](int t) {
+        const bool f = mbar_wait_warp(bar(C::kFullK + t % SK), (t / SK) & 1, abort_flag, p.err,
+                                      kSiteBwdFull);
         tc_fence_after();
         return f;
       };
-      if (ok && full(0)) {
-        issue_ss<D>(tmem + kTmemX, sm.stat, stage(0));                              // S_0
-        umma_commit_warp(sm.bar(BAR_S));
-        issue_ss<D>(tmem + kTmemY, sm.stat + C::kTileBytes, stage(0) + C::kTileBytes);  // dP_0
-        umma_commit_warp(sm.bar(BAR_DP));
+      auto full_v = [&](int t) {
+        const bool f = mbar_wait_warp(bar(C::kFullV + t % SV), (t / SV) & 1, abort_flag, p.err,
+                                      kSiteBwdFull);
+        tc_fence_after();
+        return f;
+      };
+      if (ok && full_k(0) && full_v(0)) {
+        issue_ss<D>(tmem + kTmemX, sStat, k_tile(0));                               // S_0
+        umma_commit_warp(bar(BAR_S));
+        issue_ss<D>(tmem + kTmemY, sStat + C::kTileBytes, v_tile(0));               // dP_0
+        umma_commit_warp(bar(BAR_DP));
+        umma_commit_warp(bar(C::kEmptyV + 0));
       } else {
         ok = false;
       }
       for (int t = 0; ok && t < n; ++t) {
-        const uint32_t kt = stage(t);
         if (t + 1 < n) {
-          if (!mbar_wait_warp(sm.bar(BAR_XF), t & 1, abort_flag, p.err, kSiteBwdP) || !full(t + 1))
+          if (!mbar_wait_warp(bar(BAR_XF), t & 1, abort_flag, p.err, kSiteBwdP) || !full_k(t + 1))
             break;
-          issue_ss<D>(tmem + kTmemX, sm.stat, stage(t + 1));                      // S_{t+1}
-          umma_commit_warp(sm.bar(BAR_S));
+          issue_ss<D>(tmem + kTmemX, sStat, k_tile(t + 1));                       // S_{t+1}
+          umma_commit_warp(bar(BAR_S));
         }
-        if (!mbar_wait_warp(sm.bar(BAR_DS), t & 1, abort_flag, p.err, kSiteBwdP)) break;
+        if (!mbar_wait_warp(bar(BAR_DS), t & 1, abort_flag, p.err, kSiteBwdP)) break;
         tc_fence_after();
-        issue_ts<D>(tmem + kTmemAcc0, tmem + kTmemY, kt, t == 0);            // dQ += dS K
-        umma_commit_warp(sm.bar(BAR_EMPTY + t % NS));
+        issue_ts<D>(tmem + kTmemAcc0, tmem + kTmemY, k_tile(t), t == 0);     // dQ += dS K
+        umma_commit_warp(bar(C::kEmptyK + t % SK));
         if (t + 1 < n) {
-          issue_ss<D>(tmem + kTmemY, sm.stat + C::kTileBytes, stage(t + 1) + C::kTileBytes);
-          umma_commit_warp(sm.bar(BAR_DP));                                    // dP_{t+1}
+          if (!full_v(t + 1)) break;
+          issue_ss<D>(tmem + kTmemY, sStat + C::kTileBytes, v_tile(t + 1));
+          umma_commit_warp(bar(BAR_DP));                                       // dP_{t+1}
+          umma_commit_warp(bar(C::kEmptyV + (t + 1) % SV));
         }
       }
-      umma_commit_warp(sm.bar(BAR_ACC));
+      umma_commit_warp(bar(BAR_ACC));
     }
-    umma_commit_warp(sm.bar(BAR_DONE));
-    mbar_wait_warp(sm.bar(BAR_DONE), 0, nullptr, p.err, kSiteBwdDrain);
+    umma_commit_warp(bar(BAR_DONE));
+    mbar_wait_warp(bar(BAR_DONE), 0, nullptr, p.err, kSiteBwdDrain);
    }
   } else {
     regs_increase<kBwdRegsElem>();
@@ -415,7 +454,7 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     __nv_bfloat16* drow = reinterpret_cast<__nv_bfloat16*>(p.dq) + ridx * D;
     bool ok = true;
     for (int t = 0; ok && t < n; ++t) {
-      ok = __all_sync(0xffffffffu, mbar_wait(sm.bar(BAR_S), t & 1, abort_flag, p.err, kSiteBwdS));
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(BAR_S), t & 1, abort_flag, p.err, kSiteBwdS));
       if (!ok) break;
       tc_fence_after();
       const int k0 = (ja + t) * kBT;
@@ -434,9 +473,9 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       // S_t is in registers: X may take S_{t+1}
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(sm.bar(BAR_XF));
+      if (lane == 0) mbar_arrive(bar(BAR_XF));
       probs<64>(s, p.kscale, [&](int) { return l2r4; }, [&](int j) { return vis(4 * j); });
-      ok = __all_sync(0xffffffffu, mbar_wait(sm.bar(BAR_DP), t & 1, abort_flag, p.err, kSiteBwdS));
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(BAR_DP), t & 1, abort_flag, p.err, kSiteBwdS));
       if (!ok) break;
       tc_fence_after();
       uint32_t dp[64];
@@ -455,14 +494,14 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(sm.bar(BAR_DS));
+      if (lane == 0) mbar_arrive(bar(BAR_DS));
     }
     // group g writes dQ columns [g D / 2, (g + 1) D / 2) of its row
     if (n == 0) {
       store_zero_row(drow + g * (D / 2), D / 2, valid);
     } else if (ok) {
       const bool okacc =
-          __all_sync(0xffffffffu, mbar_wait(sm.bar(BAR_ACC), 0, abort_flag, p.err, kSiteBwdAcc));
+          __all_sync(0xffffffffu, mbar_wait(bar(BAR_ACC), 0, abort_flag, p.err, kSiteBwdAcc));
       if (okacc) {
         tc_fence_after();
         store_row<D / 2>(tl + kTmemAcc0 + (uint32_t)(g * (D / 2)), p.scale, drow + g * (D / 2),
@@ -778,9 +817,11 @@ template <int D>
 int launch_bwd_t(const CUtensorMap& tq, const CUtensorMap& tdo, const CUtensorMap& tk,
                  const CUtensorMap& tv, const BwdParams& p, cudaStream_t stream) {
   using C = BwdCfg<D>;
-  static_assert(C::kSmemBytes <= 227 * 1024, "shared memory budget");
+  using CQ = DqCfg<D>;
+  static_assert(C::kSmemBytes <= 227 * 1024 && CQ::kSmemBytes <= 227 * 1024,
+                "shared memory budget");
   if (cudaFuncSetAttribute(attn_bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           C::kSmemBytes) != cudaSuccess ||
+                           CQ::kSmemBytes) != cudaSuccess ||
       cudaFuncSetAttribute(attn_bwd_dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            C::kSmemBytes) != cudaSuccess)
     return -4;
@@ -790,8 +831,8 @@ int launch_bwd_t(const CUtensorMap& tq, const CUtensorMap& tdo, const CUtensorMa
     attn_bwd_dkdv_kernel<D><<<(unsigned)nk, kBwdThreads, C::kSmemBytes, stream>>>(tq, tdo, tk,
                                                                                  tv, p);
   if (nq > 0)
-    attn_bwd_dq_kernel<D><<<(unsigned)nq, kBwdThreads, C::kSmemBytes, stream>>>(tq, tdo, tk,
-                                                                               tv, p);
+    attn_bwd_dq_kernel<D><<<(unsigned)nq, kBwdThreads, CQ::kSmemBytes, stream>>>(tq, tdo, tk,
+                                                                                tv, p);
   return cudaGetLastError() == cudaSuccess ? 0 : -4;
 }
 
