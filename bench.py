@@ -345,6 +345,14 @@ def run_ours(args, world, rank, local):
     return out
 
 
+def l2_note(*tensors) -> str:
+    """The L2 statement of a line's config: the inputs every step reads exceed the L2, so no
+    flush is needed between timed steps."""
+    nbytes = sum(t.numel() * t.element_size() for t in tensors)
+    assert nbytes > L2_BYTES, "inputs fit in L2: the line would need an L2 flush"
+    return "inputs larger than L2 (%.0f MB > %.0f MB)" % (nbytes / 1e6, L2_BYTES / 1e6)
+
+
 def bench_extras(args, world, local, peaks, peak_src):
     """The rows beyond the headline: ALiBi and symmetric-window prefill, paged decode, the
     backward pass and the FP8 prefill, one line each."""
@@ -401,7 +409,8 @@ def bench_prefill_variant(w, args, world, local, peaks, peak_src):
     kernel_ms = max_over_ranks(world, sum(per) / len(per))
     peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     achieved = flops / (kernel_ms * 1e-3) / 1e12
-    res = {"config": w.describe(), "value": round(whole_job_rate(flops, world, ms) / 1e12, 2),
+    res = {"config": {**w.describe(), "l2": l2_note(q, k, v)},
+           "value": round(whole_job_rate(flops, world, ms) / 1e12, 2),
            "unit": "TFLOP/s", "ms_per_step": round(ms, 4), "steps": steps,
            "useful_tflop_per_step": round(flops / 1e12, 4),
            "executed_tflop_per_step": round(executed / 1e12, 4),
@@ -456,6 +465,7 @@ def bench_decode_paged(args, world, local, peaks, peak_src, page: int = 256):
     io = accounting.decode_io_bytes(w.B, w.Hq, w.Hkv, w.Nk, w.d) + w.B * max_pages * 4 + w.B * 4
     peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
     res = {"config": {**w.describe(), "page_size": page, "num_pages": num_pages,
+                      "l2": l2_note(kp, vp),
                       "placement": "seeded permutation", "seq_lens": "all T"},
            "value": round(whole_job_rate(kv, world, ms) / 1e9, 1), "unit": "GB/s (KV cache)",
            "tokens_per_s": round(w.B * world / (ms * 1e-3), 1), "ms_per_step": round(ms, 4),
@@ -501,7 +511,8 @@ def bench_backward(w, args, world, local, peaks, peak_src):
     call_ms = max_over_ranks(world, sum(per) / len(per))
     peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     achieved = flops / (call_ms * 1e-3) / 1e12
-    res = {"config": w.describe(), "value": round(whole_job_rate(flops, world, ms) / 1e12, 2),
+    res = {"config": {**w.describe(), "l2": l2_note(q, k, v, o, dout)},
+           "value": round(whole_job_rate(flops, world, ms) / 1e12, 2),
            "unit": "TFLOP/s", "ms_per_step": round(ms, 4), "steps": steps,
            "useful_tflop_per_step": round(flops / 1e12, 4),
            "flop_accounting": "10 d per visible pair (S, dP, dV, dQ, dK)",
@@ -559,6 +570,7 @@ def bench_fp8(w, args, world, local, peaks, peak_src):
     peak = 2.0 * float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     achieved = flops / (call_ms * 1e-3) / 1e12
     res = {"config": {**w.describe(), "dtype": "e4m3 (P e4m3), bf16 O",
+                      "l2": l2_note(q8, k8, vt8),
                       "scales": "Q, K per 128 rows after Hadamard rotation; V per head"},
            "value": round(whole_job_rate(flops, world, ms) / 1e12, 2), "unit": "TFLOP/s",
            "ms_per_step": round(ms, 4), "steps": steps,
@@ -635,7 +647,8 @@ def bench_decode(args, world, local, peaks, peak_src):
     io = accounting.decode_io_bytes(w.B, w.Hq, w.Hkv, w.Nk, w.d)
     peak = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
     gbs = whole_job_rate(kv, world, ms) / 1e9
-    res = {"workload": w.name, "value": round(gbs, 1), "unit": "GB/s (KV cache)",
+    res = {"workload": w.name, "l2": l2_note(kc, vc), "value": round(gbs, 1),
+           "unit": "GB/s (KV cache)",
            "tokens_per_s": round(w.B * world / (ms * 1e-3), 1), "ms_per_step": round(ms, 4),
            "num_splits": S, "kv_bytes_per_step": kv,
            "roofline": {"bound": "hbm", "achieved": round(io / (call_ms * 1e-3) / 1e9, 1),
