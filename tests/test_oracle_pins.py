@@ -688,6 +688,18 @@ def test_rotation_is_orthogonal_and_keeps_the_scores(d):
     assert np.allclose(np.abs(ofp8.rotate(x, signs)), 10.0 / np.sqrt(d))
 
 
+@pytest.mark.parametrize("d", [2, 8, 64, 128])
+def test_hadamard_entries_and_rotation_of_unit_vectors(d):
+    # Sylvester's H has the closed form H[i, j] = (-1)^popcount(i & j); the rotation of the
+    # unit vector e_j is row j of H scaled by the j-th sign and 1/sqrt(d)
+    H = ofp8.hadamard(d)
+    want = np.array([[(-1.0) ** bin(i & j).count("1") for j in range(d)] for i in range(d)])
+    assert np.array_equal(H, want)
+    signs = np.random.default_rng(d + 1).choice([-1.0, 1.0], size=d)
+    R = ofp8.rotate(np.eye(d), signs)
+    assert np.allclose(R, signs[:, None] * want / np.sqrt(d), atol=1e-15, rtol=0)
+
+
 def test_e4m3_grid_points_and_error_bounds():
     # the largest finite E4M3 value is 448; 1 + 2^-3 is a grid point, 1 + 2^-4 a tie that
     # rounds to even (1); normal values round within 2^-4 relative, subnormals (below 2^-6)
