@@ -39,8 +39,10 @@ def _rank_main(rank, world, port, queue):
     queue.put((rank, slowest, rate))
 
 
-def test_two_gloo_ranks_take_the_max_and_aggregate():
-    world, port = 2, _free_port()
+def _run_two_ranks(world):
+    """Runs the ranks once on a fresh port; None if a rank failed (the port picked can be
+    taken by another process between the probe and the rendezvous)."""
+    port = _free_port()
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     procs = [ctx.Process(target=_rank_main, args=(r, world, port, q)) for r in range(world)]
@@ -48,8 +50,22 @@ def test_two_gloo_ranks_take_the_max_and_aggregate():
         p.start()
     for p in procs:
         p.join(timeout=120)
-        assert p.exitcode == 0
-    res = sorted(q.get(timeout=10) for _ in range(world))
+    if any(p.exitcode != 0 for p in procs):
+        for p in procs:
+            if p.is_alive():
+                p.kill()
+        return None
+    return sorted(q.get(timeout=10) for _ in range(world))
+
+
+def test_two_gloo_ranks_take_the_max_and_aggregate():
+    world = 2
+    res = None
+    for _ in range(3):
+        res = _run_two_ranks(world)
+        if res is not None:
+            break
+    assert res is not None, "the two gloo ranks failed three times"
     for rank, slowest, rate in res:
         assert slowest == pytest.approx(1.5 + world - 1)
         # 1e12 units per rank, 2 ranks, slowest 2.5 ms -> 8e14 units/s for the whole job
