@@ -13,6 +13,9 @@
  *   - Tensors are caller-owned DEVICE memory, contiguous, row-major in the order given
  *     ([B, H, N, d] as in PyTorch, "사례 2: 텐서 형태 불일치" on the FlashAttention page).
  *     bf16 arrays are passed as void*.  Every pointer must be 16-byte aligned.
+ *     Each array must hold at least the elements its stated shape implies: the library
+ *     sees only pointers and sizes, so it cannot check an allocation's extent (the Python
+ *     binding checks every tensor's shape, dtype and device before it calls in).
  *   - Calls are asynchronous on `stream`; they never synchronise, never allocate and keep
  *     no state across calls except a per-process cache of device attributes, so they may be
  *     recorded into a CUDA graph with fixed shapes ("CUDA 그래프와의 호환성").

@@ -417,3 +417,65 @@ def device_status(stream=None, device=None) -> int:
                                                                         torch.cuda.current_device())
     with torch.cuda.device(dev):
         return int(lib.attn_get_device_status(_stream(dev, stream)))
+
+
+def attn_fwd_alibi(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
+                   alibi_slopes: torch.Tensor, **kwargs) -> Tuple[torch.Tensor, torch.Tensor]:
+    """attn_fwd with the ALiBi bias: query head h adds -alibi_slopes[h] * |q - kv|."""
+    if alibi_slopes is None:
+        raise ValueError("attn_fwd_alibi needs alibi_slopes (fp32 [Hq] on the device)")
+    return attn_fwd(q, k, v, alibi_slopes=alibi_slopes, **kwargs)
+
+
+def attn_decode_splitkv_noalloc(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                                *, scale: Optional[float] = None,
+                                num_splits: Optional[int] = None,
+                                out: Optional[torch.Tensor] = None,
+                                lse: Optional[torch.Tensor] = None,
+                                stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """attn_decode with the split partials in the library's own device array (no workspace;
+    calls on one device share it, so issue them on one stream)."""
+    lib = _lib.load()
+    for t, n in ((q, "q"), (k_cache, "k_cache"), (v_cache, "v_cache")):
+        _need(t, n, torch.bfloat16, 4)
+    B, Hq, nq, d = q.shape
+    if nq != 1:
+        raise ValueError("decode takes one query token per sequence")
+    Hkv, T = k_cache.shape[1], k_cache.shape[2]
+    _kv_shapes(k_cache, v_cache, B, d, "k_cache", "v_cache")
+    _same_device(q, (k_cache, "k_cache"), (v_cache, "v_cache"))
+    if out is None:
+        out = torch.empty_like(q)
+    _out(out, "out", torch.bfloat16, (B, Hq, 1, d), q)
+    if lse is None:
+        lse = torch.empty((B, Hq, 1), dtype=torch.float32, device=q.device)
+    _out(lse, "lse", torch.float32, (B, Hq, 1), q)
+    with _device(q):
+        st = lib.attn_decode_splitkv_noalloc(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(out),
+                                             _ptr(lse), B, Hq, Hkv, T, d, float(scale or 0.0),
+                                             int(num_splits or 0), _stream(q.device, stream))
+    _check(st, "attn_decode_splitkv_noalloc")
+    return out, lse
+
+
+def attn_status_string(status: int) -> str:
+    return _lib.load().attn_status_string(int(status)).decode()
+
+
+def attn_last_error_site() -> int:
+    """Where the last bounded device wait that ran out gave up (0: none recorded)."""
+    return int(_lib.load().attn_last_error_site())
+
+
+def attn_version() -> int:
+    return int(_lib.load().attn_version())
+
+
+# Every C entry point of include/attn.h under its own name.
+attn_decode_splitkv = attn_decode
+attn_decode_merge = attn_merge
+attn_quantize_fp8 = quantize_fp8
+attn_get_device_status = device_status
+attn_bwd_workspace_bytes = bwd_workspace_bytes
+attn_decode_workspace_bytes = decode_workspace_bytes
+attn_decode_default_splits = default_splits

@@ -220,3 +220,32 @@ def test_tensors_on_another_device_are_refused(lib):
         api.attn_fwd(q, z((1, 2, 128, 64)), z((1, 2, 128, 64)),
                      out=z((1, 4, 128, 64), device="meta"))
     assert lib.calls == []
+
+
+# ------------------------------------------------------------------ one binding per entry point
+
+def test_every_declared_entry_point_has_a_binding_of_the_same_name():
+    import re
+    from pathlib import Path
+
+    import io_aware_softmax_b200 as pkg
+    header = (Path(__file__).resolve().parents[1] / "include" / "attn.h").read_text()
+    names = re.findall(r"ATTN_API\s+[\w\s\*]+?\b(attn_\w+)\s*\(", header)
+    assert len(names) >= 16, names
+    missing = [n for n in names if not callable(getattr(pkg, n, None))]
+    assert not missing, missing
+    assert set(names) <= set(pkg.__all__)
+
+
+def test_noalloc_and_alibi_bindings(lib):
+    q, kc = z((2, 8, 1, 128)), z((2, 2, 700, 128))
+    api.attn_decode_splitkv_noalloc(q, kc, z(kc.shape), num_splits=5)
+    api.attn_fwd_alibi(z((1, 4, 64, 64)), z((1, 2, 64, 64)), z((1, 2, 64, 64)), z((4,), F32),
+                       mask="causal")
+    assert [c[0] for c in lib.calls] == ["attn_decode_splitkv_noalloc", "attn_fwd_alibi"]
+    assert lib.calls[0][1][5:12] == (2, 8, 2, 700, 128, 0.0, 5)
+    with pytest.raises(ValueError):
+        api.attn_decode_splitkv_noalloc(q, kc, z((2, 2, 600, 128)))
+    with pytest.raises(ValueError):
+        api.attn_decode_splitkv_noalloc(q, kc, z(kc.shape), lse=z((2, 8), F32))
+    assert len(lib.calls) == 2

@@ -61,3 +61,15 @@ def test_noalloc_rejects_requests_beyond_its_array():
                                          lse.data_ptr(), B, Hq, Hkv, T, d, ctypes.c_float(0.0),
                                          splits, stream)
     assert st == -6 and lib.attn_status_string(st) == b"workspace missing or too small"
+
+
+def test_python_binding_of_the_same_name():
+    from io_aware_softmax_b200 import attn_decode_splitkv, attn_decode_splitkv_noalloc
+    B, Hq, Hkv, T, d = 3, 8, 2, 1000, 128
+    q = workloads.randn_bf16((B, Hq, 1, d), 77, 0).cuda()
+    kc = workloads.randn_bf16((B, Hkv, T, d), 77, 1).cuda()
+    vc = workloads.randn_bf16((B, Hkv, T, d), 77, 2).cuda()
+    o, lse = attn_decode_splitkv_noalloc(q, kc, vc, num_splits=6)
+    o_ref, lse_ref = attn_decode_splitkv(q, kc, vc, num_splits=6)
+    assert device_status() == 0
+    compare(o, lse, f64(o_ref), f64(lse_ref), "no-alloc binding")
