@@ -45,7 +45,7 @@ What it computes, and where that is written down (pages cited by title and secti
   PagedAttention): "3.7 어텐션 II", sections 3.7.4 and 3.7.8; the sequences of a batch have
   their own lengths, as in the varlen API of section 3.7.6.
 
-Readings taken where the pages are silent (each is listed in the design doc as well):
+Readings taken where the pages are silent:
 
 * soft-cap acts on the *scaled* score: s <- c * tanh(s / c) with s = scale * q.k;
 * causal means kv <= q (diagonal visible); the sliding window is one-sided and causal:
