@@ -3,6 +3,7 @@ the CPU: one JSON line with every key of the benchmark contract, on the same met
 and workload as the GPU arm."""
 import io
 import json
+import os
 from contextlib import redirect_stdout
 
 import bench
@@ -34,3 +35,26 @@ def test_reference_arm_line_at_one_rank(monkeypatch):
     e2e = line["e2e"]
     assert e2e["value"] == line["value"] and e2e["unit"] == line["unit"]
     assert e2e["h2d_bytes_per_step"] == 0 and e2e["d2h_bytes_per_step"] == 0
+
+
+def test_recorded_traffic_is_dropped_once_the_kernel_source_changes(tmp_path, monkeypatch):
+    # a traffic figure is only reported while the measured sources are unchanged
+    import hashlib
+
+    from io_aware_softmax_b200 import build as b
+    csrc = tmp_path / "csrc"
+    csrc.mkdir()
+    (csrc / "k.cu").write_text("__global__ void k() {}\n")
+    digest = hashlib.sha256((csrc / "k.cu").read_bytes()).hexdigest()
+    root = tmp_path / "root"
+    (root / "profiles").mkdir(parents=True)
+    (root / "profiles" / "traffic.json").write_text(json.dumps(
+        {"kern": {"bytes_per_launch": 1234, "sources": ["k.cu"], "sha256": digest}}))
+    monkeypatch.setattr(bench, "ROOT", str(root))
+    monkeypatch.setattr(b, "CSRC", str(csrc))
+    assert bench.recorded_traffic("kern") == 1234
+    assert bench.recorded_traffic("other") is None
+    (csrc / "k.cu").write_text("__global__ void k() { /* changed */ }\n")
+    assert bench.recorded_traffic("kern") is None
+    assert os.path.exists(root / "profiles" / "traffic.json")
+
