@@ -3,12 +3,9 @@
 Tolerances (bf16 inputs, fp32 accumulation, bf16 output, against the fp64 oracle):
 O max-abs 2e-2 and mean-abs 2e-3; LSE max-abs 1e-3.  Tile maps are compared bit-exactly.
 
-Stress cases with larger inputs (std 2-3, outside the workloads' N(0,1) draws) have outputs
-of magnitude ~10, where rounding alone exceeds a fixed 2e-2: P is rounded to bf16 before
-the PV product (relative error <= 2^-9 per weight, so <= 2^-9 * max|V| on O) and O itself
-is rounded to bf16 (<= 2^-9 * |O|).  For those cases ``vmax`` (the largest |V| of the head)
-widens the bound to 2e-2 + 2^-8 * (|O_ref| + vmax) per element, and the mean bound by the
-same factor over unit scale.
+Every case is held to these fixed bounds.  Stress cases that need large scores draw Q and
+K with a wider spread (std 2-3) and V from N(0,1), so the softmax is stressed while |O|
+stays near 1; the packed-document soft-cap cases keep that workload's own N(0,1)*2 draws.
 """
 import numpy as np
 import torch
@@ -22,7 +19,7 @@ def f64(t: torch.Tensor) -> np.ndarray:
     return t.detach().float().cpu().numpy().astype(np.float64)
 
 
-def compare(o_gpu, lse_gpu, o_ref, lse_ref, what="", vmax=None):
+def compare(o_gpu, lse_gpu, o_ref, lse_ref, what=""):
     o = f64(o_gpu) if isinstance(o_gpu, torch.Tensor) else o_gpu
     l = f64(lse_gpu) if isinstance(lse_gpu, torch.Tensor) else lse_gpu
     assert o.shape == o_ref.shape, (what, o.shape, o_ref.shape)
@@ -34,13 +31,8 @@ def compare(o_gpu, lse_gpu, o_ref, lse_ref, what="", vmax=None):
     lerr = np.abs(np.where(inf_ref, 0.0, l - np.where(inf_ref, 0.0, lse_ref)))
     msg = (f"{what}: O max {err.max():.3e} mean {err.mean():.3e}; "
            f"LSE max {lerr.max() if lerr.size else 0:.3e}")
-    if vmax is None:
-        assert err.max() <= TOL_O_MAX, msg
-        assert err.mean() <= TOL_O_MEAN, msg
-    else:
-        bound = TOL_O_MAX + 2.0 ** -8 * (np.abs(o_ref) + vmax)
-        assert np.all(err <= bound), msg + f" (bound {bound.max():.3e})"
-        assert err.mean() <= TOL_O_MEAN * max(1.0, vmax / 4.0), msg
+    assert err.max() <= TOL_O_MAX, msg
+    assert err.mean() <= TOL_O_MEAN, msg
     assert lerr.size == 0 or lerr.max() <= TOL_LSE, msg
     return err.max(), err.mean(), (lerr.max() if lerr.size else 0.0)
 

@@ -15,13 +15,11 @@ pytestmark = pytest.mark.gpu
 def _decode_case(B, Hq, Hkv, T, d, splits, seed, std=1.0):
     q = workloads.randn_bf16((B, Hq, 1, d), seed, 0, std).cuda()
     kc = workloads.randn_bf16((B, Hkv, T, d), seed, 1, std).cuda()
-    vc = workloads.randn_bf16((B, Hkv, T, d), seed, 2, std).cuda()
+    vc = workloads.randn_bf16((B, Hkv, T, d), seed, 2).cuda()     # std widens q and K only
     o, lse = attn_decode(q, kc, vc, num_splits=splits)
     assert device_status() == 0
     O_ref, L_ref = oracle.attention(f64(q), f64(kc), f64(vc))
-    vmax = float(vc.abs().max()) if std > 1.0 else None
-    return compare(o, lse, O_ref, L_ref, f"decode B{B} Hq{Hq} Hkv{Hkv} T{T} d{d} S{splits}",
-                   vmax=vmax)
+    return compare(o, lse, O_ref, L_ref, f"decode B{B} Hq{Hq} Hkv{Hkv} T{T} d{d} S{splits}")
 
 
 @pytest.mark.parametrize("T", [1, 7, 64, 65, 1000, 4097])

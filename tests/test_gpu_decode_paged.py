@@ -16,7 +16,7 @@ def _paged_inputs(B, Hq, Hkv, page, max_pages, d, lens, seed, spare_pages=3, std
     num_pages = B * max_pages + spare_pages
     q = workloads.randn_bf16((B, Hq, 1, d), seed, 0, std, device="cuda")
     kp = workloads.randn_bf16((num_pages, Hkv, page, d), seed, 1, std, device="cuda")
-    vp = workloads.randn_bf16((num_pages, Hkv, page, d), seed, 2, std, device="cuda")
+    vp = workloads.randn_bf16((num_pages, Hkv, page, d), seed, 2, device="cuda")  # std: q, K only
     rng = np.random.default_rng(seed)
     table = rng.permutation(num_pages)[: B * max_pages].reshape(B, max_pages).astype(np.int32)
     return (q, kp, vp, torch.from_numpy(table).cuda(),
@@ -29,9 +29,8 @@ def _paged_case(B, Hq, Hkv, page, max_pages, d, lens, splits, seed, std=1.0):
     o, lse = attn_decode_paged(q, kp, vp, table_t, lens_t, num_splits=splits)
     assert device_status() == 0
     O_ref, L_ref = oracle.decode_paged(f64(q), f64(kp), f64(vp), table, np.asarray(lens))
-    vmax = float(vp.abs().max()) if std > 1.0 else None
     return compare(o, lse, O_ref, L_ref,
-                   f"paged B{B} Hq{Hq} Hkv{Hkv} page{page} lens{lens} d{d} S{splits}", vmax=vmax)
+                   f"paged B{B} Hq{Hq} Hkv{Hkv} page{page} lens{lens} d{d} S{splits}")
 
 
 @pytest.mark.parametrize("page", [64, 128, 256])

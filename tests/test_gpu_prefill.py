@@ -15,16 +15,17 @@ pytestmark = pytest.mark.gpu
 MASK_ID = {"none": 0, "causal": 1, "sliding_causal": 2, "document_causal": 3, "sliding": 4}
 
 
-def _inputs(B, Hq, Hkv, Nq, Nk, d, seed, std=1.0):
+def _inputs(B, Hq, Hkv, Nq, Nk, d, seed, std=1.0, v_std=1.0):
+    # std widens Q and K (larger scores); V keeps its own spread
     q = workloads.randn_bf16((B, Hq, Nq, d), seed, 0, std).cuda()
     k = workloads.randn_bf16((B, Hkv, Nk, d), seed, 1, std).cuda()
-    v = workloads.randn_bf16((B, Hkv, Nk, d), seed, 2, std).cuda()
+    v = workloads.randn_bf16((B, Hkv, Nk, d), seed, 2, v_std).cuda()
     return q, k, v
 
 
 def _run_full(B, Hq, Hkv, Nq, Nk, d, mask="none", window=0, softcap=0.0, docs=None, seed=0,
-              std=1.0, scale=None, slopes=None):
-    q, k, v = _inputs(B, Hq, Hkv, Nq, Nk, d, seed, std)
+              std=1.0, scale=None, slopes=None, v_std=1.0):
+    q, k, v = _inputs(B, Hq, Hkv, Nq, Nk, d, seed, std, v_std)
     doc_t = None if docs is None else torch.tensor(docs, dtype=torch.int32, device="cuda")
     # guard bands around the outputs catch writes past the last row
     o_buf = torch.full((B * Hq * Nq * d + 4096,), float("nan"), dtype=torch.bfloat16, device="cuda")
@@ -39,10 +40,8 @@ def _run_full(B, Hq, Hkv, Nq, Nk, d, mask="none", window=0, softcap=0.0, docs=No
     O_ref, L_ref = oracle.attention(f64(q), f64(k), f64(v), scale=scale, mask_kind=MASK_ID[mask],
                                     window=window, softcap=softcap, doc_offsets=docs,
                                     alibi_slopes=slopes)
-    vmax = float(v.abs().max()) if std > 1.0 else None
     return compare(o, lse, O_ref, L_ref,
-                   f"{B}x{Hq}/{Hkv}x{Nq}x{Nk}x{d} {mask} w{window} c{softcap} alibi{slopes}",
-                   vmax=vmax)
+                   f"{B}x{Hq}/{Hkv}x{Nq}x{Nk}x{d} {mask} w{window} c{softcap} alibi{slopes}")
 
 
 def test_tiny_workload_noncausal_and_causal():
@@ -84,7 +83,9 @@ def test_document_mask(docs):
 @pytest.mark.parametrize("mask", ["none", "causal", "document_causal"])
 def test_softcap(mask):
     docs = [0, 200, 513, 800] if mask == "document_causal" else None
-    _run_full(1, 2, 2, 800, 800, 128, mask=mask, softcap=50.0, docs=docs, seed=3, std=2.0)
+    # the packed-document workload's inputs: Q, K and V all N(0,1) * 2
+    _run_full(1, 2, 2, 800, 800, 128, mask=mask, softcap=50.0, docs=docs, seed=3, std=2.0,
+              v_std=2.0)
     _run_full(1, 2, 2, 300, 300, 64, mask=mask if mask != "document_causal" else "causal",
               softcap=5.0, seed=4, std=3.0)
 
