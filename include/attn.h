@@ -214,7 +214,8 @@ ATTN_API int attn_decode_splitkv(const void* q, const void* k_cache, const void*
  *   overlap on the GPU race, so issue them on one stream.  The first call on each device looks
  *   up the array's device address (with that device current); make that first call before
  *   any stream capture.  No allocation happens in any call.
- * Errors: as attn_decode_splitkv.
+ * Errors: as attn_decode_splitkv, checked in the same order first, so an invalid request gets
+ * the same status from both; WORKSPACE then means a valid request too large for the array.
  */
 ATTN_API int attn_decode_splitkv_noalloc(const void* q, const void* k_cache, const void* v_cache,
                                          void* o, float* lse, int B, int Hq, int Hkv, int T,

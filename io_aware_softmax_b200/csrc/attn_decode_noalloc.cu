@@ -10,9 +10,10 @@
 // q, the caches and the outputs.
 //
 // Limits and rules of use:
-//   * the array is kNoAllocWorkspaceBytes (32 MiB); a request whose partials would not fit
-//     (B * Hq * splits * (d + 1) * 4 bytes, plus alignment) is rejected with
-//     ATTN_ERR_WORKSPACE before anything runs;
+//   * the array is kNoAllocWorkspaceBytes (32 MiB); a valid request whose partials would not
+//     fit (B * Hq * splits * (d + 1) * 4 bytes, plus alignment) is rejected with
+//     ATTN_ERR_WORKSPACE before anything runs (invalid arguments get attn_decode_splitkv's
+//     own statuses first);
 //   * every GPU that loads the library holds the array until the process exits;
 //   * all calls share the one array per device, so two calls that overlap on the GPU (other
 //     streams, other threads) race on it; serialise them on one stream;
@@ -24,6 +25,7 @@
 //     stream capture.
 #include <cuda_runtime.h>
 
+#include <cmath>
 #include <cstdint>
 #include <mutex>
 
@@ -57,13 +59,24 @@ extern "C" int attn_decode_splitkv_noalloc(const void* q, const void* k_cache,
                                            const void* v_cache, void* o, float* lse, int B,
                                            int Hq, int Hkv, int T, int d, float scale,
                                            int num_splits, cudaStream_t stream) {
+  // The argument checks of attn_decode_splitkv come first, in its order, so that an invalid
+  // request gets the same status from both entry points whatever its size.
   if (B < 0 || Hq < 0 || Hkv < 0 || T < 0) return ATTN_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (Hkv == 0 && Hq > 0) return ATTN_ERR_INVALID_ARG;
+  if (Hkv > 0 && Hq % Hkv != 0) return ATTN_ERR_UNSUPPORTED;
+  if (std::isnan(scale)) return ATTN_ERR_INVALID_ARG;
   if (B == 0 || Hq == 0 || T == 0) {
     // nothing needs partials: the regular entry point handles these without a workspace
     return attn_decode_splitkv(q, k_cache, v_cache, o, lse, B, Hq, Hkv, T, d, scale,
                                num_splits, nullptr, 0, stream);
   }
+  if (Hq / Hkv > 16) return ATTN_ERR_UNSUPPORTED;
+  if (!q || !o || !lse || !k_cache || !v_cache) return ATTN_ERR_INVALID_ARG;
+  auto misaligned = [](const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) != 0; };
+  if (misaligned(q) || misaligned(o) || misaligned(lse) || misaligned(k_cache) ||
+      misaligned(v_cache))
+    return ATTN_ERR_MISALIGNED;
   int device = 0;
   if (cudaGetDevice(&device) != cudaSuccess) return ATTN_ERR_CUDA;
   int splits = num_splits;
