@@ -273,6 +273,19 @@ ATTN_API int attn_decode_merge(const float* o_part, const float* lse_part, void*
 ATTN_API int attn_get_device_status(cudaStream_t stream);
 ATTN_API int attn_last_error_site(void);
 
+/*
+ * attn_set_wait_limit_ns -- sets, on the current device, how long a kernel's pipeline waits
+ * (a warp waiting for a tile, a product or a free buffer) may last before the kernel gives up
+ * and reports ATTN_ERR_DEVICE_TIMEOUT; 0 restores the built-in 0.5 s.  The waits of a
+ * kernel's teardown (for its own copies and products still in flight) keep the full limit,
+ * so a kernel that gave up still exits cleanly and later calls run normally.  It exists to
+ * exercise the failure path ("3.7 어텐션 II", 3.7.3: a failure is reported, never hidden): a
+ * limit of a few nanoseconds makes the first wait that is not already satisfied run out.
+ * It synchronises the device first; call it with no call of this library in flight.
+ * Errors: CUDA.
+ */
+ATTN_API int attn_set_wait_limit_ns(unsigned long long ns);
+
 /* Human-readable name of a status code (static storage). */
 ATTN_API const char* attn_status_string(int status);
 

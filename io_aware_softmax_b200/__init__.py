@@ -13,7 +13,7 @@ from .api import (  # noqa: F401
     attn_decode_default_splits, attn_decode_merge, attn_decode_paged, attn_decode_splitkv,
     attn_decode_splitkv_noalloc, attn_decode_workspace_bytes, attn_fwd, attn_fwd_alibi,
     attn_fwd_fp8, attn_get_device_status, attn_last_error_site, attn_merge, attn_quantize_fp8,
-    attn_status_string, attn_version, bwd_workspace_bytes, decode_workspace_bytes,
+    attn_set_wait_limit_ns, attn_status_string, attn_version, bwd_workspace_bytes, decode_workspace_bytes,
     default_splits, device_status, quantize_fp8,
 )
 from ._lib import LIB_PATH, LibraryMissing, load as load_library  # noqa: F401
@@ -23,7 +23,8 @@ __all__ = [
     "attn_fwd", "attn_fwd_alibi", "attn_bwd", "attn_bwd_workspace_bytes", "attn_quantize_fp8",
     "attn_fwd_fp8", "attn_blockmap", "attn_decode_workspace_bytes", "attn_decode_default_splits",
     "attn_decode_splitkv", "attn_decode_splitkv_noalloc", "attn_decode_paged",
-    "attn_decode_merge", "attn_get_device_status", "attn_last_error_site", "attn_status_string",
+    "attn_decode_merge", "attn_get_device_status", "attn_last_error_site",
+    "attn_set_wait_limit_ns", "attn_status_string",
     "attn_version",
     # shorter names for the same functions
     "attn_decode", "attn_merge", "quantize_fp8", "bwd_workspace_bytes", "decode_workspace_bytes",

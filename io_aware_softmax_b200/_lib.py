@@ -50,6 +50,7 @@ SIGNATURES = {
                                   c_int, c_void_p]),
     "attn_get_device_status": (c_int, [c_void_p]),
     "attn_last_error_site": (c_int, []),
+    "attn_set_wait_limit_ns": (c_int, [ctypes.c_ulonglong]),
     "attn_status_string": (ctypes.c_char_p, [c_int]),
     "attn_version": (c_int, []),
 }

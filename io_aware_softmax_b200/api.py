@@ -467,6 +467,16 @@ def attn_last_error_site() -> int:
     return int(_lib.load().attn_last_error_site())
 
 
+def attn_set_wait_limit_ns(ns: int, device=None) -> None:
+    """Limit of the kernels' pipeline waits on ``device`` (0: the built-in 0.5 s).  A wait
+    that runs out makes the call report ATTN_ERR_DEVICE_TIMEOUT through device_status()."""
+    lib = _lib.load()
+    dev = torch.device(device) if device is not None else torch.device("cuda",
+                                                                        torch.cuda.current_device())
+    with torch.cuda.device(dev):
+        _check(lib.attn_set_wait_limit_ns(int(ns)), "attn_set_wait_limit_ns")
+
+
 def attn_version() -> int:
     return int(_lib.load().attn_version())
 

@@ -15,8 +15,9 @@
 
 namespace attn {
 
-// The library's device error word: [0] = error bits, [1] = first failing wait site.
-__device__ uint32_t g_error[2] = {0u, 0u};
+// The library's device error word: [0] = error bits, [1] = first failing wait site,
+// [2..3] = limit of the kernels' pipeline waits in ns (64-bit; 0: the built-in 0.5 s).
+__device__ __align__(8) uint32_t g_error[4] = {0u, 0u, 0u, 0u};
 
 namespace {
 
@@ -327,6 +328,14 @@ extern "C" int attn_get_device_status(cudaStream_t stream) {
 }
 
 extern "C" int attn_last_error_site(void) { return g_last_site; }
+
+extern "C" int attn_set_wait_limit_ns(unsigned long long ns) {
+  const uint64_t v = ns;
+  if (cudaDeviceSynchronize() != cudaSuccess) return ATTN_ERR_CUDA;
+  return cudaMemcpyToSymbol(g_error, &v, sizeof(v), 2 * sizeof(uint32_t)) == cudaSuccess
+             ? ATTN_OK
+             : ATTN_ERR_CUDA;
+}
 
 extern "C" int attn_decode_paged(const void* q, const void* k_pages, const void* v_pages,
                                  const int* block_table, const int* seq_lens, void* o, float* lse,

@@ -357,6 +357,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
     if (lane == 0) {
       tma_prefetch_desc(&tmQ);
       int pairs = 0;
+      int loads[2] = {0, 0};   // Q loads issued per query tile (they differ after an abort)
       for_each_pair(p, [&](int bh, int pair) -> bool {
         const PairWork w = make_pair_work(p, bh, pair);
         for (int t = 0; t < 2; ++t) {
@@ -368,13 +369,15 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
           for (int c = 0; c < C::kChunks; ++c)
             tma_load_3d(sQ + t * C::kTileBytes + c * C::kChunkBytes, &tmQ, bar(BAR_Q + t),
                         c * (128 / C::kElem), w.q_first + t * kBM, w.b * p.Hq + w.h);
+          ++loads[t];
         }
         ++pairs;
         return true;
       });
-      if (pairs > 0)
-        for (int t = 0; t < 2; ++t)
-          mbar_wait(bar(BAR_Q + t), (pairs - 1) & 1, nullptr, p.err, kSiteDrain);
+      // The last load of each tile must land before the CTA may exit.
+      for (int t = 0; t < 2; ++t)
+        if (loads[t] > 0)
+          mbar_wait(bar(BAR_Q + t), (loads[t] - 1) & 1, nullptr, p.err, kSiteDrain);
     }
     __syncwarp();
    } else if (warp == kMmaWarp) {

@@ -14,6 +14,10 @@ namespace attn {
 // library's device error word (err[0] = bits, err[1] = first site; its address is passed to
 // every kernel), raises the CTA's abort flag and returns false; the kernel then unwinds,
 // frees its TMEM and exits.  The host reads the word with attn_get_device_status().
+// err[2..3] hold the limit of the pipeline waits in nanoseconds (a 64-bit value; 0 means
+// kWaitLimitNs), which attn_set_wait_limit_ns() lowers so that a test can make a wait run
+// out; the teardown's drain waits always keep kWaitLimitNs, so no copy or product is in
+// flight when a CTA exits.
 enum : uint32_t {
   kErrWaitTimeout = 1u << 0,
   kErrBadArgument = 1u << 1,
@@ -92,18 +96,28 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parit
 
 constexpr uint32_t kWaitSleepNs = 200u * 1000u;   // one sleep of a waiting thread, at most
 
+// Limit of a wait: the library's setting for pipeline waits (abort != nullptr), the full
+// kWaitLimitNs for drain waits.
+__device__ __forceinline__ uint64_t wait_limit_ns(const uint32_t* err, const volatile int* abort) {
+  if (abort == nullptr) return kWaitLimitNs;
+  const uint64_t v = *reinterpret_cast<const volatile uint64_t*>(err + 2);
+  return v != 0 ? v : kWaitLimitNs;
+}
+
 // Waits for the phase with the given parity to complete.  Returns false (after recording
-// the error and raising *abort) if it does not complete within kWaitLimitNs, or if another
+// the error and raising *abort) if it does not complete within its limit, or if another
 // thread of the CTA has already raised *abort.  With abort == nullptr (the drain waits of
 // the teardown) only the time limit ends the wait.
 static __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort,
                                                  uint32_t* err, uint32_t site) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
+  const uint64_t limit = wait_limit_ns(err, abort);
+  const uint32_t sleep_ns = limit < kWaitSleepNs ? (uint32_t)limit : kWaitSleepNs;
   for (;;) {
-    if (mbar_try_wait_sleep(bar, parity, kWaitSleepNs)) return true;
+    if (mbar_try_wait_sleep(bar, parity, sleep_ns)) return true;
     if (abort != nullptr && *abort) return false;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+    if (globaltimer_ns() - t0 > limit) {
       report_error(err, kErrWaitTimeout, site);
       if (abort != nullptr) *abort = 1;
       return false;
@@ -118,9 +132,11 @@ static __device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t par
                                                       uint32_t site) {
   if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
   const uint64_t t0 = globaltimer_ns();
+  const uint64_t limit = wait_limit_ns(err, abort);
+  const uint32_t sleep_ns = limit < kWaitSleepNs ? (uint32_t)limit : kWaitSleepNs;
   for (;;) {
-    if (__all_sync(0xffffffffu, mbar_try_wait_sleep(bar, parity, kWaitSleepNs))) return true;
-    const bool stop = (abort != nullptr && *abort) || globaltimer_ns() - t0 > kWaitLimitNs;
+    if (__all_sync(0xffffffffu, mbar_try_wait_sleep(bar, parity, sleep_ns))) return true;
+    const bool stop = (abort != nullptr && *abort) || globaltimer_ns() - t0 > limit;
     if (__any_sync(0xffffffffu, stop)) {
       if ((threadIdx.x & 31) == 0 && !(abort != nullptr && *abort)) {
         report_error(err, kErrWaitTimeout, site);
