@@ -126,6 +126,21 @@ ATTN_API int attn_bwd(const void* q, const void* k, const void* v, const void* o
              cudaStream_t stream);
 
 /*
+ * attn_bwd_alibi -- attn_bwd for scores that carry the ALiBi bias of attn_fwd_alibi
+ * ("3.7 어텐션 II", 3.7.5).  The bias depends on positions only, so the gradients keep the
+ * form of attn_bwd with P recomputed from the biased scores:
+ * P_ij = exp(scale q_i.k_j - slope_h |i - j| - LSE_i).
+ *   alibi_slopes  device fp32 [Hq], 4-byte aligned (the slopes given to attn_fwd_alibi;
+ *                 o and lse must come from that call); NULL behaves as attn_bwd.
+ * Every other argument, the workspace and the errors as attn_bwd.
+ */
+ATTN_API int attn_bwd_alibi(const void* q, const void* k, const void* v, const void* o,
+             const void* dout, const float* lse, void* dq, void* dk, void* dv, int B, int Hq,
+             int Hkv, int Nq, int Nk, int d, float scale, int mask_kind, int window,
+             float softcap, const int* doc_offsets, int num_docs, const float* alibi_slopes,
+             void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/*
  * attn_quantize_fp8 -- block quantization to E4M3 ("FlashAttention 논문 분석", section
  * "FP8 지원과 정확도 유지": an independent scale per block; Q and K optionally multiplied by a
  * random orthogonal matrix first, which leaves Q K^T unchanged).

@@ -276,8 +276,9 @@ __device__ __forceinline__ void issue_ts(uint32_t acc, uint32_t a_tmem, uint32_t
                  idesc, (!first || kk > 0) ? 1u : 0u);
 }
 
-// dQ of one 128-row query tile of head (b, h).
-template <int D>
+// dQ of one 128-row query tile of head (b, h).  kAlibi: the scores carry the ALiBi bias
+// -slope_h |q - kv|, which moves each P element's base-2 offset from l2 to l2 + slope2 |q - kv|.
+template <int D, bool kAlibi>
 __global__ void __launch_bounds__(kBwdThreads, 1)
 attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO,
                    const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
@@ -447,6 +448,7 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     const float dr = valid ? p.dvec[ridx] : 0.f;
     const float4 l2r4 = make_float4(l2r, l2r, l2r, l2r);
     const float4 dr4 = make_float4(dr, dr, dr, dr);
+    const float slope2 = kAlibi ? __ldg(p.alibi + h) * kLog2eB : 0.f;
     int rlo = 1, rhi = 0;
     if (valid) row_interval(p.mask, row, rlo, rhi);
     const uint32_t tl = tmem + ((uint32_t)(wq * 32) << 16);
@@ -474,7 +476,17 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(BAR_XF));
-      probs<64>(s, p.kscale, [&](int) { return l2r4; }, [&](int j) { return vis(4 * j); });
+      if constexpr (kAlibi) {
+        // key kc + c is |row - kc - c| away from this row
+        const float drow = (float)(row - kc);
+        probs<64>(s, p.kscale, [&](int j) {
+          const float c = (float)(4 * j);
+          return make_float4(fmaf(slope2, fabsf(drow - c), l2r), fmaf(slope2, fabsf(drow - c - 1.f), l2r),
+                             fmaf(slope2, fabsf(drow - c - 2.f), l2r), fmaf(slope2, fabsf(drow - c - 3.f), l2r));
+        }, [&](int j) { return vis(4 * j); });
+      } else {
+        probs<64>(s, p.kscale, [&](int) { return l2r4; }, [&](int j) { return vis(4 * j); });
+      }
       ok = __all_sync(0xffffffffu, mbar_wait(bar(BAR_DP), t & 1, abort_flag, p.err, kSiteBwdS));
       if (!ok) break;
       tc_fence_after();
@@ -518,8 +530,9 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   }
 }
 
-// dK and dV of one 128-key tile of KV head (b, hk), summed over the query heads of its group.
-template <int D>
+// dK and dV of one 128-key tile of KV head (b, hk), summed over the query heads of its group
+// (kAlibi as for attn_bwd_dq_kernel, with the slope of each streamed tile's query head).
+template <int D, bool kAlibi>
 __global__ void __launch_bounds__(kBwdThreads, 1)
 attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ,
                      const __grid_constant__ CUtensorMap tmDO,
@@ -742,7 +755,20 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ,
         }
         return m;
       };
-      auto l2f = [&](int c) { return *reinterpret_cast<const float4*>(l2v + c); };
+      // ALiBi: query q0 + col + c is |key - q0 - col - c| away from this key
+      const float slope2 = kAlibi ? __ldg(p.alibi + hk * p.G + t / ni) * kLog2eB : 0.f;
+      const float dkey = (float)(key - q0 - (int)col);
+      auto l2f = [&](int c) {
+        float4 l = *reinterpret_cast<const float4*>(l2v + c);
+        if constexpr (kAlibi) {
+          const float fc = (float)c;
+          l.x = fmaf(slope2, fabsf(dkey - fc), l.x);
+          l.y = fmaf(slope2, fabsf(dkey - fc - 1.f), l.y);
+          l.z = fmaf(slope2, fabsf(dkey - fc - 2.f), l.z);
+          l.w = fmaf(slope2, fabsf(dkey - fc - 3.f), l.w);
+        }
+        return l;
+      };
       auto dvf = [&](int c) { return *reinterpret_cast<const float4*>(dv + c); };
       // Step 1 (S^T ready): P^T of the group's 64 columns, in two halves of 32; the bf16
       // P^T of a half lands in columns the group has already read.
@@ -813,25 +839,25 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ,
   }
 }
 
-template <int D>
+template <int D, bool kAlibi>
 int launch_bwd_t(const CUtensorMap& tq, const CUtensorMap& tdo, const CUtensorMap& tk,
                  const CUtensorMap& tv, const BwdParams& p, cudaStream_t stream) {
   using C = BwdCfg<D>;
   using CQ = DqCfg<D>;
   static_assert(C::kSmemBytes <= 227 * 1024 && CQ::kSmemBytes <= 227 * 1024,
                 "shared memory budget");
-  if (cudaFuncSetAttribute(attn_bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  if (cudaFuncSetAttribute(attn_bwd_dq_kernel<D, kAlibi>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            CQ::kSmemBytes) != cudaSuccess ||
-      cudaFuncSetAttribute(attn_bwd_dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+      cudaFuncSetAttribute(attn_bwd_dkdv_kernel<D, kAlibi>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            C::kSmemBytes) != cudaSuccess)
     return -4;
   const long long nq = (long long)p.B * p.Hq * ((p.Nq + kBT - 1) / kBT);
   const long long nk = (long long)p.B * p.Hkv * ((p.Nk + kBT - 1) / kBT);
   if (nk > 0)
-    attn_bwd_dkdv_kernel<D><<<(unsigned)nk, kBwdThreads, C::kSmemBytes, stream>>>(tq, tdo, tk,
+    attn_bwd_dkdv_kernel<D, kAlibi><<<(unsigned)nk, kBwdThreads, C::kSmemBytes, stream>>>(tq, tdo, tk,
                                                                                  tv, p);
   if (nq > 0)
-    attn_bwd_dq_kernel<D><<<(unsigned)nq, kBwdThreads, CQ::kSmemBytes, stream>>>(tq, tdo, tk,
+    attn_bwd_dq_kernel<D, kAlibi><<<(unsigned)nq, kBwdThreads, CQ::kSmemBytes, stream>>>(tq, tdo, tk,
                                                                                 tv, p);
   return cudaGetLastError() == cudaSuccess ? 0 : -4;
 }
@@ -851,8 +877,11 @@ int launch_bwd_rowdot(const void* o, const void* dout, const float* lse, float* 
 
 int launch_attn_bwd(const CUtensorMap& tq, const CUtensorMap& tdo, const CUtensorMap& tk,
                     const CUtensorMap& tv, const BwdParams& p, int d, cudaStream_t stream) {
-  if (d == 128) return launch_bwd_t<128>(tq, tdo, tk, tv, p, stream);
-  if (d == 64) return launch_bwd_t<64>(tq, tdo, tk, tv, p, stream);
+  const bool alibi = p.alibi != nullptr;
+  if (d == 128) return alibi ? launch_bwd_t<128, true>(tq, tdo, tk, tv, p, stream)
+                             : launch_bwd_t<128, false>(tq, tdo, tk, tv, p, stream);
+  if (d == 64) return alibi ? launch_bwd_t<64, true>(tq, tdo, tk, tv, p, stream)
+                            : launch_bwd_t<64, false>(tq, tdo, tk, tv, p, stream);
   return -2;
 }
 

@@ -57,6 +57,7 @@ struct BwdParams {
   float kscale;       // scale * log2(e)
   float scale;
   MaskParams mask;
+  const float* alibi;  // fp32 [Hq] ALiBi slopes (natural-log units), or nullptr
   uint32_t* err;      // device error word of the library (bits, first site)
 };
 

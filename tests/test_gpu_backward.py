@@ -39,20 +39,23 @@ def compare_grad(got, ref, what):
     assert rmax <= TOL_MAX and rmean <= TOL_MEAN, f"{what}: max {rmax:.3e}, mean {rmean:.3e}"
 
 
-def _run(B, Hq, Hkv, Nq, Nk, d, mask="none", window=0, docs=None, seed=0, scale=None):
+def _run(B, Hq, Hkv, Nq, Nk, d, mask="none", window=0, docs=None, seed=0, scale=None,
+         slopes=None):
     q = workloads.randn_bf16((B, Hq, Nq, d), seed, 0).cuda()
     k = workloads.randn_bf16((B, Hkv, Nk, d), seed, 1).cuda()
     v = workloads.randn_bf16((B, Hkv, Nk, d), seed, 2).cuda()
     dout = workloads.randn_bf16((B, Hq, Nq, d), seed, 3).cuda()
     doc_t = None if docs is None else torch.tensor(docs, dtype=torch.int32, device="cuda")
-    o, lse = attn_fwd(q, k, v, scale=scale, mask=mask, window=window, doc_offsets=doc_t)
+    slopes_t = None if slopes is None else torch.tensor(slopes, dtype=torch.float32, device="cuda")
+    o, lse = attn_fwd(q, k, v, scale=scale, mask=mask, window=window, doc_offsets=doc_t,
+                      alibi_slopes=slopes_t)
     dq, dk, dv = attn_bwd(q, k, v, o, lse, dout, scale=scale, mask=mask, window=window,
-                          doc_offsets=doc_t)
+                          doc_offsets=doc_t, alibi_slopes=slopes_t)
     assert device_status() == 0
     rq, rk, rv = oracle.attention_backward(f64(q), f64(k), f64(v), f64(dout), scale=scale,
                                            mask_kind=MASK_ID[mask], window=window,
-                                           doc_offsets=docs)
-    tag = f"{B}x{Hq}/{Hkv}x{Nq}x{Nk}x{d} {mask} w{window}"
+                                           doc_offsets=docs, alibi_slopes=slopes)
+    tag = f"{B}x{Hq}/{Hkv}x{Nq}x{Nk}x{d} {mask} w{window}" + ("" if slopes is None else " alibi")
     compare_grad(dq, rq, "dQ " + tag)
     compare_grad(dk, rk, "dK " + tag)
     compare_grad(dv, rv, "dV " + tag)
@@ -84,6 +87,22 @@ def test_document_mask():
 @pytest.mark.parametrize("Nq,Nk", [(100, 300), (300, 129), (1, 200)])
 def test_non_square_unmasked(Nq, Nk):
     _run(1, 2, 1, Nq, Nk, 128, seed=Nq + Nk, scale=0.2)
+
+
+def _geometric_slopes(H):
+    return [2.0 ** (-8.0 * (h + 1) / H) for h in range(H)]
+
+
+@pytest.mark.parametrize("mask,N,d", [("causal", 300, 128), ("none", 257, 64),
+                                      ("sliding", 700, 128)])
+def test_alibi(mask, N, d):
+    # GQA (4 query heads on 2 KV heads): the dK/dV kernel takes each streamed tile's slope
+    _run(1, 4, 2, N, N, d, mask=mask, window=130, seed=N + d, slopes=_geometric_slopes(4))
+
+
+def test_alibi_steep_slopes_and_ragged_tail():
+    # slopes up to 2: the bias dominates the scores and P concentrates near the diagonal
+    _run(2, 2, 1, 129, 129, 128, mask="causal", seed=21, slopes=[2.0, 0.03])
 
 
 def test_softcap_is_unsupported():
