@@ -111,12 +111,13 @@ ATTN_API int attn_fwd_alibi(const void* q, const void* k, const void* v, void* o
  *   q, k, v, o, lse   as attn_fwd (o and lse: attn_fwd's outputs for these inputs)
  *   dout         bf16 [B, Hq, Nq, d]   gradient of the loss with respect to o
  *   dq           bf16 [B, Hq, Nq, d]   dk, dv  bf16 [B, Hkv, Nk, d]   (written)
- *   mask_kind, window, doc_offsets, num_docs, scale   as attn_fwd; softcap must be <= 0
+ *   mask_kind, window, doc_offsets, num_docs, scale, softcap   as attn_fwd (with a soft-cap
+ *                the capped score y = c tanh(x / c) passes dy (1 - tanh^2(x / c)) on to x)
  *   workspace    device, 16-byte aligned, attn_bwd_workspace_bytes(B, Hq, Nq) bytes (the
  *                per-row rowsum(dO * O) and base-2 LSE); contents are scratch
  * Three kernel launches on `stream`, no host synchronisation.  Rows with no visible key
  * (LSE = -inf) contribute nothing; keys no query sees get dK = dV = 0.
- * Errors: as attn_fwd, plus UNSUPPORTED for softcap > 0 and WORKSPACE.
+ * Errors: as attn_fwd, plus WORKSPACE.
  */
 ATTN_API size_t attn_bwd_workspace_bytes(int B, int Hq, int Nq);
 ATTN_API int attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
@@ -132,7 +133,8 @@ ATTN_API int attn_bwd(const void* q, const void* k, const void* v, const void* o
  * P_ij = exp(scale q_i.k_j - slope_h |i - j| - LSE_i).
  *   alibi_slopes  device fp32 [Hq], 4-byte aligned (the slopes given to attn_fwd_alibi;
  *                 o and lse must come from that call); NULL behaves as attn_bwd.
- * Every other argument, the workspace and the errors as attn_bwd.
+ * Every other argument, the workspace and the errors as attn_bwd, plus UNSUPPORTED for
+ * slopes together with softcap > 0 (as attn_fwd_alibi).
  */
 ATTN_API int attn_bwd_alibi(const void* q, const void* k, const void* v, const void* o,
              const void* dout, const float* lse, void* dq, void* dk, void* dv, int B, int Hq,

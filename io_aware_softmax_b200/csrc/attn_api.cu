@@ -426,7 +426,7 @@ extern "C" int attn_bwd_alibi(const void* q, const void* k, const void* v, const
   int st = check_mask(mask_kind, window, doc_offsets, num_docs, Nq, Nk);
   if (st != ATTN_OK) return st;
   if (std::isnan(scale) || std::isnan(softcap)) return ATTN_ERR_INVALID_ARG;
-  if (softcap > 0.f) return ATTN_ERR_UNSUPPORTED;
+  if (softcap > 0.f && alibi_slopes != nullptr) return ATTN_ERR_UNSUPPORTED;
   if (B == 0 || Hq == 0 || (Nq == 0 && Nk == 0)) return ATTN_OK;
   const void* ptrs[] = {q, k, v, o, dout, lse, dq, dk, dv};
   const int needed[] = {Nq > 0, Nk > 0, Nk > 0, Nq > 0, Nq > 0, Nq > 0, Nq > 0, Nk > 0, Nk > 0};
@@ -461,6 +461,8 @@ extern "C" int attn_bwd_alibi(const void* q, const void* k, const void* v, const
   p.scale = scale;
   p.mask = mask_params(mask_kind, window, doc_offsets, num_docs, Nq, Nk);
   p.alibi = alibi_slopes;
+  p.cap_scale = softcap > 0.f ? scale / softcap : 0.f;
+  p.cap_log2 = softcap > 0.f ? softcap * kLog2e : 0.f;
   p.err = error_word_ptr(dev);
   if (p.err == nullptr) return ATTN_ERR_CUDA;
   if (Nq > 0 && launch_bwd_rowdot(o, dout, lse, const_cast<float*>(p.dvec),

@@ -186,7 +186,7 @@ def test_backward_validation(lib):
                          kw.get("d", 128), 0.0, kw.get("mask", 1), 0, kw.get("cap", 0.0), None, 0,
                          kw.get("ws", P), kw.get("wsb", 1 << 20), None]
     assert f(*args(d=96)) == -2
-    assert f(*args(cap=30.0)) == -2
+    assert f(*args(cap=float("nan"))) == -1
     assert f(*args(mask=9)) == -1
     assert f(*args(q=ctypes.c_void_p(24))) == -3
     assert f(*args(ws=None, wsb=0)) == -6
