@@ -360,8 +360,8 @@ def bench_extras(args, world, local, peaks, peak_src):
           for x in (workloads.ALIBI_MHA, workloads.SWA_SYM_GQA)}
     paged = bench_decode_paged(args, world, local, peaks, peak_src)
     ex["paged_" + paged["config"]["workload"]] = paged
-    ex["backward_" + workloads.CAUSAL_MHA.name] = bench_backward(
-        workloads.CAUSAL_MHA, args, world, local, peaks, peak_src)
+    for x in (workloads.CAUSAL_MHA, workloads.ALIBI_MHA, workloads.DOC_SOFTCAP):
+        ex["backward_" + x.name] = bench_backward(x, args, world, local, peaks, peak_src)
     ex["fp8_" + workloads.CAUSAL_MHA.name] = bench_fp8(
         workloads.CAUSAL_MHA, args, world, local, peaks, peak_src)
     return ex
@@ -484,20 +484,28 @@ def bench_decode_paged(args, world, local, peaks, peak_src, page: int = 256):
 
 
 def bench_backward(w, args, world, local, peaks, peak_src):
-    """Useful TFLOP/s of attn_bwd (dQ, dK, dV from O, LSE and dO) on a prefill workload."""
+    """Useful TFLOP/s of attn_bwd (dQ, dK, dV from O, LSE and dO) on a prefill workload
+    (attn_bwd_alibi when the workload carries ALiBi slopes; its documents and soft-cap too)."""
     import torch
     import io_aware_softmax_b200 as attn
     dev = torch.device("cuda", torch.cuda.current_device())
     q, k, v = workloads.make_inputs(w, device=dev)
     dout = workloads.randn_bf16((w.B, w.Hq, w.Nq, w.d), w.seed, 3, 1.0, dev)
-    o, lse = attn.attn_fwd(q, k, v, scale=w.scale, mask=w.mask_kind, window=w.window)
+    slopes = (torch.tensor(workloads.alibi_slopes(w.Hq), dtype=torch.float32, device=dev)
+              if w.alibi else None)
+    docs = workloads.workload_doc_offsets(w)
+    doc_t = None if docs is None else torch.tensor(docs, dtype=torch.int32, device=dev)
+    o, lse = attn.attn_fwd(q, k, v, scale=w.scale, mask=w.mask_kind, window=w.window,
+                           alibi_slopes=slopes, softcap=w.softcap, doc_offsets=doc_t)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     ws = torch.empty(attn.bwd_workspace_bytes(w.B, w.Hq, w.Nq), dtype=torch.uint8, device=dev)
-    flops = accounting.backward_useful_flops(w.B, w.Hq, w.Nq, w.Nk, w.d, w.mask_kind, w.window)
+    flops = accounting.backward_useful_flops(w.B, w.Hq, w.Nq, w.Nk, w.d, w.mask_kind, w.window,
+                                             docs)
 
     def step():
         attn.attn_bwd(q, k, v, o, lse, dout, scale=w.scale, mask=w.mask_kind, window=w.window,
-                      dq=dq, dk=dk, dv=dv, workspace=ws)
+                      dq=dq, dk=dk, dv=dv, workspace=ws, alibi_slopes=slopes,
+                      softcap=w.softcap, doc_offsets=doc_t)
 
     steps = max(3, min(args.steps, 20))
     for _ in range(args.warmup):
@@ -519,10 +527,13 @@ def bench_backward(w, args, world, local, peaks, peak_src):
            "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak,
                         "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
                         "peak_source": f"bf16_tflops (burst, {peak_src})",
-                        "kernel": "attn_bwd_rowdot + attn_bwd_dq + attn_bwd_dkdv (one call)",
-                        "traffic": recorded_traffic("backward")},
+                        "kernel": "attn_bwd_rowdot + attn_bwd_dq + attn_bwd_dkdv (one call)"
+                                  + (" (ALiBi)" if w.alibi else "")
+                                  + (" (soft-cap)" if w.softcap else ""),
+                        "traffic": (None if (w.alibi or w.softcap or w.docs)
+                                    else recorded_traffic("backward"))},
            "gpu_launches": 3 * steps, "clocks": clk.summary()}
-    del q, k, v, o, lse, dout, dq, dk, dv, ws
+    del q, k, v, o, lse, dout, dq, dk, dv, ws, slopes, doc_t
     torch.cuda.empty_cache()
     return res
 

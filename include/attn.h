@@ -111,12 +111,13 @@ ATTN_API int attn_fwd_alibi(const void* q, const void* k, const void* v, void* o
  *   q, k, v, o, lse   as attn_fwd (o and lse: attn_fwd's outputs for these inputs)
  *   dout         bf16 [B, Hq, Nq, d]   gradient of the loss with respect to o
  *   dq           bf16 [B, Hq, Nq, d]   dk, dv  bf16 [B, Hkv, Nk, d]   (written)
- *   mask_kind, window, doc_offsets, num_docs, scale   as attn_fwd; softcap must be <= 0
+ *   mask_kind, window, doc_offsets, num_docs, scale, softcap   as attn_fwd (with a soft-cap
+ *                the capped score y = c tanh(x / c) passes dy (1 - tanh^2(x / c)) on to x)
  *   workspace    device, 16-byte aligned, attn_bwd_workspace_bytes(B, Hq, Nq) bytes (the
  *                per-row rowsum(dO * O) and base-2 LSE); contents are scratch
  * Three kernel launches on `stream`, no host synchronisation.  Rows with no visible key
  * (LSE = -inf) contribute nothing; keys no query sees get dK = dV = 0.
- * Errors: as attn_fwd, plus UNSUPPORTED for softcap > 0 and WORKSPACE.
+ * Errors: as attn_fwd, plus WORKSPACE.
  */
 ATTN_API size_t attn_bwd_workspace_bytes(int B, int Hq, int Nq);
 ATTN_API int attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
@@ -124,6 +125,22 @@ ATTN_API int attn_bwd(const void* q, const void* k, const void* v, const void* o
              int Nk, int d, float scale, int mask_kind, int window, float softcap,
              const int* doc_offsets, int num_docs, void* workspace, size_t workspace_bytes,
              cudaStream_t stream);
+
+/*
+ * attn_bwd_alibi -- attn_bwd for scores that carry the ALiBi bias of attn_fwd_alibi
+ * ("3.7 어텐션 II", 3.7.5).  The bias depends on positions only, so the gradients keep the
+ * form of attn_bwd with P recomputed from the biased scores:
+ * P_ij = exp(scale q_i.k_j - slope_h |i - j| - LSE_i).
+ *   alibi_slopes  device fp32 [Hq], 4-byte aligned (the slopes given to attn_fwd_alibi;
+ *                 o and lse must come from that call); NULL behaves as attn_bwd.
+ * Every other argument, the workspace and the errors as attn_bwd, plus UNSUPPORTED for
+ * slopes together with softcap > 0 (as attn_fwd_alibi).
+ */
+ATTN_API int attn_bwd_alibi(const void* q, const void* k, const void* v, const void* o,
+             const void* dout, const float* lse, void* dq, void* dk, void* dv, int B, int Hq,
+             int Hkv, int Nq, int Nk, int d, float scale, int mask_kind, int window,
+             float softcap, const int* doc_offsets, int num_docs, const float* alibi_slopes,
+             void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /*
  * attn_quantize_fp8 -- block quantization to E4M3 ("FlashAttention 논문 분석", section

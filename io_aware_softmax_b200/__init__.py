@@ -9,8 +9,8 @@ Every C entry point has a binding of the same name (``attn_decode_splitkv``,
 the same functions.
 """
 from .api import (  # noqa: F401
-    MASKS, AttnError, attn_blockmap, attn_bwd, attn_bwd_workspace_bytes, attn_decode,
-    attn_decode_default_splits, attn_decode_merge, attn_decode_paged, attn_decode_splitkv,
+    MASKS, AttnError, attn_blockmap, attn_bwd, attn_bwd_alibi, attn_bwd_workspace_bytes,
+    attn_decode, attn_decode_default_splits, attn_decode_merge, attn_decode_paged, attn_decode_splitkv,
     attn_decode_splitkv_noalloc, attn_decode_workspace_bytes, attn_fwd, attn_fwd_alibi,
     attn_fwd_fp8, attn_get_device_status, attn_last_error_site, attn_merge, attn_quantize_fp8,
     attn_set_wait_limit_ns, attn_status_string, attn_version, bwd_workspace_bytes, decode_workspace_bytes,
@@ -20,8 +20,8 @@ from ._lib import LIB_PATH, LibraryMissing, load as load_library  # noqa: F401
 
 __all__ = [
     # the C entry points, one binding each
-    "attn_fwd", "attn_fwd_alibi", "attn_bwd", "attn_bwd_workspace_bytes", "attn_quantize_fp8",
-    "attn_fwd_fp8", "attn_blockmap", "attn_decode_workspace_bytes", "attn_decode_default_splits",
+    "attn_fwd", "attn_fwd_alibi", "attn_bwd", "attn_bwd_alibi", "attn_bwd_workspace_bytes",
+    "attn_quantize_fp8", "attn_fwd_fp8", "attn_blockmap", "attn_decode_workspace_bytes", "attn_decode_default_splits",
     "attn_decode_splitkv", "attn_decode_splitkv_noalloc", "attn_decode_paged",
     "attn_decode_merge", "attn_get_device_status", "attn_last_error_site",
     "attn_set_wait_limit_ns", "attn_status_string",

@@ -31,6 +31,10 @@ SIGNATURES = {
     "attn_bwd": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                          c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_int, c_int, c_float,
                          c_int, c_int, c_float, c_void_p, c_int, c_void_p, c_size_t, c_void_p]),
+    "attn_bwd_alibi": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                               c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_int,
+                               c_int, c_float, c_int, c_int, c_float, c_void_p, c_int, c_void_p,
+                               c_void_p, c_size_t, c_void_p]),
     "attn_quantize_fp8": (c_int, [c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_int,
                                   c_int, c_int, c_int, c_void_p, c_void_p]),
     "attn_fwd_fp8": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,

@@ -163,8 +163,12 @@ def attn_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,
              mask="none", window: int = 0, doc_offsets: Optional[torch.Tensor] = None,
              dq: Optional[torch.Tensor] = None, dk: Optional[torch.Tensor] = None,
              dv: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
+             alibi_slopes: Optional[torch.Tensor] = None, softcap: float = 0.0,
              stream=None) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
-    """Backward of attn_fwd: (dq, dk, dv) from q, k, v, attn_fwd's (o, lse) and dout."""
+    """Backward of attn_fwd: (dq, dk, dv) from q, k, v, attn_fwd's (o, lse) and dout.
+
+    ``alibi_slopes`` (fp32 [Hq] on the device, as given to attn_fwd) selects attn_bwd_alibi;
+    ``softcap`` is the soft-cap given to attn_fwd."""
     lib = _lib.load()
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (dout, "dout")):
         _need(t, n, torch.bfloat16, 4)
@@ -190,12 +194,24 @@ def attn_bwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,
         _need(doc_offsets, "doc_offsets", torch.int32, 1)
         _same_device(q, (doc_offsets, "doc_offsets"))
         num_docs = doc_offsets.numel() - 1
+    if alibi_slopes is not None:
+        _need(alibi_slopes, "alibi_slopes", torch.float32, 1)
+        _shape(alibi_slopes, "alibi_slopes", (Hq,))
+        _same_device(q, (alibi_slopes, "alibi_slopes"))
     with _device(q):
-        st = lib.attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq),
-                          _ptr(dk), _ptr(dv), B, Hq, Hkv, Nq, Nk, d, float(scale or 0.0),
-                          _mask_id(mask), int(window), 0.0, _ptr(doc_offsets), num_docs,
-                          _ptr(workspace), ws_bytes, _stream(q.device, stream))
-    _check(st, "attn_bwd")
+        if alibi_slopes is None:
+            st = lib.attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse),
+                              _ptr(dq), _ptr(dk), _ptr(dv), B, Hq, Hkv, Nq, Nk, d,
+                              float(scale or 0.0), _mask_id(mask), int(window), float(softcap or 0.0),
+                              _ptr(doc_offsets), num_docs, _ptr(workspace), ws_bytes,
+                              _stream(q.device, stream))
+        else:
+            st = lib.attn_bwd_alibi(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse),
+                                    _ptr(dq), _ptr(dk), _ptr(dv), B, Hq, Hkv, Nq, Nk, d,
+                                    float(scale or 0.0), _mask_id(mask), int(window), float(softcap or 0.0),
+                                    _ptr(doc_offsets), num_docs, _ptr(alibi_slopes),
+                                    _ptr(workspace), ws_bytes, _stream(q.device, stream))
+    _check(st, "attn_bwd" if alibi_slopes is None else "attn_bwd_alibi")
     return dq, dk, dv
 
 
@@ -425,6 +441,15 @@ def attn_fwd_alibi(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor,
     if alibi_slopes is None:
         raise ValueError("attn_fwd_alibi needs alibi_slopes (fp32 [Hq] on the device)")
     return attn_fwd(q, k, v, alibi_slopes=alibi_slopes, **kwargs)
+
+
+def attn_bwd_alibi(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, o: torch.Tensor,
+                   lse: torch.Tensor, dout: torch.Tensor, alibi_slopes: torch.Tensor,
+                   **kwargs) -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+    """attn_bwd for scores with the ALiBi bias of attn_fwd_alibi."""
+    if alibi_slopes is None:
+        raise ValueError("attn_bwd_alibi needs alibi_slopes (fp32 [Hq] on the device)")
+    return attn_bwd(q, k, v, o, lse, dout, alibi_slopes=alibi_slopes, **kwargs)
 
 
 def attn_decode_splitkv_noalloc(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,

@@ -416,14 +416,26 @@ extern "C" int attn_bwd(const void* q, const void* k, const void* v, const void*
                         int Hq, int Hkv, int Nq, int Nk, int d, float scale, int mask_kind,
                         int window, float softcap, const int* doc_offsets, int num_docs,
                         void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  return attn_bwd_alibi(q, k, v, o, dout, lse, dq, dk, dv, B, Hq, Hkv, Nq, Nk, d, scale,
+                        mask_kind, window, softcap, doc_offsets, num_docs, nullptr, workspace,
+                        workspace_bytes, stream);
+}
+
+extern "C" int attn_bwd_alibi(const void* q, const void* k, const void* v, const void* o,
+                              const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                              int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale,
+                              int mask_kind, int window, float softcap, const int* doc_offsets,
+                              int num_docs, const float* alibi_slopes, void* workspace,
+                              size_t workspace_bytes, cudaStream_t stream) {
   if (B < 0 || Hq < 0 || Hkv < 0 || Nq < 0 || Nk < 0) return ATTN_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(alibi_slopes) & 3u) return ATTN_ERR_MISALIGNED;
   if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
   if (Hkv == 0 && Hq > 0) return ATTN_ERR_INVALID_ARG;
   if (Hkv > 0 && Hq % Hkv != 0) return ATTN_ERR_UNSUPPORTED;
   int st = check_mask(mask_kind, window, doc_offsets, num_docs, Nq, Nk);
   if (st != ATTN_OK) return st;
   if (std::isnan(scale) || std::isnan(softcap)) return ATTN_ERR_INVALID_ARG;
-  if (softcap > 0.f) return ATTN_ERR_UNSUPPORTED;
+  if (softcap > 0.f && alibi_slopes != nullptr) return ATTN_ERR_UNSUPPORTED;
   if (B == 0 || Hq == 0 || (Nq == 0 && Nk == 0)) return ATTN_OK;
   const void* ptrs[] = {q, k, v, o, dout, lse, dq, dk, dv};
   const int needed[] = {Nq > 0, Nk > 0, Nk > 0, Nq > 0, Nq > 0, Nq > 0, Nq > 0, Nk > 0, Nk > 0};
@@ -457,6 +469,9 @@ extern "C" int attn_bwd(const void* q, const void* k, const void* v, const void*
   p.kscale = scale * kLog2e;
   p.scale = scale;
   p.mask = mask_params(mask_kind, window, doc_offsets, num_docs, Nq, Nk);
+  p.alibi = alibi_slopes;
+  p.cap_scale = softcap > 0.f ? scale / softcap : 0.f;
+  p.cap_log2 = softcap > 0.f ? softcap * kLog2e : 0.f;
   p.err = error_word_ptr(dev);
   if (p.err == nullptr) return ATTN_ERR_CUDA;
   if (Nq > 0 && launch_bwd_rowdot(o, dout, lse, const_cast<float*>(p.dvec),

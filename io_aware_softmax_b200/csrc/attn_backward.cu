@@ -102,16 +102,25 @@ __device__ __forceinline__ float bf(uint32_t u) { return __uint_as_float(u); }
 //   grads: ds = p (dp - Dv) and bf16 pairs of ds (and of p, optionally) for the 32 columns
 //          [OFF, OFF + 32).
 // l2(j) and dv(j) give the four columns' values, vis(j) a 4-bit mask of visible pairs.
-template <int N, typename L2, typename Vis>
-__device__ __forceinline__ void probs(uint32_t (&s)[N], float ks, L2 l2, Vis vis) {
+// kCap: the score is soft-capped, x = cap_log2 tanh(s cap_scale) - l2 (base 2).
+template <int N, bool kCap = false, typename L2, typename Vis>
+__device__ __forceinline__ void probs(uint32_t (&s)[N], float ks, L2 l2, Vis vis,
+                                      float cap_scale = 0.f, float cap_log2 = 0.f) {
 #pragma unroll
   for (int j = 0; j < N / 4; ++j) {
     const float4 l = l2(j);
     const unsigned m = vis(j);
     const int c = 4 * j;
     float x0, x1, x2, x3;
-    ffma2(x0, x1, bf(s[c]), bf(s[c + 1]), ks, ks, -l.x, -l.y);
-    ffma2(x2, x3, bf(s[c + 2]), bf(s[c + 3]), ks, ks, -l.z, -l.w);
+    if constexpr (kCap) {
+      x0 = fmaf(cap_log2, tanh_via_ex2(bf(s[c]) * cap_scale), -l.x);
+      x1 = fmaf(cap_log2, tanh_via_ex2(bf(s[c + 1]) * cap_scale), -l.y);
+      x2 = fmaf(cap_log2, tanh_via_ex2(bf(s[c + 2]) * cap_scale), -l.z);
+      x3 = fmaf(cap_log2, tanh_via_ex2(bf(s[c + 3]) * cap_scale), -l.w);
+    } else {
+      ffma2(x0, x1, bf(s[c]), bf(s[c + 1]), ks, ks, -l.x, -l.y);
+      ffma2(x2, x3, bf(s[c + 2]), bf(s[c + 3]), ks, ks, -l.z, -l.w);
+    }
     s[c] = __float_as_uint((m & 1u) ? ex2_approx(x0) : 0.f);
     s[c + 1] = __float_as_uint((m & 2u) ? ex2_approx(x1) : 0.f);
     s[c + 2] = __float_as_uint((m & 4u) ? ex2_approx(x2) : 0.f);
@@ -119,9 +128,19 @@ __device__ __forceinline__ void probs(uint32_t (&s)[N], float ks, L2 l2, Vis vis
   }
 }
 
-template <bool kWantP, int OFF, int N, int ND, typename DV>
+// With a soft-cap (kCap) the capped score y = c tanh(x / c) passes dy (1 - tanh^2) on to the
+// scaled product x; tanh is recovered from p itself, t = (log2 p + l2) / cap_log2, so no
+// register holds it between the two steps (p = 0 leaves ds = 0 whatever the factor).
+__device__ __forceinline__ float cap_factor(float p, float l, float inv_cap_log2) {
+  const float t = (p > 0.f) ? (__log2f(p) + l) * inv_cap_log2 : 0.f;
+  return fmaf(-t, t, 1.f);
+}
+
+template <bool kWantP, int OFF, int N, int ND, bool kCap = false, typename DV,
+          typename L2 = float4 (*)(int)>
 __device__ __forceinline__ void grads(const uint32_t (&pr)[N], const uint32_t (&dp)[ND], DV dv,
-                                      uint32_t (&pk)[16], uint32_t (&dsk)[16]) {
+                                      uint32_t (&pk)[16], uint32_t (&dsk)[16], L2 l2 = nullptr,
+                                      float inv_cap_log2 = 0.f) {
   static_assert(ND == 32 || ND == N, "dp holds these 32 columns or all N");
   constexpr int DOFF = (ND == 32) ? 0 : OFF;
 #pragma unroll
@@ -129,10 +148,17 @@ __device__ __forceinline__ void grads(const uint32_t (&pr)[N], const uint32_t (&
     const float4 d = dv(j);
     const int c = OFF + 4 * j, e = DOFF + 4 * j;
     const float p0 = bf(pr[c]), p1 = bf(pr[c + 1]), p2 = bf(pr[c + 2]), p3 = bf(pr[c + 3]);
-    const float d0 = p0 * (bf(dp[e]) - d.x);
-    const float d1 = p1 * (bf(dp[e + 1]) - d.y);
-    const float d2 = p2 * (bf(dp[e + 2]) - d.z);
-    const float d3 = p3 * (bf(dp[e + 3]) - d.w);
+    float d0 = p0 * (bf(dp[e]) - d.x);
+    float d1 = p1 * (bf(dp[e + 1]) - d.y);
+    float d2 = p2 * (bf(dp[e + 2]) - d.z);
+    float d3 = p3 * (bf(dp[e + 3]) - d.w);
+    if constexpr (kCap) {
+      const float4 l = l2(j);
+      d0 *= cap_factor(p0, l.x, inv_cap_log2);
+      d1 *= cap_factor(p1, l.y, inv_cap_log2);
+      d2 *= cap_factor(p2, l.z, inv_cap_log2);
+      d3 *= cap_factor(p3, l.w, inv_cap_log2);
+    }
     if (kWantP) {
       pk[2 * j] = pack_bf16x2(p0, p1);
       pk[2 * j + 1] = pack_bf16x2(p2, p3);
@@ -276,8 +302,9 @@ __device__ __forceinline__ void issue_ts(uint32_t acc, uint32_t a_tmem, uint32_t
                  idesc, (!first || kk > 0) ? 1u : 0u);
 }
 
-// dQ of one 128-row query tile of head (b, h).
-template <int D>
+// dQ of one 128-row query tile of head (b, h).  kAlibi: the scores carry the ALiBi bias
+// -slope_h |q - kv|, which moves each P element's base-2 offset from l2 to l2 + slope2 |q - kv|.
+template <int D, bool kAlibi, bool kCap>
 __global__ void __launch_bounds__(kBwdThreads, 1)
 attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmDO,
                    const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
@@ -447,6 +474,8 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     const float dr = valid ? p.dvec[ridx] : 0.f;
     const float4 l2r4 = make_float4(l2r, l2r, l2r, l2r);
     const float4 dr4 = make_float4(dr, dr, dr, dr);
+    const float slope2 = kAlibi ? __ldg(p.alibi + h) * kLog2eB : 0.f;
+    const float inv_cap = kCap ? 1.f / p.cap_log2 : 0.f;
     int rlo = 1, rhi = 0;
     if (valid) row_interval(p.mask, row, rlo, rhi);
     const uint32_t tl = tmem + ((uint32_t)(wq * 32) << 16);
@@ -474,7 +503,18 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(BAR_XF));
-      probs<64>(s, p.kscale, [&](int) { return l2r4; }, [&](int j) { return vis(4 * j); });
+      if constexpr (kAlibi) {
+        // key kc + c is |row - kc - c| away from this row
+        const float drow = (float)(row - kc);
+        probs<64>(s, p.kscale, [&](int j) {
+          const float c = (float)(4 * j);
+          return make_float4(fmaf(slope2, fabsf(drow - c), l2r), fmaf(slope2, fabsf(drow - c - 1.f), l2r),
+                             fmaf(slope2, fabsf(drow - c - 2.f), l2r), fmaf(slope2, fabsf(drow - c - 3.f), l2r));
+        }, [&](int j) { return vis(4 * j); });
+      } else {
+        probs<64, kCap>(s, p.kscale, [&](int) { return l2r4; }, [&](int j) { return vis(4 * j); },
+                        p.cap_scale, p.cap_log2);
+      }
       ok = __all_sync(0xffffffffu, mbar_wait(bar(BAR_DP), t & 1, abort_flag, p.err, kSiteBwdS));
       if (!ok) break;
       tc_fence_after();
@@ -483,12 +523,14 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       tmem_ld_wait_x64(dp);
       {
         uint32_t pk[16], dsk[16];
-        grads<false, 0, 64, 64>(s, dp, [&](int) { return dr4; }, pk, dsk);
+        grads<false, 0, 64, 64, kCap>(s, dp, [&](int) { return dr4; }, pk, dsk,
+                                      [&](int) { return l2r4; }, inv_cap);
         tmem_st_x16(tl + kTmemY + col, dsk);
       }
       {
         uint32_t pk[16], dsk[16];
-        grads<false, 32, 64, 64>(s, dp, [&](int) { return dr4; }, pk, dsk);
+        grads<false, 32, 64, 64, kCap>(s, dp, [&](int) { return dr4; }, pk, dsk,
+                                       [&](int) { return l2r4; }, inv_cap);
         tmem_st_x16(tl + kTmemY + col + 16u, dsk);
       }
       tmem_wait_st();
@@ -518,8 +560,9 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   }
 }
 
-// dK and dV of one 128-key tile of KV head (b, hk), summed over the query heads of its group.
-template <int D>
+// dK and dV of one 128-key tile of KV head (b, hk), summed over the query heads of its group
+// (kAlibi as for attn_bwd_dq_kernel, with the slope of each streamed tile's query head).
+template <int D, bool kAlibi, bool kCap>
 __global__ void __launch_bounds__(kBwdThreads, 1)
 attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ,
                      const __grid_constant__ CUtensorMap tmDO,
@@ -709,6 +752,7 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ,
     const uint32_t tl = tmem + ((uint32_t)(wq * 32) << 16);
     const uint32_t col = 64u * (uint32_t)g;
     const long long kidx = ((long long)b * p.Hkv + hk) * p.Nk + key;
+    const float inv_cap = kCap ? 1.f / p.cap_log2 : 0.f;
     bool ok = true;
     for (int t = 0; t < n; ++t) {
       // this tile's query vectors, written ahead by warps 10-11
@@ -742,7 +786,20 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ,
         }
         return m;
       };
-      auto l2f = [&](int c) { return *reinterpret_cast<const float4*>(l2v + c); };
+      // ALiBi: query q0 + col + c is |key - q0 - col - c| away from this key
+      const float slope2 = kAlibi ? __ldg(p.alibi + hk * p.G + t / ni) * kLog2eB : 0.f;
+      const float dkey = (float)(key - q0 - (int)col);
+      auto l2f = [&](int c) {
+        float4 l = *reinterpret_cast<const float4*>(l2v + c);
+        if constexpr (kAlibi) {
+          const float fc = (float)c;
+          l.x = fmaf(slope2, fabsf(dkey - fc), l.x);
+          l.y = fmaf(slope2, fabsf(dkey - fc - 1.f), l.y);
+          l.z = fmaf(slope2, fabsf(dkey - fc - 2.f), l.z);
+          l.w = fmaf(slope2, fabsf(dkey - fc - 3.f), l.w);
+        }
+        return l;
+      };
       auto dvf = [&](int c) { return *reinterpret_cast<const float4*>(dv + c); };
       // Step 1 (S^T ready): P^T of the group's 64 columns, in two halves of 32; the bf16
       // P^T of a half lands in columns the group has already read.
@@ -751,13 +808,14 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ,
         uint32_t pk[16];
         tmem_ld_x32_async(tl + kTmemX + col, pr0);
         tmem_ld_wait_x32(pr0);
-        probs<32>(pr0, p.kscale, [&](int j) { return l2f(4 * j); }, [&](int j) { return vis(4 * j); });
+        probs<32, kCap>(pr0, p.kscale, [&](int j) { return l2f(4 * j); },
+                        [&](int j) { return vis(4 * j); }, p.cap_scale, p.cap_log2);
         pack_pairs(pr0, pk);
         tmem_st_x16(tl + kTmemX + col, pk);
         tmem_ld_x32_async(tl + kTmemX + col + 32u, pr1);
         tmem_ld_wait_x32(pr1);
-        probs<32>(pr1, p.kscale, [&](int j) { return l2f(32 + 4 * j); },
-                  [&](int j) { return vis(32 + 4 * j); });
+        probs<32, kCap>(pr1, p.kscale, [&](int j) { return l2f(32 + 4 * j); },
+                        [&](int j) { return vis(32 + 4 * j); }, p.cap_scale, p.cap_log2);
         pack_pairs(pr1, pk);
         tmem_st_x16(tl + kTmemX + col + 16u, pk);
       }
@@ -773,11 +831,13 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ,
         uint32_t dph[32], pk[16], dsk[16];
         tmem_ld_x32_async(tl + kTmemY + col, dph);
         tmem_ld_wait_x32(dph);
-        grads<false, 0, 32, 32>(pr0, dph, [&](int j) { return dvf(4 * j); }, pk, dsk);
+        grads<false, 0, 32, 32, kCap>(pr0, dph, [&](int j) { return dvf(4 * j); }, pk, dsk,
+                                      [&](int j) { return l2f(4 * j); }, inv_cap);
         tmem_st_x16(tl + kTmemY + col, dsk);
         tmem_ld_x32_async(tl + kTmemY + col + 32u, dph);
         tmem_ld_wait_x32(dph);
-        grads<false, 0, 32, 32>(pr1, dph, [&](int j) { return dvf(32 + 4 * j); }, pk, dsk);
+        grads<false, 0, 32, 32, kCap>(pr1, dph, [&](int j) { return dvf(32 + 4 * j); }, pk, dsk,
+                                      [&](int j) { return l2f(32 + 4 * j); }, inv_cap);
         tmem_st_x16(tl + kTmemY + col + 16u, dsk);
       }
       tmem_wait_st();
@@ -813,25 +873,25 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ,
   }
 }
 
-template <int D>
+template <int D, bool kAlibi, bool kCap>
 int launch_bwd_t(const CUtensorMap& tq, const CUtensorMap& tdo, const CUtensorMap& tk,
                  const CUtensorMap& tv, const BwdParams& p, cudaStream_t stream) {
   using C = BwdCfg<D>;
   using CQ = DqCfg<D>;
   static_assert(C::kSmemBytes <= 227 * 1024 && CQ::kSmemBytes <= 227 * 1024,
                 "shared memory budget");
-  if (cudaFuncSetAttribute(attn_bwd_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  if (cudaFuncSetAttribute(attn_bwd_dq_kernel<D, kAlibi, kCap>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            CQ::kSmemBytes) != cudaSuccess ||
-      cudaFuncSetAttribute(attn_bwd_dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+      cudaFuncSetAttribute(attn_bwd_dkdv_kernel<D, kAlibi, kCap>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            C::kSmemBytes) != cudaSuccess)
     return -4;
   const long long nq = (long long)p.B * p.Hq * ((p.Nq + kBT - 1) / kBT);
   const long long nk = (long long)p.B * p.Hkv * ((p.Nk + kBT - 1) / kBT);
   if (nk > 0)
-    attn_bwd_dkdv_kernel<D><<<(unsigned)nk, kBwdThreads, C::kSmemBytes, stream>>>(tq, tdo, tk,
+    attn_bwd_dkdv_kernel<D, kAlibi, kCap><<<(unsigned)nk, kBwdThreads, C::kSmemBytes, stream>>>(tq, tdo, tk,
                                                                                  tv, p);
   if (nq > 0)
-    attn_bwd_dq_kernel<D><<<(unsigned)nq, kBwdThreads, CQ::kSmemBytes, stream>>>(tq, tdo, tk,
+    attn_bwd_dq_kernel<D, kAlibi, kCap><<<(unsigned)nq, kBwdThreads, CQ::kSmemBytes, stream>>>(tq, tdo, tk,
                                                                                 tv, p);
   return cudaGetLastError() == cudaSuccess ? 0 : -4;
 }
@@ -851,8 +911,15 @@ int launch_bwd_rowdot(const void* o, const void* dout, const float* lse, float* 
 
 int launch_attn_bwd(const CUtensorMap& tq, const CUtensorMap& tdo, const CUtensorMap& tk,
                     const CUtensorMap& tv, const BwdParams& p, int d, cudaStream_t stream) {
-  if (d == 128) return launch_bwd_t<128>(tq, tdo, tk, tv, p, stream);
-  if (d == 64) return launch_bwd_t<64>(tq, tdo, tk, tv, p, stream);
+  // ALiBi and the soft-cap are not combined (the host refuses that request)
+  const bool alibi = p.alibi != nullptr, cap = p.cap_scale > 0.f;
+  if (alibi && cap) return -2;
+  if (d == 128) return alibi ? launch_bwd_t<128, true, false>(tq, tdo, tk, tv, p, stream)
+                       : cap ? launch_bwd_t<128, false, true>(tq, tdo, tk, tv, p, stream)
+                             : launch_bwd_t<128, false, false>(tq, tdo, tk, tv, p, stream);
+  if (d == 64) return alibi ? launch_bwd_t<64, true, false>(tq, tdo, tk, tv, p, stream)
+                      : cap ? launch_bwd_t<64, false, true>(tq, tdo, tk, tv, p, stream)
+                            : launch_bwd_t<64, false, false>(tq, tdo, tk, tv, p, stream);
   return -2;
 }
 

@@ -57,6 +57,9 @@ struct BwdParams {
   float kscale;       // scale * log2(e)
   float scale;
   MaskParams mask;
+  const float* alibi;  // fp32 [Hq] ALiBi slopes (natural-log units), or nullptr
+  float cap_scale;    // soft-cap c > 0: scale / c (0: no cap)
+  float cap_log2;     // c * log2(e)
   uint32_t* err;      // device error word of the library (bits, first site)
 };
 

@@ -186,13 +186,24 @@ def test_backward_validation(lib):
                          kw.get("d", 128), 0.0, kw.get("mask", 1), 0, kw.get("cap", 0.0), None, 0,
                          kw.get("ws", P), kw.get("wsb", 1 << 20), None]
     assert f(*args(d=96)) == -2
-    assert f(*args(cap=30.0)) == -2
+    assert f(*args(cap=float("nan"))) == -1
     assert f(*args(mask=9)) == -1
     assert f(*args(q=ctypes.c_void_p(24))) == -3
     assert f(*args(ws=None, wsb=0)) == -6
     assert f(*args(wsb=10)) == -6
     assert lib.attn_bwd_workspace_bytes(2, 4, 100) == 2 * ((2 * 4 * 100 * 4 + 255) // 256 * 256)
     assert lib.attn_bwd_workspace_bytes(0, 4, 100) == 0
+
+
+def test_backward_alibi_validation(lib):
+    # the same checks as attn_bwd, plus 4-byte alignment of the slopes; no launch happens
+    f = lib.attn_bwd_alibi
+    P = ctypes.c_void_p(16)
+    args = lambda **kw: [P, P, P, P, P, P, P, P, P, 1, 2, 2, 64, 64, kw.get("d", 128), 0.0, 1, 0,
+                         kw.get("cap", 0.0), None, 0, kw.get("slopes", P), P, 1 << 20, None]
+    assert f(*args(slopes=ctypes.c_void_p(18))) == -3
+    assert f(*args(d=96)) == -2
+    assert f(*args(cap=30.0)) == -2
 
 
 def test_fp8_entry_validation(lib):

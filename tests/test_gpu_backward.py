@@ -39,20 +39,25 @@ def compare_grad(got, ref, what):
     assert rmax <= TOL_MAX and rmean <= TOL_MEAN, f"{what}: max {rmax:.3e}, mean {rmean:.3e}"
 
 
-def _run(B, Hq, Hkv, Nq, Nk, d, mask="none", window=0, docs=None, seed=0, scale=None):
-    q = workloads.randn_bf16((B, Hq, Nq, d), seed, 0).cuda()
-    k = workloads.randn_bf16((B, Hkv, Nk, d), seed, 1).cuda()
+def _run(B, Hq, Hkv, Nq, Nk, d, mask="none", window=0, docs=None, seed=0, scale=None,
+         slopes=None, softcap=0.0, std=1.0):
+    q = workloads.randn_bf16((B, Hq, Nq, d), seed, 0, std).cuda()
+    k = workloads.randn_bf16((B, Hkv, Nk, d), seed, 1, std).cuda()
     v = workloads.randn_bf16((B, Hkv, Nk, d), seed, 2).cuda()
     dout = workloads.randn_bf16((B, Hq, Nq, d), seed, 3).cuda()
     doc_t = None if docs is None else torch.tensor(docs, dtype=torch.int32, device="cuda")
-    o, lse = attn_fwd(q, k, v, scale=scale, mask=mask, window=window, doc_offsets=doc_t)
+    slopes_t = None if slopes is None else torch.tensor(slopes, dtype=torch.float32, device="cuda")
+    o, lse = attn_fwd(q, k, v, scale=scale, mask=mask, window=window, doc_offsets=doc_t,
+                      alibi_slopes=slopes_t, softcap=softcap)
     dq, dk, dv = attn_bwd(q, k, v, o, lse, dout, scale=scale, mask=mask, window=window,
-                          doc_offsets=doc_t)
+                          doc_offsets=doc_t, alibi_slopes=slopes_t, softcap=softcap)
     assert device_status() == 0
     rq, rk, rv = oracle.attention_backward(f64(q), f64(k), f64(v), f64(dout), scale=scale,
                                            mask_kind=MASK_ID[mask], window=window,
-                                           doc_offsets=docs)
-    tag = f"{B}x{Hq}/{Hkv}x{Nq}x{Nk}x{d} {mask} w{window}"
+                                           doc_offsets=docs, alibi_slopes=slopes,
+                                           softcap=softcap)
+    tag = (f"{B}x{Hq}/{Hkv}x{Nq}x{Nk}x{d} {mask} w{window}"
+           + ("" if slopes is None else " alibi") + (f" cap{softcap}" if softcap else ""))
     compare_grad(dq, rq, "dQ " + tag)
     compare_grad(dk, rk, "dK " + tag)
     compare_grad(dv, rv, "dV " + tag)
@@ -86,16 +91,43 @@ def test_non_square_unmasked(Nq, Nk):
     _run(1, 2, 1, Nq, Nk, 128, seed=Nq + Nk, scale=0.2)
 
 
-def test_softcap_is_unsupported():
+def _geometric_slopes(H):
+    return [2.0 ** (-8.0 * (h + 1) / H) for h in range(H)]
+
+
+@pytest.mark.parametrize("mask,N,d", [("causal", 300, 128), ("none", 257, 64),
+                                      ("sliding", 700, 128)])
+def test_alibi(mask, N, d):
+    # GQA (4 query heads on 2 KV heads): the dK/dV kernel takes each streamed tile's slope
+    _run(1, 4, 2, N, N, d, mask=mask, window=130, seed=N + d, slopes=_geometric_slopes(4))
+
+
+def test_alibi_steep_slopes_and_ragged_tail():
+    # slopes up to 2: the bias dominates the scores and P concentrates near the diagonal
+    _run(2, 2, 1, 129, 129, 128, mask="causal", seed=21, slopes=[2.0, 0.03])
+
+
+@pytest.mark.parametrize("mask,N,d,cap,std", [("causal", 300, 128, 1.5, 1.0),
+                                               ("none", 129, 64, 3.0, 2.0),
+                                               ("sliding", 700, 128, 1.0, 1.0)])
+def test_softcap(mask, N, d, cap, std):
+    # small caps saturate many scores, so the (1 - tanh^2) factor matters
+    _run(1, 4, 2, N, N, d, mask=mask, window=130, seed=N + d, softcap=cap, std=std)
+
+
+def test_document_softcap_as_the_packed_workload():
+    # the packed-document workload's hooks (cap 50, inputs N(0,1) * 2) on short documents
+    _run(1, 3, 3, 800, 800, 128, mask="document_causal", docs=[0, 1, 127, 300, 301, 700, 800],
+         seed=9, softcap=50.0, std=2.0)
+
+
+def test_alibi_with_softcap_is_unsupported():
     q = workloads.randn_bf16((1, 2, 64, 128), 1, 0).cuda()
+    slopes = torch.tensor([0.5, 0.25], dtype=torch.float32, device="cuda")
     lse = torch.zeros((1, 2, 64), dtype=torch.float32, device="cuda")
-    from io_aware_softmax_b200 import _lib
-    lib = _lib.load()
-    ws = torch.empty(1 << 16, dtype=torch.uint8, device="cuda")
-    p = q.data_ptr()
-    st = lib.attn_bwd(p, p, p, p, p, lse.data_ptr(), p, p, p, 1, 2, 2, 64, 64, 128, 0.0, 1, 0,
-                      30.0, None, 0, ws.data_ptr(), ws.numel(), None)
-    assert st == -2
+    with pytest.raises(Exception) as e:
+        attn_bwd(q, q, q, q, lse, q, alibi_slopes=slopes, softcap=30.0)
+    assert "unsupported" in str(e.value).lower()
 
 
 def test_causal_mha_full_size_one_head():
