@@ -27,7 +27,7 @@ TOL_MAX = 1.5e-2
 TOL_MEAN = 4e-3
 
 
-def compare_grad(got, ref, what):
+def compare_grad(got, ref, what, tol_mean=TOL_MEAN):
     g = f64(got)
     assert g.shape == ref.shape, (what, g.shape, ref.shape)
     assert np.all(np.isfinite(g)), f"{what}: non-finite"
@@ -36,11 +36,11 @@ def compare_grad(got, ref, what):
     avg = max(float(np.abs(ref).mean()), 1e-4)
     rmax, rmean = float(err.max()) / big, float(err.mean()) / avg
     print(f"{what}: max {rmax:.2e} of max|ref|, mean {rmean:.2e} of mean|ref|")
-    assert rmax <= TOL_MAX and rmean <= TOL_MEAN, f"{what}: max {rmax:.3e}, mean {rmean:.3e}"
+    assert rmax <= TOL_MAX and rmean <= tol_mean, f"{what}: max {rmax:.3e}, mean {rmean:.3e}"
 
 
 def _run(B, Hq, Hkv, Nq, Nk, d, mask="none", window=0, docs=None, seed=0, scale=None,
-         slopes=None, softcap=0.0, std=1.0):
+         slopes=None, softcap=0.0, std=1.0, tol_mean=TOL_MEAN):
     q = workloads.randn_bf16((B, Hq, Nq, d), seed, 0, std).cuda()
     k = workloads.randn_bf16((B, Hkv, Nk, d), seed, 1, std).cuda()
     v = workloads.randn_bf16((B, Hkv, Nk, d), seed, 2).cuda()
@@ -58,9 +58,9 @@ def _run(B, Hq, Hkv, Nq, Nk, d, mask="none", window=0, docs=None, seed=0, scale=
                                            softcap=softcap)
     tag = (f"{B}x{Hq}/{Hkv}x{Nq}x{Nk}x{d} {mask} w{window}"
            + ("" if slopes is None else " alibi") + (f" cap{softcap}" if softcap else ""))
-    compare_grad(dq, rq, "dQ " + tag)
-    compare_grad(dk, rk, "dK " + tag)
-    compare_grad(dv, rv, "dV " + tag)
+    compare_grad(dq, rq, "dQ " + tag, tol_mean)
+    compare_grad(dk, rk, "dK " + tag, tol_mean)
+    compare_grad(dv, rv, "dV " + tag, tol_mean)
 
 
 @pytest.mark.parametrize("d", [64, 128])
@@ -103,8 +103,13 @@ def test_alibi(mask, N, d):
 
 
 def test_alibi_steep_slopes_and_ragged_tail():
-    # slopes up to 2: the bias dominates the scores and P concentrates near the diagonal
-    _run(2, 2, 1, 129, 129, 128, mask="causal", seed=21, slopes=[2.0, 0.03])
+    # Slope 2: the bias dominates the scores and the diagonal key carries P_max ~ 0.86 of
+    # every row (weights 1, e^-2, e^-4, ...).  dS = P (dP - D) then cancels: D = rowsum(dO O)
+    # is taken from the forward's stored bf16 O (2^-9 relative per element), and dP - D is
+    # only about (1 - P_max) of dP, so D's rounding reaches dS amplified by 1 / (1 - P_max)
+    # ~ 7 on that head.  Averaged with the diffuse second head (slope 0.03) the mean error
+    # bound becomes 2^-7 of the mean gradient; the maximum keeps its bound.
+    _run(2, 2, 1, 129, 129, 128, mask="causal", seed=21, slopes=[2.0, 0.03], tol_mean=2.0 ** -7)
 
 
 @pytest.mark.parametrize("mask,N,d,cap,std", [("causal", 300, 128, 1.5, 1.0),
