@@ -280,6 +280,10 @@ def run_ours(args, world, rank, local):
         return bench_decode(args, world, local, peaks, peak_src)
     if args.only == "extras":
         return {"extras": bench_extras(args, world, local, peaks, peak_src)}
+    if args.workload:
+        # one prefill workload alone (profiler captures of a single kernel)
+        return bench_prefill_variant(workloads.BY_NAME[args.workload], args, world, local,
+                                     peaks, peak_src, steps=args.steps)
     w = workloads.CAUSAL_MHA
     dev = torch.device("cuda", torch.cuda.current_device())
     q, k, v = workloads.make_inputs(w, device=dev)
@@ -303,8 +307,7 @@ def run_ours(args, world, rank, local):
     ms_step = max_over_ranks(world, total_ms / args.steps)
     kernel_ms = max_over_ranks(world, sum(per) / len(per))
     value = whole_job_rate(flops, world, ms_step) / 1e12
-    achieved = flops / (kernel_ms * 1e-3) / 1e12
-    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    clocks = clk.summary()
     out = {
         "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
@@ -317,22 +320,23 @@ def run_ours(args, world, rank, local):
                          (3 * q.numel() * 2 / 1e6),
                    "parallelism": f"replicas x{world} (independent (batch, head) units)",
                    "seed": w.seed},
-        "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak,
-                     "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
-                     "peak_source": f"bf16_tflops (burst, {peak_src})",
-                     "frac_of_spec": round(achieved / SPEC_PEAKS["bf16_tflops"], 4),
-                     "executed_tflops": round(executed / (kernel_ms * 1e-3) / 1e12, 2),
-                     "kernel": "attn_fwd_sm100_kernel<128>",
-                     "traffic": recorded_traffic("prefill_causal_mha")},
+        "roofline": prefill_roofline(flops, executed, kernel_ms, peaks, peak_src, clocks,
+                                     "attn_fwd_sm100_kernel<128>",
+                                     recorded_traffic("prefill_causal_mha"),
+                                     torch.cuda.get_device_properties(dev).multi_processor_count),
         "gpu_launches": args.steps,
     }
-    out["clocks"] = clk.summary()
+    out["clocks"] = clocks
 
     if not args.no_e2e:
         out["e2e"] = e2e_prefill(w, args, world, q, k, v)
+    del q, k, v, o, lse
+    torch.cuda.empty_cache()
+    if args.only == "all":
+        # the other two prefill workloads: sliding-window GQA and packed documents + soft-cap
+        out["configs"] = {x.name: bench_prefill_variant(x, args, world, local, peaks, peak_src)
+                          for x in (workloads.SWA_GQA, workloads.DOC_SOFTCAP)}
     if not args.no_decode and args.only == "all":
-        del q, k, v, o, lse
-        torch.cuda.empty_cache()
         out["decode"] = bench_decode(args, world, local, peaks, peak_src)
     if not args.no_extras and args.only == "all":
         out["extras"] = bench_extras(args, world, local, peaks, peak_src)
@@ -342,7 +346,94 @@ def run_ours(args, world, rank, local):
                                "cores": blas_threads(), "kind": "oracle",
                                "sample": f"{heads} whole heads (4096 query rows each, all keys) "
                                          f"of {w.name}, fp64, {dt:.1f} s"}
+        if args.only == "all":
+            out["cpu_baseline"]["per_workload"] = cpu_baselines_other(args.cpu_budget / 3)
+    out["summary"] = summary_of(out)
     return out
+
+
+def summary_of(out: dict) -> dict:
+    """One short entry per line, [value, unit, ms per step, roofline fraction]: the whole
+    line is long, so this compact copy goes last, where a reader of the output's tail sees
+    every workload's figure."""
+    def entry(x):
+        r = x.get("roofline", {})
+        return [x.get("value"), x.get("unit"), x.get("ms_per_step"), r.get("frac")]
+    sm = {out["config"]["workload"]: entry(out)}
+    for group in ("configs", "extras"):
+        for name, x in out.get(group, {}).items():
+            sm[name] = entry(x)
+    if "decode" in out:
+        sm[out["decode"]["workload"]] = entry(out["decode"])
+    if "e2e" in out:
+        sm["e2e"] = [out["e2e"]["value"], out["e2e"]["unit"], out["e2e"].get("ms_per_step"),
+                     None]
+    return sm
+
+
+def cpu_baselines_other(budget_s: float) -> dict:
+    """The oracle on bounded samples of the other three workloads, extrapolated to the whole
+    workload: whole query-row blocks of a few heads (sliding GQA, documents) or whole
+    sequences (decode), timed, scaled by the rows (sequences) the workload has."""
+    res = {}
+    for w in (workloads.SWA_GQA, workloads.DOC_SOFTCAP):
+        per_row_s, rows, dt = oracle_rows_sample(w, budget_s)
+        docs = workloads.workload_doc_offsets(w)
+        flops = accounting.prefill_useful_flops(w.B, w.Hq, w.Nq, w.Nk, w.d, w.mask_kind,
+                                                w.window, docs)
+        total_s = per_row_s * w.B * w.Hq * w.Nq
+        res[w.name] = {"value": round(flops / total_s / 1e12, 6), "unit": "TFLOP/s",
+                       "sample": f"{rows} query rows in 256-row blocks over several heads, "
+                                 f"{dt:.1f} s; extrapolated to all {w.B * w.Hq * w.Nq} rows"}
+    w = workloads.DECODE
+    seqs, dt = oracle_decode_sample(w, budget_s)
+    kv = accounting.decode_kv_bytes(w.B, w.Hkv, w.Nk, w.d)
+    per_seq = dt / seqs
+    res[w.name] = {"value": round(kv / (per_seq * w.B) / 1e9, 4), "unit": "GB/s (KV cache)",
+                   "sample": f"{seqs} whole sequences (all 32 heads, 32768 cached rows), "
+                             f"{dt:.1f} s; extrapolated to all {w.B}"}
+    return res
+
+
+def oracle_rows_sample(w: workloads.Workload, budget_s: float):
+    """Seconds per query row of the fp64 oracle on a prefill workload: 256-row blocks taken
+    at seeded places over the heads of batch entry 0 until ``budget_s`` is spent."""
+    import oracle
+    q, k, v = (x.float().numpy() for x in _cpu_head_inputs(w, 0))
+    docs = workloads.workload_doc_offsets(w)
+    G = w.Hq // w.Hkv
+    rng = np.random.default_rng(w.seed)
+    rows, t0 = 0, time.perf_counter()
+    while True:
+        h = int(rng.integers(w.Hq))
+        r0 = int(rng.integers(0, w.Nq // 256)) * 256
+        rr = np.arange(r0, min(r0 + 256, w.Nq))
+        oracle.attention_head(q[h, rr], rr, k[h // G], v[h // G], w.scale, w.mask_kind,
+                              w.window, w.softcap, docs)
+        rows += len(rr)
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return dt / rows, rows, dt
+
+
+def oracle_decode_sample(w: workloads.Workload, budget_s: float):
+    """Whole decode sequences (every query head against its KV head's full cache) through
+    the fp64 oracle until ``budget_s`` is spent; returns (sequences, seconds)."""
+    import oracle
+    G = w.Hq // w.Hkv
+    # sequence 0's inputs (the CPU draw of the same seeds), reused for every timed sequence
+    q = workloads.randn_bf16((1, w.Hq, 1, w.d), w.seed, 0)[0].float().numpy()
+    k = workloads.randn_bf16((1, w.Hkv, w.Nk, w.d), w.seed, 1)[0].float().numpy()
+    v = workloads.randn_bf16((1, w.Hkv, w.Nk, w.d), w.seed, 2)[0].float().numpy()
+    seqs, t0 = 0, time.perf_counter()
+    while seqs < w.B:
+        for h in range(w.Hq):
+            oracle.attention_head(q[h], np.arange(1), k[h // G], v[h // G], w.scale)
+        seqs += 1
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    return seqs, time.perf_counter() - t0
 
 
 def l2_note(*tensors) -> str:
@@ -378,9 +469,34 @@ def decode_workload(args):
     return w
 
 
-def bench_prefill_variant(w, args, world, local, peaks, peak_src):
-    """Useful TFLOP/s of attn_fwd on another prefill workload (ALiBi, symmetric window):
-    the same timing as the headline, fewer steps."""
+def tensor_peak_at_clock(sm_mhz, n_sms: int) -> float | None:
+    """Dense bf16 tensor throughput (TFLOP/s) of the chip at the sampled SM clock: one
+    128x128x16 tcgen05 product (524288 flops) every 64 cycles per SM, measured with a probe,
+    i.e. 8192 flops per cycle per SM."""
+    if not sm_mhz:
+        return None
+    return 8192.0 * n_sms * sm_mhz * 1e6 / 1e12
+
+
+def prefill_roofline(flops, executed, kernel_ms, peaks, peak_src, clocks, kernel, traffic,
+                     n_sms):
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    achieved = flops / (kernel_ms * 1e-3) / 1e12
+    exe = executed / (kernel_ms * 1e-3) / 1e12
+    at_clk = tensor_peak_at_clock(clocks.get("sm_mhz"), n_sms)
+    return {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
+            "frac": round(achieved / peak, 4), "peak_source": f"bf16_tflops (burst, {peak_src})",
+            "frac_of_spec": round(achieved / SPEC_PEAKS["bf16_tflops"], 4),
+            "executed_tflops": round(exe, 2),
+            "tensor_peak_at_clock": round(at_clk, 1) if at_clk else None,
+            "executed_frac_at_clock": round(exe / at_clk, 4) if at_clk else None,
+            "kernel_ms": round(kernel_ms, 4), "kernel": kernel, "traffic": traffic}
+
+
+def bench_prefill_variant(w, args, world, local, peaks, peak_src, steps=None):
+    """Useful TFLOP/s of attn_fwd on a prefill workload other than the headline (sliding-
+    window GQA, packed documents with soft-cap, ALiBi, symmetric window): the same timing as
+    the headline, fewer steps."""
     import torch
     import io_aware_softmax_b200 as attn
     dev = torch.device("cuda", torch.cuda.current_device())
@@ -389,15 +505,18 @@ def bench_prefill_variant(w, args, world, local, peaks, peak_src):
     lse = torch.empty((w.B, w.Hq, w.Nq), dtype=torch.float32, device=dev)
     slopes = (torch.tensor(workloads.alibi_slopes(w.Hq), dtype=torch.float32, device=dev)
               if w.alibi else None)
-    flops = accounting.prefill_useful_flops(w.B, w.Hq, w.Nq, w.Nk, w.d, w.mask_kind, w.window)
+    docs = workloads.workload_doc_offsets(w)
+    doc_t = None if docs is None else torch.from_numpy(docs).to(dev)
+    flops = accounting.prefill_useful_flops(w.B, w.Hq, w.Nq, w.Nk, w.d, w.mask_kind, w.window,
+                                            docs)
     executed = accounting.prefill_executed_flops(w.B, w.Hq, w.Nq, w.Nk, w.d, w.mask_kind,
-                                                 w.window)
+                                                 w.window, docs)
 
     def step():
         attn.attn_fwd(q, k, v, scale=w.scale, mask=w.mask_kind, window=w.window,
-                      alibi_slopes=slopes, out=o, lse=lse)
+                      softcap=w.softcap, doc_offsets=doc_t, alibi_slopes=slopes, out=o, lse=lse)
 
-    steps = max(3, min(args.steps, 30))
+    steps = steps or max(3, min(args.steps, 30))
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
@@ -407,21 +526,20 @@ def bench_prefill_variant(w, args, world, local, peaks, peak_src):
         raise RuntimeError(f"device status not ok after {w.name}")
     ms = max_over_ranks(world, total_ms / steps)
     kernel_ms = max_over_ranks(world, sum(per) / len(per))
-    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
-    achieved = flops / (kernel_ms * 1e-3) / 1e12
-    res = {"config": {**w.describe(), "l2": l2_note(q, k, v)},
+    clocks = clk.summary()
+    kernel = "attn_fwd_sm100_kernel<%d>%s" % (w.d, " (ALiBi)" if w.alibi else "")
+    cfg = {**w.describe(), "l2": l2_note(q, k, v)}
+    if docs is not None:
+        cfg["num_docs"] = len(docs) - 1
+    res = {"config": cfg,
            "value": round(whole_job_rate(flops, world, ms) / 1e12, 2),
            "unit": "TFLOP/s", "ms_per_step": round(ms, 4), "steps": steps,
            "useful_tflop_per_step": round(flops / 1e12, 4),
            "executed_tflop_per_step": round(executed / 1e12, 4),
-           "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak,
-                        "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
-                        "peak_source": f"bf16_tflops (burst, {peak_src})",
-                        "frac_of_spec": round(achieved / SPEC_PEAKS["bf16_tflops"], 4),
-                        "executed_tflops": round(executed / (kernel_ms * 1e-3) / 1e12, 2),
-                        "kernel": "attn_fwd_sm100_kernel<128>" + (" (ALiBi)" if w.alibi else ""),
-                        "traffic": recorded_traffic("prefill_" + w.name)},
-           "gpu_launches": steps, "clocks": clk.summary()}
+           "roofline": prefill_roofline(flops, executed, kernel_ms, peaks, peak_src, clocks,
+                                        kernel, recorded_traffic("prefill_" + w.name),
+                                        torch.cuda.get_device_properties(dev).multi_processor_count),
+           "gpu_launches": steps, "clocks": clocks}
     del q, k, v, o, lse
     torch.cuda.empty_cache()
     return res
@@ -580,12 +698,34 @@ def bench_fp8(w, args, world, local, peaks, peak_src):
     call_ms = max_over_ranks(world, sum(per) / len(per))
     peak = 2.0 * float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     achieved = flops / (call_ms * 1e-3) / 1e12
+    # the whole FP8 path from bf16 inputs: quantize Q, K, V, then the FP8 prefill
+    def full_step():
+        q8_, qs_, k8_, ks_, vt8_, vs_ = quant()
+        attn.attn_fwd_fp8(q8_, qs_, k8_, ks_, vt8_, vs_, scale=w.scale, mask=w.mask_kind,
+                          window=w.window, out=o, lse=lse)
+
+    for _ in range(2):
+        full_step()
+    torch.cuda.synchronize()
+    full_ms, _ = time_launches(full_step, steps, world)
+    full_ms = max_over_ranks(world, full_ms / steps)
+    quant_bytes = 3 * q.numel() * 2 + 3 * q.numel()   # bf16 read, E4M3 written (Hq = Hkv)
+    qt = max_over_ranks(world, qt_ms / 3)
     res = {"config": {**w.describe(), "dtype": "e4m3 (P e4m3), bf16 O",
                       "l2": l2_note(q8, k8, vt8),
                       "scales": "Q, K per 128 rows after Hadamard rotation; V per head"},
+           "with_quantize": {"value": round(whole_job_rate(flops, world, full_ms) / 1e12, 2),
+                             "unit": "TFLOP/s", "ms_per_step": round(full_ms, 4),
+                             "note": "quantization of the bf16 Q, K, V inside the timed step"},
+           "quantize": {"ms": round(qt, 4), "bytes": quant_bytes,
+                        "gbs": round(quant_bytes / (qt * 1e-3) / 1e9, 1),
+                        "frac_of_hbm": round(quant_bytes / (qt * 1e-3) / 1e9 /
+                                             float(peaks.get("hbm_gbs",
+                                                             FALLBACK_PEAKS["hbm_gbs"])), 4),
+                        "launches": "Q, K: 1 each; V (transposed, one scale per head): 3"},
+           "accuracy": fp8_accuracy(w),
            "value": round(whole_job_rate(flops, world, ms) / 1e12, 2), "unit": "TFLOP/s",
            "ms_per_step": round(ms, 4), "steps": steps,
-           "quantize_ms": round(max_over_ranks(world, qt_ms / 3), 4),
            "useful_tflop_per_step": round(flops / 1e12, 4),
            "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak,
                         "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
@@ -597,6 +737,36 @@ def bench_fp8(w, args, world, local, peaks, peak_src):
     del q, k, v, q8, k8, vt8, o, lse
     torch.cuda.empty_cache()
     return res
+
+
+def fp8_accuracy(w, heads: int = 4, n: int = 1024, seed: int = 71) -> dict:
+    """FP8 output error against the bf16 path (attn_fwd) on the same inputs, with and without
+    the Hadamard rotation: N(0,1) inputs whose Q and K carry 0.1 % outlier entries of std 10,
+    causal, d = 128, a few heads of the workload's length scale."""
+    import torch
+    import io_aware_softmax_b200 as attn
+    dev = torch.device("cuda", torch.cuda.current_device())
+    gen = torch.Generator(device=dev).manual_seed(seed)
+    q, k, v = (workloads.randn_bf16((1, heads, n, w.d), seed, i, 1.0, dev) for i in range(3))
+    for t in (q, k):
+        hit = torch.rand(t.shape, generator=gen, device=dev) < 1e-3
+        t[hit] = (torch.randn(t.shape, generator=gen, device=dev)[hit] * 10.0).to(t.dtype)
+    o_ref, l_ref = attn.attn_fwd(q, k, v, mask="causal")
+    out = {"vs": "attn_fwd (bf16) on the same inputs",
+           "input": f"1x{heads}x{n}x{w.d}, causal, N(0,1) with 0.1 % outlier entries (std 10) "
+                    "in Q and K"}
+    for name, rot in (("rotated", True), ("plain", False)):
+        signs = (torch.from_numpy(np.random.default_rng(seed).choice([-1.0, 1.0], w.d)
+                                  .astype(np.float32)).to(dev) if rot else None)
+        q8, qs = attn.quantize_fp8(q, block_rows=128, signs=signs)
+        k8, ks = attn.quantize_fp8(k, block_rows=128, signs=signs)
+        vt8, vs = attn.quantize_fp8(v, block_rows=n, transpose=True)
+        o, l = attn.attn_fwd_fp8(q8, qs, k8, ks, vt8, vs[:, :, 0].contiguous(), mask="causal")
+        err = (o.float() - o_ref.float())
+        out[name] = {"o_rmse": round(float(err.pow(2).mean().sqrt()), 6),
+                     "o_max": round(float(err.abs().max()), 5),
+                     "lse_max": round(float((l - l_ref).abs().max()), 6)}
+    return out
 
 
 def e2e_prefill(w, args, world, q, k, v):
@@ -747,6 +917,9 @@ def main(argv=None):
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle time")
     ap.add_argument("--only", choices=["all", "prefill", "decode", "extras"], default="all",
                     help="run one part only (profiling runs)")
+    ap.add_argument("--workload", choices=sorted(n for n, x in workloads.BY_NAME.items()
+                                                 if x.kind == "prefill"), default=None,
+                    help="time attn_fwd on this prefill workload only (profiling runs)")
     ap.add_argument("--decode-batch", type=int, default=None,
                     help="decode batch size override (smaller caches for ncu captures)")
     args = ap.parse_args(argv)
