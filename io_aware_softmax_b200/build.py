@@ -21,7 +21,7 @@ LIB_NAME = "libattn_b200.so"
 LIB_PATH = os.path.join(PKG_DIR, LIB_NAME)
 SOURCES = ["attn_api.cu", "attn_prefill.cu", "attn_decode.cu", "attn_blockmap.cu",
            "attn_decode_noalloc.cu", "attn_backward.cu", "attn_fp8.cu"]
-HEADERS = ["attn_internal.h", "mask.cuh", "sm100_ptx.cuh", "tmem_ldst.cuh"]
+HEADERS = ["attn_internal.h", "mask.cuh", "sm100_ptx.cuh", "tmem_ldst.cuh", "tanh_poly.cuh"]
 ARCH_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 # Kernels that split their launch registers between warpgroups with setmaxnreg (two

@@ -12,6 +12,7 @@
 #include "../../include/attn.h"
 #include "attn_internal.h"
 #include "sm100_ptx.cuh"
+#include "tanh_poly.cuh"
 
 namespace attn {
 
@@ -192,6 +193,9 @@ extern "C" int attn_fwd_alibi(const void* q, const void* k, const void* v, void*
   p.softcap = softcap > 0.f ? softcap : 0.f;
   p.cap_scale = softcap > 0.f ? scale / softcap : 0.f;
   p.cap_log2 = softcap > 0.f ? softcap * kLog2e : 0.f;
+  static_assert(sizeof(p.cap_poly) / sizeof(float) == kTanhPolyTerms, "soft-cap polynomial");
+  for (int i = 0; i < kTanhPolyTerms; ++i) p.cap_poly[i] = kTanhPoly[i] * p.cap_log2;
+  p.cap_fast_max = softcap > 0.f ? kTanhPolyMaxY / p.cap_scale : 0.f;
   p.mask = mask_params(mask_kind, window, doc_offsets, num_docs, Nq, Nk);
   p.alibi = alibi_slopes;
   if ((long long)p.num_pairs * B * Hq > (1LL << 31) - 1) return ATTN_ERR_UNSUPPORTED;

@@ -349,6 +349,7 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     mbar_init(bar(BAR_ACC), 1);
     mbar_init(bar(BAR_DONE), 1);
     *abort_flag = 0;
+    init_wait_limit(abort_flag, p.err);
     fence_mbar_init();
   }
   if (warp == kBwdMmaWarp) {
@@ -614,6 +615,7 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ,
       mbar_init(sm.bar(BAR_VE + i), 8);      // every element-wise warp
     }
     *abort_flag = 0;
+    init_wait_limit(abort_flag, p.err);
     fence_mbar_init();
   }
   if (warp == kBwdMmaWarp) {

@@ -47,8 +47,9 @@ struct DecCfg {
 };
 
 __host__ __device__ constexpr int dec_smem_bytes(int D, int G) {
-  // ring + per-warp (m, l, O rows) scratch for the in-CTA merge + barriers + alignment
-  return kStagesDec * 2 * (D / 64) * kTok * 128 + kConsumerWarps * G * (D + 2) * 4 + 64 + 1024;
+  // ring + per-warp (m, l, O rows) scratch for the in-CTA merge + barriers, the abort flag
+  // and the wait limit (with their 8-byte alignment) + alignment of the base
+  return kStagesDec * 2 * (D / 64) * kTok * 128 + kConsumerWarps * G * (D + 2) * 4 + 96 + 1024;
 }
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
@@ -132,6 +133,7 @@ attn_decode_split_kernel(const __grid_constant__ CUtensorMap tmK,
       mbar_init(empty_bar(s), kConsumerWarps);
     }
     *abort_flag = 0;
+    init_wait_limit(abort_flag, p.err);
     fence_mbar_init();
   }
   __syncthreads();

@@ -21,6 +21,10 @@ struct FwdParams {
   float softcap;      // > 0: soft-cap enabled
   float cap_scale;    // scale / softcap
   float cap_log2;     // softcap * log2(e)
+  // Soft-cap on the FMA pipe: cap_log2 * tanh(y) = y * sum_i cap_poly[i] y^(2i) for
+  // |y| = |s cap_scale| <= 1, i.e. for raw scores |s| <= cap_fast_max
+  float cap_poly[7];
+  float cap_fast_max;
   MaskParams mask;
   const float* alibi; // fp32 [Hq] ALiBi slopes (natural-log units per key of distance) or null
   // FP8 (E4M3) inputs, null otherwise: per 128-row block scales of Q and K, per head of V

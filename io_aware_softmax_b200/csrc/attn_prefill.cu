@@ -101,6 +101,30 @@ __device__ __forceinline__ float tile_row_max(uint32_t (&s)[128], int c_lo, int 
   return max3f(m0, m1, fmaxf(m2, m3));
 }
 
+// Soft-cap path: the row maximum over the visible columns [c_lo, c_hi] (all columns when not
+// kMasked) and the largest |s| over all 128 columns, leaving s unmasked (the polynomial tanh
+// is evaluated on every column and the mask applied after it).
+template <bool kMasked>
+__device__ __forceinline__ float tile_row_max_keep(const uint32_t (&s)[128], int c_lo, int c_hi,
+                                                   float& mabs) {
+  float m0 = -INFINITY, m1 = -INFINITY, a0 = 0.f, a1 = 0.f;
+#pragma unroll
+  for (int c = 0; c < 128; c += 4) {
+    float v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      v[u] = f32(s[c + u]);
+      if (kMasked && (unsigned)(c + u - c_lo) > (unsigned)(c_hi - c_lo)) v[u] = -INFINITY;
+    }
+    m0 = max3f(m0, v[0], v[1]);
+    m1 = max3f(m1, v[2], v[3]);
+    a0 = max3f(a0, fabsf(f32(s[c])), fabsf(f32(s[c + 1])));
+    a1 = max3f(a1, fabsf(f32(s[c + 2])), fabsf(f32(s[c + 3])));
+  }
+  mabs = fmaxf(a0, a1);
+  return fmaxf(m0, m1);
+}
+
 // Scaled (base-2) score of a raw score: s * scale * log2(e), or with the soft-cap
 // c * log2(e) * tanh(s * scale / c).  -inf (masked) stays -inf.
 template <bool kSoftcap>
@@ -188,6 +212,42 @@ __device__ __forceinline__ float tile_row_exp_half(const uint32_t (&s)[128], int
   return ((a0 + a1) + (b0 + b1)) + ((c0 + c1) + (d0 + d1));
 }
 
+// Soft-capped P = 2^(c log2(e) tanh(s scale / c) - m_use) for one 64-column half of a row
+// whose raw scores all satisfy |s| <= p.cap_fast_max: tanh is the odd polynomial
+// y * sum_i a_i y^(2i) (|y| <= 1) with c log2(e) folded into p.cap_poly, evaluated in paired
+// FMAs, so the exponential is the only MUFU operation per score.  kMasked: columns outside
+// [c_lo, c_hi] get P = 0.  Returns the half's sum.
+template <bool kMasked>
+__device__ __forceinline__ float tile_row_exp_half_cap(const uint32_t (&s)[128], int base,
+                                                       const FwdParams& p, float m_use,
+                                                       uint32_t (&pk)[32], int c_lo, int c_hi) {
+  float a0 = 0.f, a1 = 0.f, b0 = 0.f, b1 = 0.f;
+  const float cs = p.cap_scale;
+#pragma unroll
+  for (int c = 0; c < 64; c += 2) {
+    float y0, y1, w0, w1;
+    fmul2(y0, y1, f32(s[base + c]), f32(s[base + c + 1]), cs, cs);
+    fmul2(w0, w1, y0, y1, y0, y1);
+    float q0 = p.cap_poly[6], q1 = p.cap_poly[6];
+#pragma unroll
+    for (int i = 5; i >= 0; --i) ffma2(q0, q1, q0, q1, w0, w1, p.cap_poly[i], p.cap_poly[i]);
+    float x0, x1;
+    ffma2(x0, x1, y0, y1, q0, q1, -m_use, -m_use);
+    if (kMasked) {
+      if ((unsigned)(base + c - c_lo) > (unsigned)(c_hi - c_lo)) x0 = -INFINITY;
+      if ((unsigned)(base + c + 1 - c_lo) > (unsigned)(c_hi - c_lo)) x1 = -INFINITY;
+    }
+    const float e0 = ex2_approx(x0);
+    const float e1 = ex2_approx(x1);
+    if ((c >> 1) & 1)
+      add2(b0, b1, e0, e1);
+    else
+      add2(a0, a1, e0, e1);
+    pk[c >> 1] = pack_bf16x2(e0, e1);
+  }
+  return (a0 + a1) + (b0 + b1);
+}
+
 // K/V tiles [a, b] (relative to the CTA's first tile) that query tile t must visit; n = 0
 // when the tile has no valid row.
 struct TileRange {
@@ -254,7 +314,7 @@ __device__ __forceinline__ void for_each_pair(const FwdParams& p, F&& f) {
   }
 }
 
-template <int D, bool kAlibi, bool kFp8>
+template <int D, bool kAlibi, bool kFp8, bool kCap>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
                       const __grid_constant__ CUtensorMap tmK,
@@ -262,6 +322,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
   using C = Cfg<D, kFp8>;
   constexpr int NS = C::kStages;
   static_assert(!(kFp8 && (kAlibi || D != 128)), "FP8 path: d = 128, no bias");
+  static_assert(!(kCap && (kFp8 || kAlibi)), "soft-cap: bf16 path without bias");
   // FP8: the lazy-rescale bound is 2^2 and P is stored as E4M3 of 64 P (<= 256 < 448), so
   // probabilities down to 2^-12 of the reference stay in E4M3's normal range.
   constexpr float kThreshold = kFp8 ? 2.0f : kRescaleThreshold;
@@ -299,6 +360,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
     }
     mbar_init(bar(BAR_DONE), 1);
     *abort_flag = 0;
+    init_wait_limit(abort_flag, p.err);
     fence_mbar_init();
   }
   if (warp == kMmaWarp) {
@@ -563,16 +625,26 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
         const bool masked =
             !(lo_last <= k0 && k0 + kBN - 1 <= hi_first && k0 + kBN <= p.Nk);
         float mx;
+        bool cap_poly = false;   // soft-cap row small enough for the polynomial tanh
         const float ks_eff = kFp8 ? p.kscale * qs * __ldg(ksc + k0 / kBN) : p.kscale;
         if constexpr (kFp8) {
           const float mx_raw = masked ? tile_row_max<true>(s, row_lo - k0, row_hi - k0)
                                       : tile_row_max<false>(s, 0, 0);
           mx = mx_raw * ks_eff;
+        } else if constexpr (kCap) {
+          // The cap is increasing, so the row max of the capped scores is the cap of the raw
+          // row max.  The polynomial tanh covers the row when its largest |s| is in range;
+          // otherwise the row takes the exact form on masked scores.
+          float mabs;
+          const float mx_raw = masked ? tile_row_max_keep<true>(s, row_lo - k0, row_hi - k0, mabs)
+                                      : tile_row_max_keep<false>(s, 0, 0, mabs);
+          cap_poly = mabs <= p.cap_fast_max;
+          if (!cap_poly && masked) mask_row(s, row_lo - k0, row_hi - k0);
+          mx = scaled_score<true>(mx_raw, p);
         } else if constexpr (!kAlibi) {
           const float mx_raw = masked ? tile_row_max<true>(s, row_lo - k0, row_hi - k0)
                                       : tile_row_max<false>(s, 0, 0);
-          mx = (p.softcap > 0.f) ? scaled_score<true>(mx_raw, p)
-                                 : scaled_score<false>(mx_raw, p);
+          mx = scaled_score<false>(mx_raw, p);
         } else {
           // The bias changes the order of the scores, so the row max is taken over the
           // biased, base-2 scores themselves.
@@ -615,8 +687,14 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
             uint32_t pk[32];
             if constexpr (kAlibi) {
               sum += tile_row_exp_half<false>(s, 64 * half, p, 1.f, m_use, pk);
-            } else if (p.softcap > 0.f) {
-              sum += tile_row_exp_half<true>(s, 64 * half, p, p.kscale, m_use, pk);
+            } else if constexpr (kCap) {
+              if (!cap_poly)
+                sum += tile_row_exp_half<true>(s, 64 * half, p, p.kscale, m_use, pk);
+              else if (masked)
+                sum += tile_row_exp_half_cap<true>(s, 64 * half, p, m_use, pk, row_lo - k0,
+                                                   row_hi - k0);
+              else
+                sum += tile_row_exp_half_cap<false>(s, 64 * half, p, m_use, pk, 0, 0);
             } else {
               sum += tile_row_exp_half<false>(s, 64 * half, p, p.kscale, m_use, pk);
             }
@@ -682,31 +760,37 @@ __global__ void attn_fill_empty_kernel(__nv_bfloat16* o, float* lse, size_t rows
   if (i < rows) lse[i] = -INFINITY;
 }
 
-template <int D, bool kAlibi, bool kFp8 = false>
+template <int D, bool kAlibi, bool kFp8 = false, bool kCap = false>
 int launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                const FwdParams& p, cudaStream_t stream) {
   using C = Cfg<D, kFp8>;
   static_assert(C::kSmemBytes <= 227 * 1024, "shared memory budget");
-  cudaError_t e = cudaFuncSetAttribute(attn_fwd_sm100_kernel<D, kAlibi, kFp8>,
+  cudaError_t e = cudaFuncSetAttribute(attn_fwd_sm100_kernel<D, kAlibi, kFp8, kCap>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        C::kSmemBytes);
   if (e != cudaSuccess) return -4;
   const long long units = (long long)((p.num_pairs + 1) / 2) * p.B * p.Hq;
   const long long grid = units < p.num_sms ? units : p.num_sms;
-  attn_fwd_sm100_kernel<D, kAlibi, kFp8>
+  attn_fwd_sm100_kernel<D, kAlibi, kFp8, kCap>
       <<<(unsigned)grid, kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, p);
   return cudaGetLastError() == cudaSuccess ? 0 : -4;
 }
 
 }  // namespace
 
+// One kernel per combination of hooks, so that each carries only its own softmax code (the
+// unrolled per-row loops are long, and a kernel holding several variants ran slower).
 int launch_attn_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                     const FwdParams& p, int d, cudaStream_t stream) {
   const bool alibi = p.alibi != nullptr;
+  const bool cap = p.softcap > 0.f;
   if (p.q_scales != nullptr) return d == 128 ? launch_fwd<128, false, true>(tq, tk, tv, p, stream) : -2;
+  if (alibi && cap) return -2;
   if (d == 128) return alibi ? launch_fwd<128, true>(tq, tk, tv, p, stream)
+                       : cap ? launch_fwd<128, false, false, true>(tq, tk, tv, p, stream)
                              : launch_fwd<128, false>(tq, tk, tv, p, stream);
   if (d == 64) return alibi ? launch_fwd<64, true>(tq, tk, tv, p, stream)
+                      : cap ? launch_fwd<64, false, false, true>(tq, tk, tv, p, stream)
                             : launch_fwd<64, false>(tq, tk, tv, p, stream);
   return -2;
 }

@@ -96,11 +96,20 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parit
 
 constexpr uint32_t kWaitSleepNs = 200u * 1000u;   // one sleep of a waiting thread, at most
 
-// Limit of a wait: the library's setting for pipeline waits (abort != nullptr), the full
+// Every kernel keeps, in shared memory, its CTA's abort flag followed by two words that hold
+// the pipeline-wait limit (low, high), copied from err[2..3] by one thread before the CTA's
+// first barrier: a wait reads its limit from shared memory, never from global memory.
+__device__ __forceinline__ void init_wait_limit(volatile int* abort, const uint32_t* err) {
+  const volatile uint32_t* e = err;
+  abort[1] = (int)e[2];
+  abort[2] = (int)e[3];
+}
+
+// Limit of a wait: the kernel's setting for pipeline waits (abort != nullptr), the full
 // kWaitLimitNs for drain waits.
-__device__ __forceinline__ uint64_t wait_limit_ns(const uint32_t* err, const volatile int* abort) {
+__device__ __forceinline__ uint64_t wait_limit_ns(const volatile int* abort) {
   if (abort == nullptr) return kWaitLimitNs;
-  const uint64_t v = *reinterpret_cast<const volatile uint64_t*>(err + 2);
+  const uint64_t v = ((uint64_t)(uint32_t)abort[2] << 32) | (uint32_t)abort[1];
   return v != 0 ? v : kWaitLimitNs;
 }
 
@@ -112,7 +121,7 @@ static __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, 
                                                  uint32_t* err, uint32_t site) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
-  const uint64_t limit = wait_limit_ns(err, abort);
+  const uint64_t limit = wait_limit_ns(abort);
   const uint32_t sleep_ns = limit < kWaitSleepNs ? (uint32_t)limit : kWaitSleepNs;
   for (;;) {
     if (mbar_try_wait_sleep(bar, parity, sleep_ns)) return true;
@@ -132,7 +141,7 @@ static __device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t par
                                                       uint32_t site) {
   if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
   const uint64_t t0 = globaltimer_ns();
-  const uint64_t limit = wait_limit_ns(err, abort);
+  const uint64_t limit = wait_limit_ns(abort);
   const uint32_t sleep_ns = limit < kWaitSleepNs ? (uint32_t)limit : kWaitSleepNs;
   for (;;) {
     if (__all_sync(0xffffffffu, mbar_try_wait_sleep(bar, parity, sleep_ns))) return true;
@@ -340,6 +349,14 @@ __device__ __forceinline__ void ffma2(float& d0, float& d1, float a0, float a1, 
       "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
       : "=f"(d0), "=f"(d1)
       : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
+}
+__device__ __forceinline__ void fmul2(float& d0, float& d1, float a0, float a1, float b0,
+                                      float b1) {
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
 }
 __device__ __forceinline__ void add2(float& a0, float& a1, float b0, float b1) {
   asm("{\n\t.reg .b64 ra, rb;\n\t"

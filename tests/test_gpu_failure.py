@@ -49,13 +49,16 @@ def test_prefill_wait_that_runs_out_is_reported_and_the_next_call_is_clean():
 
 
 def test_decode_wait_that_runs_out_is_reported_and_the_next_call_is_clean():
-    q = workloads.randn_bf16((2, 8, 1, 128), 52, 0).cuda()
-    kc = workloads.randn_bf16((2, 2, 3000, 128), 52, 1).cuda()
-    vc = workloads.randn_bf16((2, 2, 3000, 128), 52, 2).cuda()
-    status = _run_with_tiny_limit(lambda: attn_decode(q, kc, vc, num_splits=4))
+    # one sequence, one split: a single CTA streams 1024 cache stages through its three-stage
+    # ring, so its consumers wait for a copy from memory at almost every stage (the device
+    # timer advances in steps of up to a microsecond; waits this long always see it move)
+    q = workloads.randn_bf16((1, 4, 1, 128), 52, 0).cuda()
+    kc = workloads.randn_bf16((1, 1, 65536, 128), 52, 1).cuda()
+    vc = workloads.randn_bf16((1, 1, 65536, 128), 52, 2).cuda()
+    status = _run_with_tiny_limit(lambda: attn_decode(q, kc, vc, num_splits=1))
     assert status == ATTN_ERR_DEVICE_TIMEOUT
     assert attn_last_error_site() != 0
-    o, lse = attn_decode(q, kc, vc, num_splits=4)
+    o, lse = attn_decode(q, kc, vc, num_splits=1)
     assert device_status() == 0
     O_ref, L_ref = oracle.attention(f64(q), f64(kc), f64(vc))
     compare(o, lse, O_ref, L_ref, "decode after a timed-out call")

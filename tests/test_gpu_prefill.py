@@ -88,6 +88,9 @@ def test_softcap(mask):
               v_std=2.0)
     _run_full(1, 2, 2, 300, 300, 64, mask=mask if mask != "document_causal" else "causal",
               softcap=5.0, seed=4, std=3.0)
+    # cap 10 with std-2 inputs: |scale s / cap| ~ 0.4, so rows above and below the
+    # polynomial tanh's range of 1 mix inside every warp
+    _run_full(1, 2, 2, 520, 520, 128, mask=mask, softcap=10.0, docs=docs, seed=5, std=2.0)
 
 
 @pytest.mark.parametrize("Nq,Nk", [(1, 300), (100, 1000), (300, 129), (513, 64)])
