@@ -5,8 +5,8 @@
 // by the orthogonal matrix diag(signs) H / sqrt(d) (H the Sylvester Hadamard matrix), which
 // leaves Q K^T unchanged and spreads outlier columns over all of d.
 //
-// Row-major output with blocks of at most 128 rows: one launch, one CTA per block, a warp
-// per row at a time, the block read twice (amax, then codes; the second read hits cache).
+// Row-major output with blocks of at most 128 rows: one launch, one CTA per block, the
+// block held in registers between its amax and its codes (read once).
 // Larger blocks or a transposed output: three launches over chunks of 64 rows of one
 // (batch, head), 256 threads each, a warp per 8 consecutive rows.  In both, lane l holds
 // columns [l d/32, (l + 1) d/32) of a row and the Hadamard butterflies run in registers and
@@ -206,41 +206,49 @@ quant_codes_kernel(const __nv_bfloat16* __restrict__ x, uint8_t* __restrict__ ou
   }
 }
 
-// Small row-major blocks in one launch: amax of the block, its scale, then the codes.
+// Row-major blocks of at most 128 rows in one pass: one CTA per block, warp w holding rows
+// w, w + 8, ... of it.  Every row of the block is loaded (and rotated) into registers before
+// any is used -- 16 independent loads in flight per warp -- then the block's amax is reduced
+// across the CTA and the codes are written from the same registers: the input is read once.
 template <int D>
 __global__ void __launch_bounds__(kQuantThreads)
 quant_block_kernel(const __nv_bfloat16* __restrict__ x, uint8_t* __restrict__ out,
                    float* __restrict__ scales, int N, int block_rows, int nblk,
                    const float* __restrict__ signs) {
   constexpr int E = D / 32;
-  __shared__ unsigned int s_amax;
+  constexpr int kWarps = kQuantThreads / 32;
+  constexpr int kRows = 128 / kWarps;                 // rows per warp, at most
+  __shared__ float s_amax[kWarps];
   const int bh = blockIdx.x / nblk, blk = blockIdx.x % nblk;
   const int r0 = blk * block_rows, r1 = min(N, r0 + block_rows);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  constexpr int kWarps = kQuantThreads / 32;
-  if (threadIdx.x == 0) s_amax = 0u;
-  __syncthreads();
-  float amax = 0.f;
-  for (int r = r0 + warp; r < r1; r += kWarps) {
-    float v[E];
-    load_row<D>(x, (long long)bh * N + r, true, signs, v);
+  float v[kRows][E];
 #pragma unroll
-    for (int e = 0; e < E; ++e) amax = fmaxf(amax, fabsf(v[e]));
+  for (int i = 0; i < kRows; ++i) {
+    const int r = r0 + warp + i * kWarps;
+    load_row<D>(x, (long long)bh * N + r, r < r1, signs, v[i]);
   }
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < kRows; ++i)
+#pragma unroll
+    for (int e = 0; e < E; ++e) amax = fmaxf(amax, fabsf(v[i][e]));   // rows past r1 are 0
 #pragma unroll
   for (int s = 16; s > 0; s >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, s));
-  if (lane == 0) atomicMax(&s_amax, __float_as_uint(amax));   // non-negative: order of bits
+  if (lane == 0) s_amax[warp] = amax;
   __syncthreads();
-  amax = __uint_as_float(s_amax);
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w) amax = fmaxf(amax, s_amax[w]);
   const float inv = amax > 0.f ? kE4m3Max / amax : 1.f;
   if (threadIdx.x == 0) scales[(long long)bh * nblk + blk] = amax > 0.f ? amax / kE4m3Max : 1.f;
-  for (int r = r0 + warp; r < r1; r += kWarps) {
-    float v[E];
-    load_row<D>(x, (long long)bh * N + r, true, signs, v);
+#pragma unroll
+  for (int i = 0; i < kRows; ++i) {
+    const int r = r0 + warp + i * kWarps;
+    if (r >= r1) break;
     uint32_t c = 0;
 #pragma unroll
     for (int e = 0; e < E; ++e)
-      c |= (uint32_t)__nv_cvt_float_to_fp8(v[e] * inv, __NV_SATFINITE, __NV_E4M3) << (8 * e);
+      c |= (uint32_t)__nv_cvt_float_to_fp8(v[i][e] * inv, __NV_SATFINITE, __NV_E4M3) << (8 * e);
     uint8_t* dst = out + ((long long)bh * N + r) * D + lane * E;
     if constexpr (E == 4)
       *reinterpret_cast<uint32_t*>(dst) = c;
