@@ -16,9 +16,12 @@
  *     Each array must hold at least the elements its stated shape implies: the library
  *     sees only pointers and sizes, so it cannot check an allocation's extent (the Python
  *     binding checks every tensor's shape, dtype and device before it calls in).
- *   - Calls are asynchronous on `stream`; they never synchronise, never allocate and keep
- *     no state across calls except a per-process cache of device attributes, so they may be
- *     recorded into a CUDA graph with fixed shapes ("CUDA 그래프와의 호환성").
+ *   - The compute entry points (attn_fwd, attn_fwd_alibi, attn_bwd, attn_bwd_alibi,
+ *     attn_quantize_fp8, attn_fwd_fp8, attn_blockmap, attn_decode_splitkv, attn_decode_paged,
+ *     attn_decode_merge) are asynchronous on `stream`; they never synchronise, never allocate
+ *     and keep no state across calls except a per-process cache of device attributes, so
+ *     they may be recorded into a CUDA graph with fixed shapes ("CUDA 그래프와의 호환성").
+ *     attn_get_device_status and attn_set_wait_limit_ns synchronise.
  *   - Arguments are validated before anything is launched; an unsupported case returns
  *     ATTN_ERR_UNSUPPORTED and nothing runs -- there is no fallback path ("3.7 어텐션 II",
  *     section 3.7.3, on diagnosing silent fallbacks: here the failure is the diagnosis).
