@@ -31,6 +31,7 @@ ARCH_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a"]
 # (kernel name fragment, source, constant of the two big warpgroups, constant of the third)
 SPLIT_KERNELS = [
     ("attn_fwd_sm100_kernel", "attn_prefill.cu", "kRegsSoftmax", "kRegsOther"),
+    ("attn_fwd_sm100_kernel", "attn_prefill.cu", "kRegsSoftmaxCap", "kRegsOtherCap"),
     ("attn_bwd_dq_kernel", "attn_backward.cu", "kBwdRegsElem", "kBwdRegsOther"),
     ("attn_bwd_dkdv_kernel", "attn_backward.cu", "kBwdRegsElem", "kBwdRegsOther"),
 ]
@@ -41,8 +42,8 @@ PREFILL_THREADS = SPLIT_THREADS
 
 def split_regs(source: str, big: str, other: str) -> int:
     src = open(os.path.join(CSRC, source), encoding="utf-8").read()
-    n_big = int(re.search(big + r"\s*=\s*(\d+)", src).group(1))
-    n_other = int(re.search(other + r"\s*=\s*(\d+)", src).group(1))
+    n_big = int(re.search(big + r"\s*=\s*(\d+);", src).group(1))
+    n_other = int(re.search(other + r"\s*=\s*(\d+);", src).group(1))
     return 2 * 128 * n_big + 128 * n_other
 
 

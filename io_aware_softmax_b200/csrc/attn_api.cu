@@ -187,15 +187,32 @@ extern "C" int attn_fwd_alibi(const void* q, const void* k, const void* v, void*
   p.Nq = Nq;
   p.Nk = Nk;
   p.G = Hq / Hkv;
-  p.num_pairs = (Nq + 255) / 256;
+  // GQA with an even group: a CTA's two query tiles are two heads of one KV group at the
+  // same rows (same keys, same mask, each K/V tile used by both); otherwise two adjacent
+  // 128-row tiles of one head
+  p.head_pairs = (p.G % 2 == 0) ? 1 : 0;
+  p.num_pairs = p.head_pairs ? (Nq + 127) / 128 : (Nq + 255) / 256;
   p.num_sms = sm_count(current_device());
   p.kscale = scale * kLog2e;
   p.softcap = softcap > 0.f ? softcap : 0.f;
   p.cap_scale = softcap > 0.f ? scale / softcap : 0.f;
   p.cap_log2 = softcap > 0.f ? softcap * kLog2e : 0.f;
+  // The soft-cap's polynomial tanh in the raw score s: cap_log2 tanh(s cap_scale) =
+  // s sum_i b_i s^(2i) with b_i = cap_log2 a_i cap_scale^(2i + 1), for |s cap_scale| <= 1/2.
+  // The kernels take it only when every b_i is a normal float (no term flushed to zero).
   static_assert(sizeof(p.cap_poly) / sizeof(float) == kTanhPolyTerms, "soft-cap polynomial");
-  for (int i = 0; i < kTanhPolyTerms; ++i) p.cap_poly[i] = kTanhPoly[i] * p.cap_log2;
-  p.cap_fast_max = softcap > 0.f ? kTanhPolyMaxY / p.cap_scale : 0.f;
+  p.cap_fast_max = -1.f;
+  if (softcap > 0.f) {
+    bool normal = true;
+    double cs_pow = (double)p.cap_scale;
+    for (int i = 0; i < kTanhPolyTerms; ++i) {
+      const double b = (double)kTanhPoly[i] * (double)p.cap_log2 * cs_pow;
+      p.cap_poly[i] = (float)b;
+      normal = normal && std::isnormal(p.cap_poly[i]);
+      cs_pow *= (double)p.cap_scale * (double)p.cap_scale;
+    }
+    if (normal) p.cap_fast_max = kTanhPolyMaxY / p.cap_scale;
+  }
   p.mask = mask_params(mask_kind, window, doc_offsets, num_docs, Nq, Nk);
   p.alibi = alibi_slopes;
   if ((long long)p.num_pairs * B * Hq > (1LL << 31) - 1) return ATTN_ERR_UNSUPPORTED;
@@ -515,8 +532,10 @@ extern "C" int attn_quantize_fp8(const void* x, void* out, float* scales, int B,
       (reinterpret_cast<uintptr_t>(signs) & 3u))
     return ATTN_ERR_MISALIGNED;
   if (!transpose && (reinterpret_cast<uintptr_t>(out) & 3u)) return ATTN_ERR_MISALIGNED;
+  uint32_t* err = error_word_ptr(current_device());
+  if (err == nullptr) return ATTN_ERR_CUDA;
   return launch_quantize_e4m3(x, out, scales, B, H, N, d, block_rows, transpose, n_pad, signs,
-                              stream) == 0
+                              err, sm_count(current_device()), stream) == 0
              ? ATTN_OK
              : ATTN_ERR_CUDA;
 }
@@ -556,7 +575,11 @@ extern "C" int attn_fwd_fp8(const void* q8, const void* k8, const void* vt8,
   p.Nq = Nq;
   p.Nk = Nk;
   p.G = Hq / Hkv;
-  p.num_pairs = (Nq + 255) / 256;
+  // GQA with an even group: a CTA's two query tiles are two heads of one KV group at the
+  // same rows (same keys, same mask, each K/V tile used by both); otherwise two adjacent
+  // 128-row tiles of one head
+  p.head_pairs = (p.G % 2 == 0) ? 1 : 0;
+  p.num_pairs = p.head_pairs ? (Nq + 127) / 128 : (Nq + 255) / 256;
   p.num_sms = sm_count(current_device());
   p.kscale = scale * kLog2e;
   p.mask = mask_params(mask_kind, window, doc_offsets, num_docs, Nq, Nk);

@@ -15,15 +15,17 @@ struct FwdParams {
   float* lse;         // fp32 [B, Hq, Nq]
   int B, Hq, Hkv, Nq, Nk;
   int G;              // Hq / Hkv
-  int num_pairs;      // ceil(Nq / 256): query pairs per (b, h)
+  int num_pairs;      // work units per (b, h) [adjacent tiles: ceil(Nq / 256)] or per
+                      // (b, head pair) [head pairs: ceil(Nq / 128)]
+  int head_pairs;     // 1: a CTA's two query tiles are query heads 2m, 2m + 1 at the same rows
   int num_sms;        // persistent grid size (SMs of the device)
   float kscale;       // scale * log2(e)
   float softcap;      // > 0: soft-cap enabled
   float cap_scale;    // scale / softcap
   float cap_log2;     // softcap * log2(e)
-  // Soft-cap on the FMA pipe: cap_log2 * tanh(y) = y * sum_i cap_poly[i] y^(2i) for
-  // |y| = |s cap_scale| <= 1, i.e. for raw scores |s| <= cap_fast_max
-  float cap_poly[7];
+  // Soft-cap on the FMA pipe: cap_log2 * tanh(s cap_scale) = s * sum_i cap_poly[i] s^(2i)
+  // for raw scores |s| <= cap_fast_max (|s cap_scale| <= 1/2); cap_fast_max < 0 disables it
+  float cap_poly[5];
   float cap_fast_max;
   MaskParams mask;
   const float* alibi; // fp32 [Hq] ALiBi slopes (natural-log units per key of distance) or null
@@ -81,7 +83,7 @@ int launch_attn_bwd(const CUtensorMap& tq, const CUtensorMap& tdo, const CUtenso
                     const CUtensorMap& tv, const BwdParams& p, int d, cudaStream_t stream);
 int launch_quantize_e4m3(const void* x, void* out, float* scales, int B, int H, int N, int d,
                          int block_rows, int transpose, int n_pad, const float* signs,
-                         cudaStream_t stream);
+                         uint32_t* err, int num_sms, cudaStream_t stream);
 int launch_merge(const float* o_part, const float* lse_part, void* o, float* lse, long long rows,
                  int S, int d, cudaStream_t stream);
 

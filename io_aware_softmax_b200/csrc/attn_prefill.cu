@@ -48,9 +48,13 @@ constexpr int kMmaWarp = 8;
 constexpr int kTmaWarp = 9;
 constexpr int kQWarp = 10;
 // Registers per thread after the split; the launch gives 168 (65536 / 384, rounded down to
-// a multiple of 8): 2 * 128 * 192 + 128 * 112 = 63488 <= 384 * 168 = 64512.
+// a multiple of 8): 2 * 128 * 192 + 128 * 112 = 63488 <= 384 * 168 = 64512.  The soft-cap
+// variant holds its polynomial's coefficients beside the row and takes
+// 2 * 128 * 200 + 128 * 104 = 64512.
 constexpr uint32_t kRegsSoftmax = 192;
 constexpr uint32_t kRegsOther = 112;
+constexpr uint32_t kRegsSoftmaxCap = 200;
+constexpr uint32_t kRegsOtherCap = 104;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;   // log2 units: rescale when max grows > 2^8
 constexpr float kLn2 = 0.69314718055994531f;
@@ -101,37 +105,51 @@ __device__ __forceinline__ float tile_row_max(uint32_t (&s)[128], int c_lo, int 
   return max3f(m0, m1, fmaxf(m2, m3));
 }
 
-// Soft-cap path: the row maximum over the visible columns [c_lo, c_hi] (all columns when not
-// kMasked) and the largest |s| over all 128 columns, leaving s unmasked (the polynomial tanh
-// is evaluated on every column and the mask applied after it).
-template <bool kMasked>
-__device__ __forceinline__ float tile_row_max_keep(const uint32_t (&s)[128], int c_lo, int c_hi,
-                                                   float& mabs) {
-  float m0 = -INFINITY, m1 = -INFINITY, a0 = 0.f, a1 = 0.f;
+// Largest |s| of a tile row (all 128 columns; masked ones included, which only makes the
+// soft-cap path's range test stricter).
+__device__ __forceinline__ float tile_row_absmax(const uint32_t (&s)[128]) {
+  float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
 #pragma unroll
-  for (int c = 0; c < 128; c += 4) {
-    float v[4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      v[u] = f32(s[c + u]);
-      if (kMasked && (unsigned)(c + u - c_lo) > (unsigned)(c_hi - c_lo)) v[u] = -INFINITY;
-    }
-    m0 = max3f(m0, v[0], v[1]);
-    m1 = max3f(m1, v[2], v[3]);
+  for (int c = 0; c < 128; c += 8) {
     a0 = max3f(a0, fabsf(f32(s[c])), fabsf(f32(s[c + 1])));
     a1 = max3f(a1, fabsf(f32(s[c + 2])), fabsf(f32(s[c + 3])));
+    a2 = max3f(a2, fabsf(f32(s[c + 4])), fabsf(f32(s[c + 5])));
+    a3 = max3f(a3, fabsf(f32(s[c + 6])), fabsf(f32(s[c + 7])));
   }
-  mabs = fmaxf(a0, a1);
-  return fmaxf(m0, m1);
+  return fmaxf(fmaxf(a0, a1), fmaxf(a2, a3));
 }
 
-// Scaled (base-2) score of a raw score: s * scale * log2(e), or with the soft-cap
-// c * log2(e) * tanh(s * scale / c).  -inf (masked) stays -inf.
-template <bool kSoftcap>
-__device__ __forceinline__ float scaled_score(float s, const FwdParams& p) {
-  if (!kSoftcap) return s * p.kscale;
-  if (s == -INFINITY) return -INFINITY;
-  return p.cap_log2 * tanh_via_ex2(s * p.cap_scale);
+// Soft-cap, in place: every raw score of the row becomes its base-2 capped score
+// c log2(e) tanh(s scale / c).  kPoly (the row's |s scale / c| are all <= 1/2): the odd
+// polynomial s sum_i b_i s^(2i) of p.cap_poly (c log2(e) and the powers of scale / c folded
+// into the coefficients), evaluated in Estrin's scheme in paired FMAs -- depth 5 instead of
+// Horner's 6, so more of the row's independent pairs fit in the FMA pipe's latency;
+// otherwise the identity tanh(y) = 1 - 2 / (e^(2y) + 1) on ex2 and rcp.  The mask is
+// applied afterwards (the transform leaves no score at -inf).
+template <bool kPoly>
+__device__ __forceinline__ void cap_row(uint32_t (&s)[128], const FwdParams& p) {
+  if constexpr (kPoly) {
+    const float b0 = p.cap_poly[0], b1 = p.cap_poly[1], b2 = p.cap_poly[2], b3 = p.cap_poly[3],
+                b4 = p.cap_poly[4];
+#pragma unroll
+    for (int c = 0; c < 128; c += 2) {
+      const float s0 = f32(s[c]), s1 = f32(s[c + 1]);
+      float w0, w1, u0, u1, v0, v1, z0, z1;
+      fmul2(w0, w1, s0, s1, s0, s1);                   // w = s^2
+      ffma2(u0, u1, w0, w1, b1, b1, b0, b0);           // b1 w + b0
+      ffma2(v0, v1, w0, w1, b3, b3, b2, b2);           // b3 w + b2
+      fmul2(z0, z1, w0, w1, w0, w1);                   // w^2
+      ffma2(v0, v1, z0, z1, b4, b4, v0, v1);           // b4 w^2 + b3 w + b2
+      ffma2(u0, u1, v0, v1, z0, z1, u0, u1);           // ... w^2 + b1 w + b0
+      fmul2(u0, u1, u0, u1, s0, s1);
+      s[c] = __float_as_uint(u0);
+      s[c + 1] = __float_as_uint(u1);
+    }
+  } else {
+#pragma unroll
+    for (int c = 0; c < 128; ++c)
+      s[c] = __float_as_uint(p.cap_log2 * tanh_via_ex2(f32(s[c]) * p.cap_scale));
+  }
 }
 
 // Masked columns (outside [c_lo, c_hi]) of one tile row become -inf.
@@ -183,22 +201,16 @@ __device__ __forceinline__ float tile_row_exp_half_e4m3(const uint32_t (&s)[128]
   return (((a0 + a1) + (b0 + b1)) * (1.0f / 64.0f));
 }
 
-// P = 2^(x - m_use) for one 64-column half of a tile row, packed as bf16 pairs; returns
-// the half's fp32 sum (four independent packed accumulators).
-template <bool kSoftcap>
-__device__ __forceinline__ float tile_row_exp_half(const uint32_t (&s)[128], int base,
-                                                   const FwdParams& p, float ks, float m_use,
-                                                   uint32_t (&pk)[32]) {
+// P = 2^(x ks - m_use) for one 64-column half of a tile row (x the raw score, or the
+// base-2 score itself with ks = 1), packed as bf16 pairs; returns the half's fp32 sum (four
+// independent packed accumulators).
+__device__ __forceinline__ float tile_row_exp_half(const uint32_t (&s)[128], int base, float ks,
+                                                   float m_use, uint32_t (&pk)[32]) {
   float a0 = 0.f, a1 = 0.f, b0 = 0.f, b1 = 0.f, c0 = 0.f, c1 = 0.f, d0 = 0.f, d1 = 0.f;
 #pragma unroll
   for (int c = 0; c < 64; c += 2) {
     float x0, x1;
-    if (!kSoftcap) {
-      ffma2(x0, x1, f32(s[base + c]), f32(s[base + c + 1]), ks, ks, -m_use, -m_use);
-    } else {
-      x0 = scaled_score<true>(f32(s[base + c]), p) - m_use;
-      x1 = scaled_score<true>(f32(s[base + c + 1]), p) - m_use;
-    }
+    ffma2(x0, x1, f32(s[base + c]), f32(s[base + c + 1]), ks, ks, -m_use, -m_use);
     const float e0 = ex2_approx(x0);
     const float e1 = ex2_approx(x1);
     switch ((c >> 1) & 3) {
@@ -210,42 +222,6 @@ __device__ __forceinline__ float tile_row_exp_half(const uint32_t (&s)[128], int
     pk[c >> 1] = pack_bf16x2(e0, e1);
   }
   return ((a0 + a1) + (b0 + b1)) + ((c0 + c1) + (d0 + d1));
-}
-
-// Soft-capped P = 2^(c log2(e) tanh(s scale / c) - m_use) for one 64-column half of a row
-// whose raw scores all satisfy |s| <= p.cap_fast_max: tanh is the odd polynomial
-// y * sum_i a_i y^(2i) (|y| <= 1) with c log2(e) folded into p.cap_poly, evaluated in paired
-// FMAs, so the exponential is the only MUFU operation per score.  kMasked: columns outside
-// [c_lo, c_hi] get P = 0.  Returns the half's sum.
-template <bool kMasked>
-__device__ __forceinline__ float tile_row_exp_half_cap(const uint32_t (&s)[128], int base,
-                                                       const FwdParams& p, float m_use,
-                                                       uint32_t (&pk)[32], int c_lo, int c_hi) {
-  float a0 = 0.f, a1 = 0.f, b0 = 0.f, b1 = 0.f;
-  const float cs = p.cap_scale;
-#pragma unroll
-  for (int c = 0; c < 64; c += 2) {
-    float y0, y1, w0, w1;
-    fmul2(y0, y1, f32(s[base + c]), f32(s[base + c + 1]), cs, cs);
-    fmul2(w0, w1, y0, y1, y0, y1);
-    float q0 = p.cap_poly[6], q1 = p.cap_poly[6];
-#pragma unroll
-    for (int i = 5; i >= 0; --i) ffma2(q0, q1, q0, q1, w0, w1, p.cap_poly[i], p.cap_poly[i]);
-    float x0, x1;
-    ffma2(x0, x1, y0, y1, q0, q1, -m_use, -m_use);
-    if (kMasked) {
-      if ((unsigned)(base + c - c_lo) > (unsigned)(c_hi - c_lo)) x0 = -INFINITY;
-      if ((unsigned)(base + c + 1 - c_lo) > (unsigned)(c_hi - c_lo)) x1 = -INFINITY;
-    }
-    const float e0 = ex2_approx(x0);
-    const float e1 = ex2_approx(x1);
-    if ((c >> 1) & 1)
-      add2(b0, b1, e0, e1);
-    else
-      add2(a0, a1, e0, e1);
-    pk[c >> 1] = pack_bf16x2(e0, e1);
-  }
-  return (a0 + a1) + (b0 + b1);
 }
 
 // K/V tiles [a, b] (relative to the CTA's first tile) that query tile t must visit; n = 0
@@ -268,22 +244,41 @@ __device__ __forceinline__ TileRange tile_range(const FwdParams& p, int tq0, int
   return r;
 }
 
-// One query pair: rows [q_first, q_first + 256) of (b, h), the K/V tiles the pair visits,
-// [jt0, jt0 + n_tiles), and each query tile's own sub-range of them.
+// One unit of work for the CTA's two query tiles t = 0, 1: query head h[t], rows
+// [q0[t], q0[t] + 128) of batch entry b, the K/V tiles the two visit, [jt0, jt0 + n_tiles),
+// and each tile's own sub-range of them.  Two layouts:
+//   * adjacent tiles (the default): one head, rows [256 pair, 256 pair + 256);
+//   * a head pair (GQA with an even group size): query heads 2m and 2m + 1 of one KV group
+//     at the same 128 rows, so both tiles see the same keys under the same mask and every
+//     K/V tile the CTA loads feeds both.
 struct PairWork {
-  int b, h, hk, q_first, jt0, n_tiles;
+  int b, hk, h[2], q0[2], jt0, n_tiles;
   TileRange rng[2];
 };
 
 __device__ __forceinline__ PairWork make_pair_work(const FwdParams& p, int bh, int pair) {
   PairWork w;
-  w.b = bh / p.Hq;
-  w.h = bh % p.Hq;
-  w.hk = w.h / p.G;
-  w.q_first = pair * 2 * kBM;
-  const int q_last = min(w.q_first + 2 * kBM - 1, p.Nq - 1);
+  int q_first, q_span;
+  if (p.head_pairs) {
+    const int hp = p.Hq >> 1;
+    w.b = bh / hp;
+    w.h[0] = 2 * (bh % hp);
+    w.h[1] = w.h[0] + 1;
+    q_first = pair * kBM;
+    w.q0[0] = w.q0[1] = q_first;
+    q_span = kBM;
+  } else {
+    w.b = bh / p.Hq;
+    w.h[0] = w.h[1] = bh % p.Hq;
+    q_first = pair * 2 * kBM;
+    w.q0[0] = q_first;
+    w.q0[1] = q_first + kBM;
+    q_span = 2 * kBM;
+  }
+  w.hk = w.h[0] / p.G;
+  const int q_last = min(q_first + q_span - 1, p.Nq - 1);
   int lo_a, hi_a, lo_b, hi_b;
-  row_interval(p.mask, w.q_first, lo_a, hi_a);
+  row_interval(p.mask, q_first, lo_a, hi_a);
   row_interval(p.mask, q_last, lo_b, hi_b);
   w.jt0 = 0;
   w.n_tiles = 0;
@@ -291,8 +286,8 @@ __device__ __forceinline__ PairWork make_pair_work(const FwdParams& p, int bh, i
     w.jt0 = lo_a / kBN;
     w.n_tiles = hi_b / kBN - w.jt0 + 1;
   }
-  w.rng[0] = tile_range(p, w.q_first, w.jt0, w.n_tiles);
-  w.rng[1] = tile_range(p, w.q_first + kBM, w.jt0, w.n_tiles);
+  w.rng[0] = tile_range(p, w.q0[0], w.jt0, w.n_tiles);
+  w.rng[1] = tile_range(p, w.q0[1], w.jt0, w.n_tiles);
   return w;
 }
 
@@ -305,7 +300,7 @@ template <typename F>
 __device__ __forceinline__ void for_each_pair(const FwdParams& p, F&& f) {
   const int P = p.num_pairs;
   const int upb = (P + 1) / 2;
-  const long long total = (long long)p.B * p.Hq * upb;
+  const long long total = (long long)p.B * (p.head_pairs ? p.Hq / 2 : p.Hq) * upb;
   for (long long u = blockIdx.x; u < total; u += gridDim.x) {
     const int bh = (int)(u / upb);
     const int k = (int)(u % upb);
@@ -373,7 +368,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
   const uint32_t tmem = *tmem_slot;
 
   if (warp >= kMmaWarp) {
-   regs_decrease<kRegsOther>();
+   regs_decrease<kCap ? kRegsOtherCap : kRegsOther>();
    if (warp == kTmaWarp) {
     // ------------------------------------------------------------ K/V TMA producer
     if (lane == 0) {
@@ -430,7 +425,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
 #pragma unroll
           for (int c = 0; c < C::kChunks; ++c)
             tma_load_3d(sQ + t * C::kTileBytes + c * C::kChunkBytes, &tmQ, bar(BAR_Q + t),
-                        c * (128 / C::kElem), w.q_first + t * kBM, w.b * p.Hq + w.h);
+                        c * (128 / C::kElem), w.q0[t], w.b * p.Hq + w.h[t]);
           ++loads[t];
         }
         ++pairs;
@@ -577,7 +572,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
     __syncwarp();
    }
   } else {
-    regs_increase<kRegsSoftmax>();
+    regs_increase<kCap ? kRegsSoftmaxCap : kRegsSoftmax>();
     // ------------------------------------------------------------ softmax warpgroups
     const int t = warp >> 2;                 // query tile of this warpgroup
     const int wq = warp & 3;                 // TMEM lane quarter this warp may access
@@ -591,15 +586,16 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
     for_each_pair(p, [&](int bh, int pair) -> bool {
       const PairWork w = make_pair_work(p, bh, pair);
       const TileRange rng = t ? w.rng[1] : w.rng[0];
-      const int tq0 = w.q_first + t * kBM;
+      const int tq0 = w.q0[t];
+      const int head = w.h[t];
       const int row = tq0 + r;
       int row_lo, row_hi;
       row_interval(p.mask, row, row_lo, row_hi);
       // ALiBi slope of this head in base-2 units (0: no bias).
-      const float slope2 = kAlibi ? __ldg(p.alibi + w.h) * kLog2eF : 0.f;
+      const float slope2 = kAlibi ? __ldg(p.alibi + head) * kLog2eF : 0.f;
       // FP8: the block scale of this query tile; a K tile's scale joins it per tile.
       const float qs = (kFp8 && tq0 < p.Nq)
-                           ? __ldg(p.q_scales + (size_t)(w.b * p.Hq + w.h) * p.nqt + tq0 / kBM)
+                           ? __ldg(p.q_scales + (size_t)(w.b * p.Hq + head) * p.nqt + tq0 / kBM)
                            : 1.f;
       const float* ksc = kFp8 ? p.k_scales + (size_t)(w.b * p.Hkv + w.hk) * p.nkt : nullptr;
       // Tile-level bounds: a K/V tile needs no mask when every valid row of this query
@@ -625,26 +621,24 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
         const bool masked =
             !(lo_last <= k0 && k0 + kBN - 1 <= hi_first && k0 + kBN <= p.Nk);
         float mx;
-        bool cap_poly = false;   // soft-cap row small enough for the polynomial tanh
         const float ks_eff = kFp8 ? p.kscale * qs * __ldg(ksc + k0 / kBN) : p.kscale;
         if constexpr (kFp8) {
           const float mx_raw = masked ? tile_row_max<true>(s, row_lo - k0, row_hi - k0)
                                       : tile_row_max<false>(s, 0, 0);
           mx = mx_raw * ks_eff;
         } else if constexpr (kCap) {
-          // The cap is increasing, so the row max of the capped scores is the cap of the raw
-          // row max.  The polynomial tanh covers the row when its largest |s| is in range;
-          // otherwise the row takes the exact form on masked scores.
-          float mabs;
-          const float mx_raw = masked ? tile_row_max_keep<true>(s, row_lo - k0, row_hi - k0, mabs)
-                                      : tile_row_max_keep<false>(s, 0, 0, mabs);
-          cap_poly = mabs <= p.cap_fast_max;
-          if (!cap_poly && masked) mask_row(s, row_lo - k0, row_hi - k0);
-          mx = scaled_score<true>(mx_raw, p);
+          // The row's scores become base-2 capped scores in place (the polynomial tanh when
+          // the row's largest |s| is in its range), then the mask, then the row max.
+          if (tile_row_absmax(s) <= p.cap_fast_max)
+            cap_row<true>(s, p);
+          else
+            cap_row<false>(s, p);
+          if (masked) mask_row(s, row_lo - k0, row_hi - k0);
+          mx = tile_row_max<false>(s, 0, 0);
         } else if constexpr (!kAlibi) {
           const float mx_raw = masked ? tile_row_max<true>(s, row_lo - k0, row_hi - k0)
                                       : tile_row_max<false>(s, 0, 0);
-          mx = scaled_score<false>(mx_raw, p);
+          mx = mx_raw * p.kscale;
         } else {
           // The bias changes the order of the scores, so the row max is taken over the
           // biased, base-2 scores themselves.
@@ -686,17 +680,11 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
           } else {
             uint32_t pk[32];
             if constexpr (kAlibi) {
-              sum += tile_row_exp_half<false>(s, 64 * half, p, 1.f, m_use, pk);
+              sum += tile_row_exp_half(s, 64 * half, 1.f, m_use, pk);
             } else if constexpr (kCap) {
-              if (!cap_poly)
-                sum += tile_row_exp_half<true>(s, 64 * half, p, p.kscale, m_use, pk);
-              else if (masked)
-                sum += tile_row_exp_half_cap<true>(s, 64 * half, p, m_use, pk, row_lo - k0,
-                                                   row_hi - k0);
-              else
-                sum += tile_row_exp_half_cap<false>(s, 64 * half, p, m_use, pk, 0, 0);
+              sum += tile_row_exp_half(s, 64 * half, 1.f, m_use, pk);   // capped
             } else {
-              sum += tile_row_exp_half<false>(s, 64 * half, p, p.kscale, m_use, pk);
+              sum += tile_row_exp_half(s, 64 * half, p.kscale, m_use, pk);
             }
             tmem_st_x32(tP + 32u * half, pk);
           }
@@ -721,7 +709,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
       const float o_mul = kFp8 ? __ldg(p.v_scales + w.b * p.Hkv + w.hk) / kPScale : 1.f;
       const float inv_l = (l > 0.f) ? o_mul / l : 0.f;
       const float lse = (l > 0.f) ? (m_ref + log2f(l)) * kLn2 : -INFINITY;
-      const size_t row_index = (size_t)(w.b * p.Hq + w.h) * (size_t)p.Nq + (size_t)row;
+      const size_t row_index = (size_t)(w.b * p.Hq + head) * (size_t)p.Nq + (size_t)row;
       __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(p.o) + row_index * D;
 #pragma unroll
       for (int cc = 0; cc < D / 32; ++cc) {
@@ -769,7 +757,8 @@ int launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& 
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        C::kSmemBytes);
   if (e != cudaSuccess) return -4;
-  const long long units = (long long)((p.num_pairs + 1) / 2) * p.B * p.Hq;
+  const long long units =
+      (long long)((p.num_pairs + 1) / 2) * p.B * (p.head_pairs ? p.Hq / 2 : p.Hq);
   const long long grid = units < p.num_sms ? units : p.num_sms;
   attn_fwd_sm100_kernel<D, kAlibi, kFp8, kCap>
       <<<(unsigned)grid, kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, p);

@@ -8,7 +8,7 @@ import torch
 import oracle
 import workloads
 from io_aware_softmax_b200 import attn_fwd, device_status
-from tests.gpu_common import compare, f64, sample_rows
+from tests.gpu_common import BF16_UNIT_ROUNDOFF, compare, f64, sample_rows
 
 pytestmark = pytest.mark.gpu
 
@@ -37,11 +37,17 @@ def _run_full(B, Hq, Hkv, Nq, Nk, d, mask="none", window=0, softcap=0.0, docs=No
              alibi_slopes=slopes_t, out=o, lse=lse)
     assert device_status() == 0
     assert torch.isnan(o_buf[B * Hq * Nq * d:]).all() and torch.isnan(l_buf[B * Hq * Nq:]).all()
-    O_ref, L_ref = oracle.attention(f64(q), f64(k), f64(v), scale=scale, mask_kind=MASK_ID[mask],
-                                    window=window, softcap=softcap, doc_offsets=docs,
-                                    alibi_slopes=slopes)
+    kw = dict(scale=scale, mask_kind=MASK_ID[mask], window=window, softcap=softcap,
+              doc_offsets=docs, alibi_slopes=slopes)
+    O_ref, L_ref = oracle.attention(f64(q), f64(k), f64(v), **kw)
+    bound = None
+    if v_std > 1.0:
+        # wide V: the derived per-element bound of bf16 rounding (see gpu_common)
+        PV_abs, _ = oracle.attention(f64(q), f64(k), np.abs(f64(v)), **kw)
+        bound = BF16_UNIT_ROUNDOFF * (np.abs(O_ref) + PV_abs)
     return compare(o, lse, O_ref, L_ref,
-                   f"{B}x{Hq}/{Hkv}x{Nq}x{Nk}x{d} {mask} w{window} c{softcap} alibi{slopes}")
+                   f"{B}x{Hq}/{Hkv}x{Nq}x{Nk}x{d} {mask} w{window} c{softcap} alibi{slopes}",
+                   o_bound=bound)
 
 
 def test_tiny_workload_noncausal_and_causal():
@@ -64,9 +70,17 @@ def test_ragged_lengths(d, N, mask):
     _run_full(1, 2, 2, N, N, d, mask=mask, seed=N)
 
 
-@pytest.mark.parametrize("Hq,Hkv", [(4, 1), (8, 2), (6, 3)])
+@pytest.mark.parametrize("Hq,Hkv", [(4, 1), (8, 2), (6, 3), (2, 1), (9, 3), (3, 1)])
 def test_gqa_mqa_head_mapping(Hq, Hkv):
+    # even groups run two query heads of a KV group side by side, odd ones two row tiles
     _run_full(2, Hq, Hkv, 300, 300, 128, mask="causal", seed=Hq * 10 + Hkv)
+
+
+@pytest.mark.parametrize("mask,window,docs,d", [
+    ("sliding_causal", 200, None, 128), ("document_causal", 0, [0, 130, 131, 500, 777], 128),
+    ("none", 0, None, 64), ("sliding", 90, None, 64)])
+def test_gqa_head_pairs_under_every_mask(mask, window, docs, d):
+    _run_full(2, 8, 2, 777, 777, d, mask=mask, window=window, docs=docs, seed=window + d)
 
 
 @pytest.mark.parametrize("window", [0, 1, 100, 127, 128, 129, 255, 600])
