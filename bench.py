@@ -10,9 +10,10 @@ d=128): KV-cache GB/s and tokens/s of one ``attn_decode_splitkv`` call (split + 
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-Multi-GPU: one process per GPU (torchrun); every rank runs the same workload on its own GPU
-(independent replicas of (batch, head) units, no collective on the data path); the value is
-all ranks' work divided by the slowest rank's device time.
+Multi-GPU: one process per GPU (torchrun); the (batch, head) units are independent, so each
+rank runs its own slice of every workload -- whole batch entries, or whole KV-head groups
+when the batch does not divide -- with no collective on the data path; the value is all
+ranks' work divided by the slowest rank's device time.
 """
 from __future__ import annotations
 
@@ -180,8 +181,25 @@ def max_over_ranks(world, x: float) -> float:
 
 
 def whole_job_rate(units_per_rank: float, world: int, ms_max: float) -> float:
-    """Weak scaling of independent replicas: all ranks' units over the slowest rank's time."""
+    """All ranks' units over the slowest rank's time (every rank runs an equal part)."""
     return units_per_rank * world / (ms_max * 1e-3)
+
+
+def my_part(w: workloads.Workload, world: int) -> workloads.Workload:
+    """This rank's part of a workload: its own batch entries or KV-head groups (no exchange
+    between ranks), or the whole workload when neither divides evenly."""
+    return workloads.rank_part(w, world, int(os.environ.get("RANK", "0")))
+
+
+def split_note(w_full: workloads.Workload, w: workloads.Workload, world: int) -> str:
+    if world == 1:
+        return "1 GPU, the whole workload"
+    if w.B != w_full.B:
+        return f"{world} ranks, each its own {w.B} of the {w_full.B} batch entries, no collective"
+    if w.Hkv != w_full.Hkv:
+        return (f"{world} ranks, each its own {w.Hkv} of the {w_full.Hkv} KV heads (with their "
+                f"query heads), no collective")
+    return f"{world} replicas of the whole workload (B and Hkv not divisible), no collective"
 
 
 # ----------------------------------------------------------------------- CPU baseline
@@ -284,7 +302,8 @@ def run_ours(args, world, rank, local):
         # one prefill workload alone (profiler captures of a single kernel)
         return bench_prefill_variant(workloads.BY_NAME[args.workload], args, world, local,
                                      peaks, peak_src, steps=args.steps)
-    w = workloads.CAUSAL_MHA
+    w_full = workloads.CAUSAL_MHA
+    w = my_part(w_full, world)
     dev = torch.device("cuda", torch.cuda.current_device())
     q, k, v = workloads.make_inputs(w, device=dev)
     o = torch.empty_like(q)
@@ -311,14 +330,15 @@ def run_ours(args, world, rank, local):
     out = {
         "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic",
-        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.Nq, "d": w.d,
-                   "mask": "causal", "useful_tflop_per_step": round(flops / 1e12, 4),
-                   "executed_tflop_per_step": round(executed / 1e12, 4),
-                   "l2": "inputs larger than L2 (q+k+v %.0f MB > 126 MB)" %
+        "higher_is_better": True, "scaling": "strong" if w is not w_full or world == 1 else "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "B": w_full.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.Nq,
+                   "d": w.d, "mask": "causal",
+                   "useful_tflop_per_step": round(flops * world / 1e12, 4),
+                   "executed_tflop_per_step": round(executed * world / 1e12, 4),
+                   "l2": "inputs larger than L2 (q+k+v %.0f MB > 126 MB per GPU)" %
                          (3 * q.numel() * 2 / 1e6),
-                   "parallelism": f"replicas x{world} (independent (batch, head) units)",
+                   "parallelism": split_note(w_full, w, world),
                    "seed": w.seed},
         "roofline": prefill_roofline(flops, executed, kernel_ms, peaks, peak_src, clocks,
                                      "attn_fwd_sm100_kernel<128>",
@@ -458,15 +478,15 @@ def bench_extras(args, world, local, peaks, peak_src):
     return ex
 
 
-def decode_workload(args):
-    """The decode workload, with the batch overridden by --decode-batch (smaller caches for
-    profiler captures)."""
+def decode_workload(args, world: int = 1):
+    """This rank's part of the decode workload, with the batch overridden by --decode-batch
+    (smaller caches for profiler captures)."""
     import dataclasses
     w = workloads.DECODE
     if args.decode_batch:
         w = dataclasses.replace(w, B=args.decode_batch, name=w.name.replace(
             f"b{w.B}_", f"b{args.decode_batch}_"))
-    return w
+    return my_part(w, world)
 
 
 def tensor_peak_at_clock(sm_mhz, n_sms: int) -> float | None:
@@ -499,11 +519,12 @@ def bench_prefill_variant(w, args, world, local, peaks, peak_src, steps=None):
     the headline, fewer steps."""
     import torch
     import io_aware_softmax_b200 as attn
+    w_full, w = w, my_part(w, world)
     dev = torch.device("cuda", torch.cuda.current_device())
     q, k, v = workloads.make_inputs(w, device=dev)
     o = torch.empty_like(q)
     lse = torch.empty((w.B, w.Hq, w.Nq), dtype=torch.float32, device=dev)
-    slopes = (torch.tensor(workloads.alibi_slopes(w.Hq), dtype=torch.float32, device=dev)
+    slopes = (torch.tensor(workloads.workload_alibi_slopes(w), dtype=torch.float32, device=dev)
               if w.alibi else None)
     docs = workloads.workload_doc_offsets(w)
     doc_t = None if docs is None else torch.from_numpy(docs).to(dev)
@@ -528,7 +549,7 @@ def bench_prefill_variant(w, args, world, local, peaks, peak_src, steps=None):
     kernel_ms = max_over_ranks(world, sum(per) / len(per))
     clocks = clk.summary()
     kernel = "attn_fwd_sm100_kernel<%d>%s" % (w.d, " (ALiBi)" if w.alibi else "")
-    cfg = {**w.describe(), "l2": l2_note(q, k, v)}
+    cfg = {**w.describe(), "l2": l2_note(q, k, v), "parallelism": split_note(w_full, w, world)}
     if docs is not None:
         cfg["num_docs"] = len(docs) - 1
     res = {"config": cfg,
@@ -550,7 +571,7 @@ def bench_decode_paged(args, world, local, peaks, peak_src, page: int = 256):
     every sequence at full length (the same KV bytes as the contiguous line)."""
     import torch
     import io_aware_softmax_b200 as attn
-    w = decode_workload(args)
+    w = decode_workload(args, world)
     dev = torch.device("cuda", torch.cuda.current_device())
     max_pages = w.Nk // page
     num_pages = w.B * max_pages
@@ -606,10 +627,11 @@ def bench_backward(w, args, world, local, peaks, peak_src):
     (attn_bwd_alibi when the workload carries ALiBi slopes; its documents and soft-cap too)."""
     import torch
     import io_aware_softmax_b200 as attn
+    w = my_part(w, world)
     dev = torch.device("cuda", torch.cuda.current_device())
     q, k, v = workloads.make_inputs(w, device=dev)
-    dout = workloads.randn_bf16((w.B, w.Hq, w.Nq, w.d), w.seed, 3, 1.0, dev)
-    slopes = (torch.tensor(workloads.alibi_slopes(w.Hq), dtype=torch.float32, device=dev)
+    dout = workloads.randn_bf16((w.B, w.Hq, w.Nq, w.d), w.seed, 3, 1.0, dev, w.b0)
+    slopes = (torch.tensor(workloads.workload_alibi_slopes(w), dtype=torch.float32, device=dev)
               if w.alibi else None)
     docs = workloads.workload_doc_offsets(w)
     doc_t = None if docs is None else torch.tensor(docs, dtype=torch.int32, device=dev)
@@ -662,6 +684,7 @@ def bench_fp8(w, args, world, local, peaks, peak_src):
     quantization runs before the timed region and is timed on its own."""
     import torch
     import io_aware_softmax_b200 as attn
+    w = my_part(w, world)
     dev = torch.device("cuda", torch.cuda.current_device())
     q, k, v = workloads.make_inputs(w, device=dev)
     signs = torch.from_numpy(np.random.default_rng(w.seed).choice([-1.0, 1.0], w.d)
@@ -803,7 +826,7 @@ def e2e_prefill(w, args, world, q, k, v):
 def bench_decode(args, world, local, peaks, peak_src):
     import torch
     import io_aware_softmax_b200 as attn
-    w = decode_workload(args)
+    w = decode_workload(args, world)
     dev = torch.device("cuda", torch.cuda.current_device())
     q, kc, vc = workloads.make_inputs(w, device=dev)
     S = attn.default_splits(w.B, w.Hkv, w.Nk, dev.index)

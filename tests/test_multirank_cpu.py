@@ -1,9 +1,11 @@
 """The N > 1 plumbing of bench.py on CPU: two gloo ranks on 127.0.0.1.
 
-The path shards into independent (batch, head) units, so N GPUs run N replicas with no
-collective on the data path; the only cross-rank steps are the barriers around the timed
+The path shards into independent (batch, head) units, so each of N GPUs runs its own slice
+of them (whole batch entries, or whole KV-head groups when the batch does not divide) with
+no collective on the data path; the only cross-rank steps are the barriers around the timed
 region and the max over ranks of the device times.  These tests run those steps as two
-processes with the gloo backend."""
+processes with the gloo backend, and check that the ranks' slices tile every workload and
+hold the whole workload's input numbers."""
 import io
 import os
 import socket
@@ -34,9 +36,21 @@ def _rank_main(rank, world, port, queue):
     # each rank reports its own time; every rank must see the slowest one
     slowest = bench.max_over_ranks(w, 1.5 + rank)
     rate = bench.whole_job_rate(1e12, w, slowest)
+    # this rank's slice of every workload, as bench.py takes it
+    import workloads
+    parts = {}
+    for wl in workloads.ALL:
+        p = bench.my_part(wl, w)
+        parts[wl.name] = (p.b0, p.B, p.hk0, p.Hkv, p.Hq)
+    # and the input numbers of a small GQA workload's slice (B = 1: split by KV heads)
+    import dataclasses
+    small = dataclasses.replace(workloads.SWA_GQA, B=1, Nq=16, Nk=16, d=64)
+    q, k, v = workloads.make_inputs(bench.my_part(small, w))
     bench.barrier(w)
     dist.destroy_process_group()
-    queue.put((rank, slowest, rate))
+    # plain arrays (bf16 -> float32 is exact): tensors would be shared with the parent through
+    # this process's memory, which is gone once it exits
+    queue.put((rank, slowest, rate, parts, tuple(t.float().numpy() for t in (q, k, v))))
 
 
 def _run_two_ranks(world):
@@ -48,14 +62,21 @@ def _run_two_ranks(world):
     procs = [ctx.Process(target=_rank_main, args=(r, world, port, q)) for r in range(world)]
     for p in procs:
         p.start()
+    # read the results before joining: a child cannot exit while its queue data is unread
+    res = []
+    try:
+        for _ in range(world):
+            res.append(q.get(timeout=120))
+    except Exception:
+        res = None
     for p in procs:
-        p.join(timeout=120)
-    if any(p.exitcode != 0 for p in procs):
+        p.join(timeout=60)
+    if res is None or any(p.exitcode != 0 for p in procs):
         for p in procs:
             if p.is_alive():
                 p.kill()
         return None
-    return sorted(q.get(timeout=10) for _ in range(world))
+    return sorted(res, key=lambda r: r[0])
 
 
 def test_two_gloo_ranks_take_the_max_and_aggregate():
@@ -66,10 +87,30 @@ def test_two_gloo_ranks_take_the_max_and_aggregate():
         if res is not None:
             break
     assert res is not None, "the two gloo ranks failed three times"
-    for rank, slowest, rate in res:
+    for rank, slowest, rate, _, _ in res:
         assert slowest == pytest.approx(1.5 + world - 1)
         # 1e12 units per rank, 2 ranks, slowest 2.5 ms -> 8e14 units/s for the whole job
         assert rate == pytest.approx(1e12 * world / 2.5e-3)
+    import torch
+    import workloads
+    for wl in workloads.ALL:
+        got = [parts[wl.name] for _, _, _, parts, _ in res]
+        if wl.B % world == 0:
+            # whole batch entries: consecutive, disjoint, covering [0, B), all heads each
+            assert [g[0] for g in got] == [r * wl.B // world for r in range(world)]
+            assert all(g[1] == wl.B // world and g[3] == wl.Hkv for g in got)
+        else:
+            # whole KV-head groups with their query heads, covering [0, Hkv)
+            assert wl.Hkv % world == 0
+            assert [g[2] for g in got] == [r * wl.Hkv // world for r in range(world)]
+            assert all(g[1] == wl.B and g[3] == wl.Hkv // world and
+                       g[4] == wl.Hq // world for g in got)
+    import dataclasses
+    small = dataclasses.replace(workloads.SWA_GQA, B=1, Nq=16, Nk=16, d=64)
+    full = workloads.make_inputs(small)
+    for i in range(3):
+        got = torch.cat([torch.from_numpy(r[4][i]) for r in res], dim=1)
+        assert torch.equal(got, full[i].float())
 
 
 def _reference_rank(rank, world, queue):

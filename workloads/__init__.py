@@ -43,6 +43,12 @@ class Workload:
     doc_seed: int = 0
     alibi: bool = False       # geometric ALiBi slopes 2^(-8 (h + 1) / Hq)
     seed: int = 0
+    # One rank's part of a workload split over several GPUs (see rank_part): batch entries
+    # [b0, b0 + B) and KV heads [hk0, hk0 + Hkv) of a workload with full_Hkv KV heads
+    # (0: all of them).  The inputs are the same numbers the whole workload draws there.
+    b0: int = 0
+    hk0: int = 0
+    full_Hkv: int = 0
 
     @property
     def scale(self) -> float:
@@ -62,6 +68,9 @@ class Workload:
             out["doc_seed"] = self.doc_seed
         out["input_std"] = self.input_std
         out["seed"] = self.seed
+        if self.b0 or self.hk0 or self.full_Hkv:
+            out["part"] = {"batch": [self.b0, self.b0 + self.B],
+                           "kv_heads": [self.hk0, self.hk0 + self.Hkv]}
         return out
 
 
@@ -92,6 +101,13 @@ SWA_SYM_GQA = dataclasses.replace(SWA_GQA, name="swa_sym_gqa_b4_hq32_hkv8_n16384
 def alibi_slopes(H: int):
     """The geometric ALiBi slopes 2^(-8 (h + 1) / H), one per query head."""
     return [2.0 ** (-8.0 * (h + 1) / H) for h in range(H)]
+
+
+def workload_alibi_slopes(w: "Workload"):
+    """The slopes of the query heads ``w`` holds (a rank's part keeps the whole workload's)."""
+    G = w.Hq // w.Hkv
+    full = alibi_slopes((w.full_Hkv or w.Hkv) * G)
+    return full[w.hk0 * G:w.hk0 * G + w.Hq]
 
 ALL = [TINY, TINY_CAUSAL, CAUSAL_MHA, SWA_GQA, DOC_SOFTCAP, DECODE, ALIBI_MHA, SWA_SYM_GQA]
 BY_NAME = {w.name: w for w in ALL}
@@ -127,19 +143,20 @@ def _tensor_seed(seed: int, tensor_id: int, b: int) -> int:
     return ((seed * 16 + tensor_id) * 65536 + b) & 0x7FFFFFFFFFFFFFFF
 
 
-def randn_bf16(shape, seed: int, tensor_id: int, std: float = 1.0, device="cpu"):
+def randn_bf16(shape, seed: int, tensor_id: int, std: float = 1.0, device="cpu", b0: int = 0):
     """bf16 tensor of i.i.d. N(0, std^2) draws: fp32 normal draws from a torch generator
     seeded per (seed, tensor, leading index), times ``std``, rounded to bf16 (RNE).
 
     The bits depend on ``device`` (CPU and CUDA generators differ) but are reproducible
     for a given device.  Drawing one leading slice at a time keeps the fp32 temporary
-    small for multi-GiB caches."""
+    small for multi-GiB caches.  ``b0`` draws leading slices b0, b0 + 1, ... (one rank's
+    batch entries of a larger tensor)."""
     import torch
 
     out = torch.empty(tuple(shape), dtype=torch.bfloat16, device=device)
     g = torch.Generator(device=device)
     for b in range(shape[0]):
-        g.manual_seed(_tensor_seed(seed, tensor_id, b))
+        g.manual_seed(_tensor_seed(seed, tensor_id, b0 + b))
         x = torch.randn(tuple(shape[1:]), generator=g, dtype=torch.float32, device=device)
         if std != 1.0:
             x.mul_(std)
@@ -149,8 +166,32 @@ def randn_bf16(shape, seed: int, tensor_id: int, std: float = 1.0, device="cpu")
 
 
 def make_inputs(w: Workload, device="cpu"):
-    """(q, k, v) bf16 tensors of workload ``w``: q [B,Hq,Nq,d], k/v [B,Hkv,Nk,d]."""
-    q = randn_bf16((w.B, w.Hq, w.Nq, w.d), w.seed, 0, w.input_std, device)
-    k = randn_bf16((w.B, w.Hkv, w.Nk, w.d), w.seed, 1, w.input_std, device)
-    v = randn_bf16((w.B, w.Hkv, w.Nk, w.d), w.seed, 2, w.input_std, device)
+    """(q, k, v) bf16 tensors of workload ``w``: q [B,Hq,Nq,d], k/v [B,Hkv,Nk,d].  For a
+    rank's part, the part's slices of the whole workload's tensors."""
+    G = w.Hq // w.Hkv if w.Hkv else 1
+    hkv = w.full_Hkv or w.Hkv
+    q = randn_bf16((w.B, hkv * G, w.Nq, w.d), w.seed, 0, w.input_std, device, w.b0)
+    k = randn_bf16((w.B, hkv, w.Nk, w.d), w.seed, 1, w.input_std, device, w.b0)
+    v = randn_bf16((w.B, hkv, w.Nk, w.d), w.seed, 2, w.input_std, device, w.b0)
+    if hkv != w.Hkv:
+        q = q[:, w.hk0 * G:(w.hk0 + w.Hkv) * G].contiguous()
+        k = k[:, w.hk0:w.hk0 + w.Hkv].contiguous()
+        v = v[:, w.hk0:w.hk0 + w.Hkv].contiguous()
     return q, k, v
+
+
+def rank_part(w: Workload, world: int, rank: int) -> Workload:
+    """The part of ``w`` that rank ``rank`` of ``world`` GPUs runs.  (batch, head) units are
+    independent, so the ranks split them with no exchange: whole batch entries when
+    ``world`` divides B, else whole KV-head groups (their query heads with them) when it
+    divides Hkv; if neither, every rank runs the whole workload (replicas)."""
+    if world <= 1:
+        return w
+    if w.B % world == 0:
+        n = w.B // world
+        return dataclasses.replace(w, B=n, b0=rank * n, full_Hkv=w.Hkv)
+    if w.Hkv % world == 0:
+        n = w.Hkv // world
+        G = w.Hq // w.Hkv
+        return dataclasses.replace(w, Hq=n * G, Hkv=n, hk0=rank * n, full_Hkv=w.Hkv)
+    return w
