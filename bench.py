@@ -466,15 +466,24 @@ def l2_note(*tensors) -> str:
 
 def bench_extras(args, world, local, peaks, peak_src):
     """The rows beyond the headline: ALiBi and symmetric-window prefill, paged decode, the
-    backward pass and the FP8 prefill, one line each."""
-    ex = {x.name: bench_prefill_variant(x, args, world, local, peaks, peak_src)
-          for x in (workloads.ALIBI_MHA, workloads.SWA_SYM_GQA)}
-    paged = bench_decode_paged(args, world, local, peaks, peak_src)
-    ex["paged_" + paged["config"]["workload"]] = paged
-    for x in (workloads.CAUSAL_MHA, workloads.ALIBI_MHA, workloads.DOC_SOFTCAP):
-        ex["backward_" + x.name] = bench_backward(x, args, world, local, peaks, peak_src)
-    ex["fp8_" + workloads.CAUSAL_MHA.name] = bench_fp8(
-        workloads.CAUSAL_MHA, args, world, local, peaks, peak_src)
+    backward pass and the FP8 prefill, one line each (--extra picks one group of them)."""
+    pick = getattr(args, "extra", None)
+    ex = {}
+    if pick in (None, "alibi"):
+        ex[workloads.ALIBI_MHA.name] = bench_prefill_variant(workloads.ALIBI_MHA, args, world,
+                                                             local, peaks, peak_src)
+    if pick in (None, "sym"):
+        ex[workloads.SWA_SYM_GQA.name] = bench_prefill_variant(workloads.SWA_SYM_GQA, args,
+                                                               world, local, peaks, peak_src)
+    if pick in (None, "paged"):
+        paged = bench_decode_paged(args, world, local, peaks, peak_src)
+        ex["paged_" + paged["config"]["workload"]] = paged
+    if pick in (None, "backward"):
+        for x in (workloads.CAUSAL_MHA, workloads.ALIBI_MHA, workloads.DOC_SOFTCAP):
+            ex["backward_" + x.name] = bench_backward(x, args, world, local, peaks, peak_src)
+    if pick in (None, "fp8"):
+        ex["fp8_" + workloads.CAUSAL_MHA.name] = bench_fp8(
+            workloads.CAUSAL_MHA, args, world, local, peaks, peak_src)
     return ex
 
 
@@ -943,6 +952,8 @@ def main(argv=None):
     ap.add_argument("--workload", choices=sorted(n for n, x in workloads.BY_NAME.items()
                                                  if x.kind == "prefill"), default=None,
                     help="time attn_fwd on this prefill workload only (profiling runs)")
+    ap.add_argument("--extra", choices=["alibi", "sym", "paged", "backward", "fp8"],
+                    default=None, help="with --only extras: that line alone (profiling runs)")
     ap.add_argument("--decode-batch", type=int, default=None,
                     help="decode batch size override (smaller caches for ncu captures)")
     args = ap.parse_args(argv)
