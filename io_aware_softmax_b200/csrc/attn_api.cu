@@ -193,6 +193,14 @@ extern "C" int attn_fwd_alibi(const void* q, const void* k, const void* v, void*
   p.head_pairs = (p.G % 2 == 0) ? 1 : 0;
   p.num_pairs = p.head_pairs ? (Nq + 127) / 128 : (Nq + 255) / 256;
   p.num_sms = sm_count(current_device());
+  // Packed documents: a unit's cost follows the document layout, so the units are dealt by
+  // cost (sorted in every CTA) when they are few enough to sort in shared memory.
+  p.sched = 0;
+  if (mask_kind == ATTN_MASK_DOCUMENT_CAUSAL) {
+    const long long U = (long long)p.num_pairs * B * (p.head_pairs ? Hq / 2 : Hq);
+    const long long G = std::min<long long>(U, p.num_sms);
+    if (U <= kSchedUnits && (U + G - 1) / G + 1 <= kSchedMax) p.sched = 1;
+  }
   p.kscale = scale * kLog2e;
   p.softcap = softcap > 0.f ? softcap : 0.f;
   p.cap_scale = softcap > 0.f ? scale / softcap : 0.f;

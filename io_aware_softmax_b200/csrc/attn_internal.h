@@ -10,6 +10,11 @@
 
 namespace attn {
 
+// Cost-ordered scheduling of the prefill (FwdParams::sched): at most kSchedUnits work units
+// in all (their sort keys fill 16 KB of the K/V ring before it is used) and kSchedMax per CTA.
+constexpr int kSchedUnits = 4096;
+constexpr int kSchedMax = 63;
+
 struct FwdParams {
   void* o;            // bf16 [B, Hq, Nq, d]
   float* lse;         // fp32 [B, Hq, Nq]
@@ -18,6 +23,7 @@ struct FwdParams {
   int num_pairs;      // work units per (b, h) [adjacent tiles: ceil(Nq / 256)] or per
                       // (b, head pair) [head pairs: ceil(Nq / 128)]
   int head_pairs;     // 1: a CTA's two query tiles are query heads 2m, 2m + 1 at the same rows
+  int sched;          // 1: units dealt by cost (sorted, snake) instead of in index order
   int num_sms;        // persistent grid size (SMs of the device)
   float kscale;       // scale * log2(e)
   float softcap;      // > 0: soft-cap enabled

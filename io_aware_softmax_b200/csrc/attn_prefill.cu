@@ -73,7 +73,10 @@ struct Cfg {
   static constexpr int kBarOff = kRingOff + kStages * kTileBytes;
   // barriers: q[2], q_free[2], full[S], empty[S], s[2], p[2][2 key halves], o[2], done
   static constexpr int kNumBars = 13 + 2 * kStages;
-  static constexpr int kSmemBytes = kBarOff + kNumBars * 8 + 16 + 1024;
+  // after the barriers: TMEM slot, abort flag and wait limit (16 bytes), then this CTA's
+  // work list when the grid is scheduled by cost (count + up to kSchedMax unit indices)
+  static constexpr int kSchedOff = kBarOff + kNumBars * 8 + 16;
+  static constexpr int kSmemBytes = kSchedOff + 4 * (1 + kSchedMax) + 1024;
 };
 
 enum : uint32_t {
@@ -297,8 +300,17 @@ __device__ __forceinline__ PairWork make_pair_work(const FwdParams& p, int bh, i
 // balances the work, and consecutive units share a head, so the K/V tiles of the heads in
 // flight stay in L2.  f returns false to stop (abort).
 template <typename F>
-__device__ __forceinline__ void for_each_pair(const FwdParams& p, F&& f) {
+__device__ __forceinline__ void for_each_pair(const FwdParams& p, const int* sched, F&& f) {
   const int P = p.num_pairs;
+  if (p.sched) {
+    // the CTA's own list, built at kernel start (build_schedule): one query pair per entry
+    const int n = sched[0];
+    for (int i = 0; i < n; ++i) {
+      const int u = sched[1 + i];
+      if (!f(u / P, u % P)) return;
+    }
+    return;
+  }
   const int upb = (P + 1) / 2;
   const long long total = (long long)p.B * (p.head_pairs ? p.Hq / 2 : p.Hq) * upb;
   for (long long u = blockIdx.x; u < total; u += gridDim.x) {
@@ -307,6 +319,58 @@ __device__ __forceinline__ void for_each_pair(const FwdParams& p, F&& f) {
     if (!f(bh, P - 1 - k)) return;
     if (k != P - 1 - k && !f(bh, k)) return;
   }
+}
+
+// Cost-ordered deal of the work units (one query pair or head pair each) for masks under
+// which the units' costs follow the data (packed documents).  Every CTA computes the same
+// thing: the cost of every unit (the K/V tiles it visits, plus one for its fill and
+// epilogue), a sort by descending cost (ties by index, so the order is the same in every
+// CTA), and a snake deal of the sorted units -- CTA c takes sorted positions c and
+// 2 G - 1 - c of every 2 G, G the grid -- which gives each CTA one of the heaviest and one of
+// the lightest of each round (within 2 % of the longest-first greedy deal on the packed-
+// document workload, against 20 % above the mean for dealing in index order).  keys is
+// scratch shared memory for the sort; the CTA's list goes to sched[0] (count), sched[1..].
+__device__ __forceinline__ void build_schedule(const FwdParams& p, uint32_t* keys, int* sched) {
+  const int P = p.num_pairs;
+  const int U = p.B * (p.head_pairs ? p.Hq / 2 : p.Hq) * P;
+  int Up = 1;
+  while (Up < U) Up <<= 1;
+  for (int u = threadIdx.x; u < Up; u += kThreads) {
+    uint32_t key = 0xffffffffu;
+    if (u < U) {
+      const PairWork w = make_pair_work(p, u / P, u % P);
+      key = ((uint32_t)(0xffff - min(w.n_tiles + 1, 0xffff)) << 16) | (uint32_t)u;
+    }
+    keys[u] = key;
+  }
+  __syncthreads();
+  // bitonic sort, ascending keys = descending cost, then ascending unit index
+  for (int k = 2; k <= Up; k <<= 1)
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      for (int i = threadIdx.x; i < Up; i += kThreads) {
+        const int ixj = i ^ j;
+        if (ixj > i) {
+          const uint32_t a = keys[i], b = keys[ixj];
+          if ((a > b) == ((i & k) == 0)) {
+            keys[i] = b;
+            keys[ixj] = a;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  const int G = (int)gridDim.x, c = (int)blockIdx.x, G2 = 2 * G;
+  for (int r = threadIdx.x; r < U; r += kThreads) {
+    const int m = r % G2;
+    if (m == c || m == G2 - 1 - c) sched[1 + 2 * (r / G2) + (m >= G ? 1 : 0)] = (int)(keys[r] & 0xffffu);
+  }
+  if (threadIdx.x == 0) {
+    const int rem = U % G2;
+    sched[0] = 2 * (U / G2) + (rem > c ? 1 : 0) + (rem > G2 - 1 - c ? 1 : 0);
+  }
+  // the K/V ring's copies will overwrite the keys through the async proxy
+  fence_proxy_async_smem();
+  __syncthreads();
 }
 
 template <int D, bool kAlibi, bool kFp8, bool kCap>
@@ -366,6 +430,8 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  int* sched = reinterpret_cast<int*>(base + C::kSchedOff);
+  if (p.sched) build_schedule(p, reinterpret_cast<uint32_t*>(base + C::kRingOff), sched);
 
   if (warp >= kMmaWarp) {
    regs_decrease<kCap ? kRegsOtherCap : kRegsOther>();
@@ -375,7 +441,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
       int issued = 0;          // ring loads issued so far, across all pairs
-      for_each_pair(p, [&](int bh, int pair) -> bool {
+      for_each_pair(p, sched, [&](int bh, int pair) -> bool {
         const PairWork w = make_pair_work(p, bh, pair);
         const int zkv = w.b * p.Hkv + w.hk;
         for (int i = 0; i < 2 * w.n_tiles; ++i) {
@@ -415,7 +481,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
       tma_prefetch_desc(&tmQ);
       int pairs = 0;
       int loads[2] = {0, 0};   // Q loads issued per query tile (they differ after an abort)
-      for_each_pair(p, [&](int bh, int pair) -> bool {
+      for_each_pair(p, sched, [&](int bh, int pair) -> bool {
         const PairWork w = make_pair_work(p, bh, pair);
         for (int t = 0; t < 2; ++t) {
           if (pairs > 0 &&
@@ -510,7 +576,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
         if (jv == rg.b) umma_commit_warp(bar(BAR_O + t));
         return true;
       };
-      for_each_pair(p, [&](int bh, int pair) -> bool {
+      for_each_pair(p, sched, [&](int bh, int pair) -> bool {
         const PairWork w = make_pair_work(p, bh, pair);
         const TileRange r0 = w.rng[0], r1 = w.rng[1];
         if (!mbar_wait_warp(bar(BAR_Q + 0), pairs & 1, abort_flag, p.err, kSiteQ)) return ok = false;
@@ -583,7 +649,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
     const uint32_t tO = tmem + lane_off + 256u + 128u * t;
     int scount = 0, ocount = 0;
 
-    for_each_pair(p, [&](int bh, int pair) -> bool {
+    for_each_pair(p, sched, [&](int bh, int pair) -> bool {
       const PairWork w = make_pair_work(p, bh, pair);
       const TileRange rng = t ? w.rng[1] : w.rng[0];
       const int tq0 = w.q0[t];
@@ -757,8 +823,8 @@ int launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& 
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        C::kSmemBytes);
   if (e != cudaSuccess) return -4;
-  const long long units =
-      (long long)((p.num_pairs + 1) / 2) * p.B * (p.head_pairs ? p.Hq / 2 : p.Hq);
+  const long long per_head = p.sched ? p.num_pairs : (p.num_pairs + 1) / 2;
+  const long long units = per_head * p.B * (p.head_pairs ? p.Hq / 2 : p.Hq);
   const long long grid = units < p.num_sms ? units : p.num_sms;
   attn_fwd_sm100_kernel<D, kAlibi, kFp8, kCap>
       <<<(unsigned)grid, kThreads, C::kSmemBytes, stream>>>(tq, tk, tv, p);
