@@ -542,8 +542,13 @@ extern "C" int attn_quantize_fp8(const void* x, void* out, float* scales, int B,
   if (!transpose && (reinterpret_cast<uintptr_t>(out) & 3u)) return ATTN_ERR_MISALIGNED;
   uint32_t* err = error_word_ptr(current_device());
   if (err == nullptr) return ATTN_ERR_CUDA;
-  return launch_quantize_e4m3(x, out, scales, B, H, N, d, block_rows, transpose, n_pad, signs,
-                              err, sm_count(current_device()), stream) == 0
+  // row-major blocks of at most 128 rows take tiled copies (the other layouts plain loads)
+  CUtensorMap tx;
+  const bool tiled = !transpose && block_rows <= 128 &&
+                     make_map_3d(&tx, x, d, N, (long long)B * H, block_rows);
+  return launch_quantize_e4m3(tiled ? &tx : nullptr, x, out, scales, B, H, N, d, block_rows,
+                              transpose, n_pad, signs, err, sm_count(current_device()),
+                              stream) == 0
              ? ATTN_OK
              : ATTN_ERR_CUDA;
 }

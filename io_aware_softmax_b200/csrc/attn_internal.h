@@ -87,9 +87,11 @@ int launch_bwd_rowdot(const void* o, const void* dout, const float* lse, float* 
                       long long rows, int d, cudaStream_t stream);
 int launch_attn_bwd(const CUtensorMap& tq, const CUtensorMap& tdo, const CUtensorMap& tk,
                     const CUtensorMap& tv, const BwdParams& p, int d, cudaStream_t stream);
-int launch_quantize_e4m3(const void* x, void* out, float* scales, int B, int H, int N, int d,
-                         int block_rows, int transpose, int n_pad, const float* signs,
-                         uint32_t* err, int num_sms, cudaStream_t stream);
+// tmx: tiled map of x (make_map_3d over [B H, N, d] with block_rows-row boxes) for
+// row-major blocks of at most 128 rows, or nullptr.
+int launch_quantize_e4m3(const CUtensorMap* tmx, const void* x, void* out, float* scales, int B,
+                         int H, int N, int d, int block_rows, int transpose, int n_pad,
+                         const float* signs, uint32_t* err, int num_sms, cudaStream_t stream);
 int launch_merge(const float* o_part, const float* lse_part, void* o, float* lse, long long rows,
                  int S, int d, cudaStream_t stream);
 

@@ -184,6 +184,36 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
+// --------------------------------------------------------------------------- clusters
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+// The address of the same shared-memory location in CTA `rank` of this cluster.
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t saddr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+  return r;
+}
+
+__device__ __forceinline__ void st_shared_cluster_u32(uint32_t addr, uint32_t v) {
+  asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+
+// Cluster barrier halves.  Every thread of every CTA of the cluster arrives once per phase;
+// the wait returns when all have arrived (all CTAs of a cluster run at the same time).
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_arrive() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
 // --------------------------------------------------------------------------- tcgen05
 __device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem),
@@ -381,6 +411,16 @@ __device__ __forceinline__ void add2(float& a0, float& a1, float b0, float b1) {
       "add.rn.f32x2 ra, ra, rb;\n\tmov.b64 {%0, %1}, ra;\n\t}"
       : "+f"(a0), "+f"(a1)
       : "f"(b0), "f"(b1));
+}
+
+// One butterfly on two lanes at once: (a, b) <- (a + b, a - b) for both pairs, each result
+// rounded once (the same bits as the scalar add and subtract).
+__device__ __forceinline__ void butterfly2(float& a0, float& a1, float& b0, float& b1) {
+  asm("{\n\t.reg .b64 ra, rb, rs, rd;\n\t"
+      "mov.b64 ra, {%0, %1};\n\tmov.b64 rb, {%2, %3};\n\t"
+      "add.rn.f32x2 rs, ra, rb;\n\tsub.rn.f32x2 rd, ra, rb;\n\t"
+      "mov.b64 {%0, %1}, rs;\n\tmov.b64 {%2, %3}, rd;\n\t}"
+      : "+f"(a0), "+f"(a1), "+f"(b0), "+f"(b1));
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

@@ -48,12 +48,17 @@ def test_quantizer_is_bit_exact_without_rotation(d, N):
     assert np.allclose(scales.cpu().numpy(), want_s, rtol=1e-6, atol=0)
 
 
-@pytest.mark.parametrize("N,n_pad", [(300, 304), (128, 144), (5, 16)])
-def test_quantizer_transposed_per_head(N, n_pad):
-    x = workloads.randn_bf16((2, 2, N, 128), N, 1)
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("N,n_pad", [(300, 304), (128, 144), (5, 16), (2100, 2112),
+                                     (130, 400), (1100, 1424)])
+def test_quantizer_transposed_per_head(d, N, n_pad):
+    # one scale per head (the V layout of attn_fwd_fp8): a cluster of CTAs per head; more
+    # sub-blocks of 128 keys than CTAs (2100), and n_pad reaching past the last sub-block
+    # with keys (130 -> 400, 1100 -> 1424), whose columns must come out zero
+    x = workloads.randn_bf16((2, 2, N, d), N + d, 1)
     codes, scales = quantize_fp8(x.cuda(), block_rows=N, transpose=True, n_pad=n_pad)
     assert device_status() == 0
-    assert codes.shape == (2, 2, 128, n_pad) and scales.shape == (2, 2, 1)
+    assert codes.shape == (2, 2, d, n_pad) and scales.shape == (2, 2, 1)
     want_c, want_s = ofp8.quantize_blocks(x.float().numpy(), N)
     got = _codes(codes)
     assert np.array_equal(got[..., :N], np.swapaxes(want_c, 2, 3))
@@ -64,10 +69,12 @@ def test_quantizer_transposed_per_head(N, n_pad):
 @pytest.mark.parametrize("d", [64, 128])
 @pytest.mark.parametrize("N,block_rows,transpose", [(700, 300, False), (700, 700, False),
                                                     (300, 64, True), (130, 7, True),
-                                                    (100, 3, False)])
-def test_quantizer_chunked_blocks_are_bit_exact(d, N, block_rows, transpose):
-    # blocks longer than 128 rows, several blocks per chunk, and transposed outputs with
-    # several blocks per head go through the chunked amax / codes / finalize launches
+                                                    (100, 3, False), (500, 64, False),
+                                                    (333, 100, False), (129, 16, False)])
+def test_quantizer_blocks_are_bit_exact(d, N, block_rows, transpose):
+    # row-major blocks of at most 128 rows (a tiled copy of block_rows rows each, ragged last
+    # blocks), blocks longer than 128 rows, and transposed outputs with several blocks per
+    # head (the chunked amax / codes / finalize launches)
     x = (workloads.randn_bf16((2, 2, N, d), N + block_rows, 3).float()
          * torch.tensor([1.0, 7.0]).view(1, 2, 1, 1)).to(torch.bfloat16)
     n_pad = -(-N // 16) * 16
@@ -82,6 +89,42 @@ def test_quantizer_chunked_blocks_are_bit_exact(d, N, block_rows, transpose):
     else:
         assert np.array_equal(got, want_c)
     assert np.allclose(scales.cpu().numpy(), want_s, rtol=1e-6, atol=0)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_quantizer_row_major_output_aligned_to_4_bytes(d):
+    # a row-major output that is 4-byte but not 16-byte aligned takes 4-byte stores
+    from io_aware_softmax_b200 import _lib
+    N = 300
+    x = workloads.randn_bf16((1, 2, N, d), 77, 4).cuda()
+    buf = torch.zeros(2 * N * d + 64, dtype=torch.uint8, device="cuda")
+    scales = torch.empty((1, 2, 3), dtype=torch.float32, device="cuda")
+    st = _lib.load().attn_quantize_fp8(x.data_ptr(), buf.data_ptr() + 4, scales.data_ptr(), 1, 2,
+                                       N, d, 128, 0, 0, None,
+                                       torch.cuda.current_stream().cuda_stream)
+    torch.cuda.synchronize()
+    assert st == 0 and device_status() == 0
+    got = buf[4:4 + 2 * N * d].view(torch.float8_e4m3fn).float().cpu().numpy().reshape(1, 2, N, d)
+    want_c, want_s = ofp8.quantize_blocks(x.cpu().float().numpy(), 128)
+    assert np.array_equal(got.astype(np.float64), want_c)
+    assert torch.all(buf[:4] == 0) and torch.all(buf[4 + 2 * N * d:] == 0)   # nothing outside
+    assert np.allclose(scales.cpu().numpy(), want_s, rtol=1e-6, atol=0)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_rotated_codes_agree_between_kernels(d):
+    # rotation in one thread's registers (row-major, 128-row blocks) and across lanes
+    # (transposed blocks of 128 rows) round every operation alike: the same bits
+    x = workloads.randn_bf16((2, 2, 300, d), 5 * d, 5)
+    x[0, 1, :, 3] *= 50
+    signs = torch.from_numpy(np.random.default_rng(d + 1).choice([-1.0, 1.0], d)
+                             .astype(np.float32)).cuda()
+    c_row, s_row = quantize_fp8(x.cuda(), block_rows=128, signs=signs)
+    c_t, s_t = quantize_fp8(x.cuda(), block_rows=128, signs=signs, transpose=True, n_pad=304)
+    assert device_status() == 0
+    assert torch.equal(s_row, s_t)
+    assert torch.equal(c_row.view(torch.uint8),
+                       c_t.view(torch.uint8)[..., :300].transpose(2, 3))
 
 
 @pytest.mark.parametrize("d", [64, 128])
