@@ -219,7 +219,11 @@ extern "C" int attn_fwd_alibi(const void* q, const void* k, const void* v, void*
       normal = normal && std::isnormal(p.cap_poly[i]);
       cs_pow *= (double)p.cap_scale * (double)p.cap_scale;
     }
-    if (normal) p.cap_fast_max = kTanhPolyMaxY / p.cap_scale;
+    // The polynomial's leading coefficient is positive, so a masked score (-inf) comes out
+    // of it as -inf: the kernels need no other mask on the polynomial path.
+    static_assert(kTanhPoly[kTanhPolyTerms - 1] > 0.f, "leading coefficient");
+    if (normal)
+      p.cap_fast_max = kTanhPolyMaxY / p.cap_scale;
   }
   p.mask = mask_params(mask_kind, window, doc_offsets, num_docs, Nq, Nk);
   p.alibi = alibi_slopes;

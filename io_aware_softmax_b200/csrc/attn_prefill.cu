@@ -122,44 +122,36 @@ __device__ __forceinline__ float tile_row_absmax(const uint32_t (&s)[128]) {
   return fmaxf(fmaxf(a0, a1), fmaxf(a2, a3));
 }
 
-// Soft-cap, in place: every raw score of the row becomes its base-2 capped score
-// c log2(e) tanh(s scale / c).  kPoly (the row's |s scale / c| are all <= 1/2): the odd
-// polynomial s sum_i b_i s^(2i) of p.cap_poly (c log2(e) and the powers of scale / c folded
-// into the coefficients), evaluated in Estrin's scheme in paired FMAs -- depth 5 instead of
-// Horner's 6, so more of the row's independent pairs fit in the FMA pipe's latency;
-// otherwise the identity tanh(y) = 1 - 2 / (e^(2y) + 1) on ex2 and rcp.  The mask is
-// applied afterwards (the transform leaves no score at -inf).
-template <bool kPoly>
-__device__ __forceinline__ void cap_row(uint32_t (&s)[128], const FwdParams& p) {
-  if constexpr (kPoly) {
-    const float b0 = p.cap_poly[0], b1 = p.cap_poly[1], b2 = p.cap_poly[2], b3 = p.cap_poly[3],
-                b4 = p.cap_poly[4];
-#pragma unroll
-    for (int c = 0; c < 128; c += 2) {
-      const float s0 = f32(s[c]), s1 = f32(s[c + 1]);
-      float w0, w1, u0, u1, v0, v1, z0, z1;
-      fmul2(w0, w1, s0, s1, s0, s1);                   // w = s^2
-      ffma2(u0, u1, w0, w1, b1, b1, b0, b0);           // b1 w + b0
-      ffma2(v0, v1, w0, w1, b3, b3, b2, b2);           // b3 w + b2
-      fmul2(z0, z1, w0, w1, w0, w1);                   // w^2
-      ffma2(v0, v1, z0, z1, b4, b4, v0, v1);           // b4 w^2 + b3 w + b2
-      ffma2(u0, u1, v0, v1, z0, z1, u0, u1);           // ... w^2 + b1 w + b0
-      fmul2(u0, u1, u0, u1, s0, s1);
-      s[c] = __float_as_uint(u0);
-      s[c + 1] = __float_as_uint(u1);
-    }
-  } else {
-#pragma unroll
-    for (int c = 0; c < 128; ++c)
-      s[c] = __float_as_uint(p.cap_log2 * tanh_via_ex2(f32(s[c]) * p.cap_scale));
-  }
+// The soft-cap polynomial of p.cap_poly at one raw score s (|s| <= cap_fast_max): the
+// base-2 capped score c log2(e) tanh(s scale / c) = s (b0 + w (b1 + w (b2 + w (b3 + w b4)))),
+// w = s^2, c log2(e) and the powers of scale / c folded into the b_i.  Horner's scheme: four
+// multiply-adds after the square; tile_row_exp_half_cap takes the same steps per score in
+// paired instructions (each lane rounded as here), so this is the value it gives that score
+// before subtracting the reference max.  b4 > 0, so s = -inf (a masked score) gives -inf.
+__device__ __forceinline__ float cap_poly_at(float s, const FwdParams& p) {
+  const float w = s * s;
+  float t = fmaf(p.cap_poly[4], w, p.cap_poly[3]);
+  t = fmaf(t, w, p.cap_poly[2]);
+  t = fmaf(t, w, p.cap_poly[1]);
+  t = fmaf(t, w, p.cap_poly[0]);
+  return t * s;
 }
 
-// Masked columns (outside [c_lo, c_hi]) of one tile row become -inf.
-__device__ __forceinline__ void mask_row(uint32_t (&s)[128], int c_lo, int c_hi) {
+// Soft-cap, in place, outside the polynomial's range: every raw score of the row becomes its
+// base-2 capped score c log2(e) tanh(s scale / c) by the identity
+// tanh(y) = 1 - 2 / (e^(2y) + 1) on ex2 and rcp (a masked NaN stays NaN).
+__device__ __forceinline__ void cap_row_exact(uint32_t (&s)[128], const FwdParams& p) {
 #pragma unroll
   for (int c = 0; c < 128; ++c)
-    if ((unsigned)(c - c_lo) > (unsigned)(c_hi - c_lo)) s[c] = kNegInfBits;
+    s[c] = __float_as_uint(p.cap_log2 * tanh_via_ex2(f32(s[c]) * p.cap_scale));
+}
+
+// Masked columns (outside [c_lo, c_hi]) of one tile row become `bits` (-inf by default).
+__device__ __forceinline__ void mask_row(uint32_t (&s)[128], int c_lo, int c_hi,
+                                         uint32_t bits = kNegInfBits) {
+#pragma unroll
+  for (int c = 0; c < 128; ++c)
+    if ((unsigned)(c - c_lo) > (unsigned)(c_hi - c_lo)) s[c] = bits;
 }
 
 // ALiBi: the row's scores become base-2 biased scores in place,
@@ -175,6 +167,39 @@ __device__ __forceinline__ void alibi_row(uint32_t (&s)[128], const FwdParams& p
     s[c] = __float_as_uint(t0);
     s[c + 1] = __float_as_uint(t1);
   }
+}
+
+// Soft-capped P = 2^(cap(s) - m_use) for one 64-column half of a tile row of raw scores
+// (every |s| <= cap_fast_max, masked ones -inf): the polynomial of cap_poly_at with the
+// subtraction of m_use folded into its last step, so the cap costs the FMA pipe five paired
+// instructions per pair of scores on top of the plain exponential.  A masked score's -inf
+// stays -inf through the polynomial (positive leading coefficient), so its exponential is 0.
+// Returns the half's sum.
+__device__ __forceinline__ float tile_row_exp_half_cap(const uint32_t (&s)[128], int base,
+                                                       const FwdParams& p, float m_use,
+                                                       uint32_t (&pk)[32]) {
+  const float b0 = p.cap_poly[0], b1 = p.cap_poly[1], b2 = p.cap_poly[2], b3 = p.cap_poly[3],
+              b4 = p.cap_poly[4];
+  float a0 = 0.f, a1 = 0.f, c0 = 0.f, c1 = 0.f;
+#pragma unroll
+  for (int c = 0; c < 64; c += 2) {
+    const float s0 = f32(s[base + c]), s1 = f32(s[base + c + 1]);
+    float w0, w1, t0, t1;
+    fmul2(w0, w1, s0, s1, s0, s1);
+    ffma2(t0, t1, w0, w1, b4, b4, b3, b3);
+    ffma2(t0, t1, t0, t1, w0, w1, b2, b2);
+    ffma2(t0, t1, t0, t1, w0, w1, b1, b1);
+    ffma2(t0, t1, t0, t1, w0, w1, b0, b0);
+    ffma2(t0, t1, t0, t1, s0, s1, -m_use, -m_use);   // cap(s) - m_use
+    const float e0 = ex2_approx(t0);
+    const float e1 = ex2_approx(t1);
+    if ((c >> 1) & 1)
+      add2(c0, c1, e0, e1);
+    else
+      add2(a0, a1, e0, e1);
+    pk[c >> 1] = pack_bf16x2(e0, e1);
+  }
+  return (a0 + a1) + (c0 + c1);
 }
 
 // FP8 path: 2^(x - m_use + 6) = 64 P for one 64-column half of a tile row, packed four
@@ -687,20 +712,28 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
         const bool masked =
             !(lo_last <= k0 && k0 + kBN - 1 <= hi_first && k0 + kBN <= p.Nk);
         float mx;
+        bool cap_fused = false;   // soft-cap folded into the exponentials (see below)
         const float ks_eff = kFp8 ? p.kscale * qs * __ldg(ksc + k0 / kBN) : p.kscale;
         if constexpr (kFp8) {
           const float mx_raw = masked ? tile_row_max<true>(s, row_lo - k0, row_hi - k0)
                                       : tile_row_max<false>(s, 0, 0);
           mx = mx_raw * ks_eff;
         } else if constexpr (kCap) {
-          // The row's scores become base-2 capped scores in place (the polynomial tanh when
-          // the row's largest |s| is in its range), then the mask, then the row max.
-          if (tile_row_absmax(s) <= p.cap_fast_max)
-            cap_row<true>(s, p);
-          else
-            cap_row<false>(s, p);
-          if (masked) mask_row(s, row_lo - k0, row_hi - k0);
-          mx = tile_row_max<false>(s, 0, 0);
+          // When the row's raw scores (masked ones included) lie in the polynomial's range,
+          // the cap (increasing) of the raw max over the visible columns is the row max of
+          // the capped scores, and the cap itself is applied inside the exponential loop
+          // (masked scores -inf).  Otherwise the scores become base-2 capped scores in place
+          // by the ex2/rcp identity, then -inf where masked, then the row max.
+          cap_fused = tile_row_absmax(s) <= p.cap_fast_max;
+          if (cap_fused) {
+            mx = masked ? tile_row_max<true>(s, row_lo - k0, row_hi - k0)
+                        : tile_row_max<false>(s, 0, 0);
+            if (mx != -INFINITY) mx = cap_poly_at(mx, p);
+          } else {
+            cap_row_exact(s, p);
+            if (masked) mask_row(s, row_lo - k0, row_hi - k0);
+            mx = tile_row_max<false>(s, 0, 0);
+          }
         } else if constexpr (!kAlibi) {
           const float mx_raw = masked ? tile_row_max<true>(s, row_lo - k0, row_hi - k0)
                                       : tile_row_max<false>(s, 0, 0);
@@ -748,7 +781,10 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
             if constexpr (kAlibi) {
               sum += tile_row_exp_half(s, 64 * half, 1.f, m_use, pk);
             } else if constexpr (kCap) {
-              sum += tile_row_exp_half(s, 64 * half, 1.f, m_use, pk);   // capped
+              if (cap_fused)
+                sum += tile_row_exp_half_cap(s, 64 * half, p, m_use, pk);
+              else
+                sum += tile_row_exp_half(s, 64 * half, 1.f, m_use, pk);   // capped in place
             } else {
               sum += tile_row_exp_half(s, 64 * half, p.kscale, m_use, pk);
             }

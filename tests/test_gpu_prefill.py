@@ -105,6 +105,9 @@ def test_softcap(mask):
     # cap 10 with std-2 inputs: |scale s / cap| ~ 0.4, so rows above and below the
     # polynomial tanh's range of 1 mix inside every warp
     _run_full(1, 2, 2, 520, 520, 128, mask=mask, softcap=10.0, docs=docs, seed=5, std=2.0)
+    # a small cap (0.5) on small scores: the polynomial path with cap_log2 < 1, where the
+    # masked columns' stand-in score must still give exponentials of exactly 0
+    _run_full(1, 2, 2, 520, 520, 128, mask=mask, softcap=0.5, docs=docs, seed=6, std=0.2)
 
 
 @pytest.mark.parametrize("Nq,Nk", [(1, 300), (100, 1000), (300, 129), (513, 64)])

@@ -1,7 +1,8 @@
 """The soft-cap's polynomial tanh (csrc/tanh_poly.cuh): the committed coefficients are what
 the generator computes, and the polynomial meets its error bound against numpy's tanh, both
 as fitted (float32 Horner steps in y^2, times y) and as the kernel evaluates it (coefficients
-folded into the raw score, Estrin's order, float32)."""
+folded into the raw score, Horner's scheme in float32 multiply-adds, the reference max
+subtracted in the last one) -- where a masked score, -inf, must stay -inf."""
 import importlib.util
 import os
 import re
@@ -44,13 +45,31 @@ def test_polynomial_tanh_error_bound():
     assert np.all(np.sign(y * acc) == np.sign(y))          # odd, no sign flips near 0
 
 
+def _fma(a, b, c):
+    # float32 fused multiply-add: the exact product plus c, rounded once (float64 holds the
+    # product of two float32 values exactly; the sum is rounded to float64 first, which
+    # agrees with a single rounding except in ties far below the bounds checked here)
+    return (a.astype(np.float64) * b.astype(np.float64) + c.astype(np.float64)).astype(np.float32)
+
+
+def _horner(b, s):
+    # the kernel's steps: w = s^2, t = b4 w + b3, then t w + b_i for i = 2, 1, 0
+    w = (s * s).astype(np.float32)
+    t = _fma(np.full_like(w, b[4]), w, np.full_like(w, b[3]))
+    for i in (2, 1, 0):
+        t = _fma(t, w, np.full_like(w, b[i]))
+    return t
+
+
 def test_folded_coefficients_in_the_raw_score():
-    # The kernel evaluates c log2(e) tanh(s cs) as s (b0 + b1 w + (b2 + b3 w + b4 w^2) w^2),
-    # w = s^2, b_i = c log2(e) a_i cs^(2i+1) rounded to float32, all in float32 (Estrin's
-    # order).  The base-2 capped score must stay within 1e-5 plus four float32 roundings of
-    # its own size (2.4e-7 relative) over |s cs| <= 1/2 (LSE is checked to 1e-3), for caps
-    # from 1 to 1000 at d = 64 and 128.
+    # The kernel evaluates c log2(e) tanh(s cs) as s (b0 + w (b1 + w (b2 + w (b3 + w b4)))),
+    # w = s^2, b_i = c log2(e) a_i cs^(2i+1) rounded to float32, all in float32 with fused
+    # multiply-adds (Horner's scheme); the last step also subtracts the row's reference max
+    # m, t s - m in one multiply-add.  Over |s cs| <= 1/2 the base-2 capped score must stay
+    # within 1e-5 plus 2.4e-7 of its own size (about four float32 roundings), for caps from 1
+    # to 1000 at d = 64 and 128 (LSE is checked to 1e-3).
     a = _committed().astype(np.float64)
+    assert a[-1] > 0        # a masked score, -inf, must come out of the polynomial as -inf
     for d in (64, 128):
         for cap in (1.0, 5.0, 50.0, 1000.0):
             cs = np.float32((1.0 / np.sqrt(d)) / cap)
@@ -59,13 +78,17 @@ def test_folded_coefficients_in_the_raw_score():
                          dtype=np.float32)
             assert np.all(np.abs(b) >= np.finfo(np.float32).tiny)   # all normal: path taken
             s = np.linspace(-0.5 / float(cs), 0.5 / float(cs), 200001).astype(np.float32)
-            w = s * s
-            u = b[1] * w + b[0]
-            v = b[3] * w + b[2]
-            z = w * w
-            v = b[4] * z + v
-            u = v * z + u
-            x = (u * s).astype(np.float64)
+            t = _horner(b, s)
             ref = L * np.tanh(s.astype(np.float64) * float(cs))
+            x = (t * s).astype(np.float64)
             assert np.all(np.abs(x - ref) <= 1e-5 + 2.4e-7 * np.abs(ref)), (
                 d, cap, np.abs(x - ref).max())
+            m = np.float32(L * 0.3)                                  # a reference max
+            xm = _fma(t, s, np.full_like(s, -m)).astype(np.float64)
+            assert np.all(np.abs(xm - (ref - float(m))) <=
+                          1e-5 + 2.4e-7 * (np.abs(ref) + float(m))), (
+                d, cap, np.abs(xm - (ref - float(m))).max())
+            with np.errstate(invalid="ignore", over="ignore"):
+                neg_inf = np.array([-np.inf], dtype=np.float32)
+                x_masked = _fma(_horner(b, neg_inf), neg_inf, np.array([-m], np.float32))
+            assert x_masked[0] == -np.inf
