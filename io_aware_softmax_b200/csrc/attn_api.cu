@@ -73,6 +73,28 @@ bool make_map_3d(CUtensorMap* map, const void* ptr, int d, long long rows, long 
   return r == CUDA_SUCCESS;
 }
 
+// The soft-cap's polynomial tanh in the raw score s: cap_log2 tanh(s cap_scale) =
+// s sum_i b_i s^(2i) with b_i = cap_log2 a_i cap_scale^(2i + 1), for |s cap_scale| <= 1/2
+// (fast_max = 1 / (2 cap_scale) in raw units).  The kernels take it only when every b_i is a
+// normal float (no term flushed to zero); otherwise fast_max = -1 turns it off.
+void soft_cap_poly(float cap_scale, float cap_log2, float (&poly)[kTanhPolyTerms],
+                   float& fast_max) {
+  // The leading coefficient is positive, so a masked score (-inf) comes out of the
+  // polynomial as -inf: the kernels need no other mask on the polynomial path.
+  static_assert(kTanhPoly[kTanhPolyTerms - 1] > 0.f, "leading coefficient");
+  fast_max = -1.f;
+  for (int i = 0; i < kTanhPolyTerms; ++i) poly[i] = 0.f;
+  if (!(cap_scale > 0.f)) return;
+  bool normal = true;
+  double cs_pow = (double)cap_scale;
+  for (int i = 0; i < kTanhPolyTerms; ++i) {
+    poly[i] = (float)((double)kTanhPoly[i] * (double)cap_log2 * cs_pow);
+    normal = normal && std::isnormal(poly[i]);
+    cs_pow *= (double)cap_scale * (double)cap_scale;
+  }
+  if (normal) fast_max = kTanhPolyMaxY / cap_scale;
+}
+
 int check_mask(int mask_kind, int window, const int* doc_offsets, int num_docs, int Nq, int Nk) {
   if (mask_kind < ATTN_MASK_NONE || mask_kind > ATTN_MASK_SLIDING) return ATTN_ERR_INVALID_ARG;
   if (mask_kind != ATTN_MASK_NONE && Nq != Nk) return ATTN_ERR_UNSUPPORTED;
@@ -205,26 +227,7 @@ extern "C" int attn_fwd_alibi(const void* q, const void* k, const void* v, void*
   p.softcap = softcap > 0.f ? softcap : 0.f;
   p.cap_scale = softcap > 0.f ? scale / softcap : 0.f;
   p.cap_log2 = softcap > 0.f ? softcap * kLog2e : 0.f;
-  // The soft-cap's polynomial tanh in the raw score s: cap_log2 tanh(s cap_scale) =
-  // s sum_i b_i s^(2i) with b_i = cap_log2 a_i cap_scale^(2i + 1), for |s cap_scale| <= 1/2.
-  // The kernels take it only when every b_i is a normal float (no term flushed to zero).
-  static_assert(sizeof(p.cap_poly) / sizeof(float) == kTanhPolyTerms, "soft-cap polynomial");
-  p.cap_fast_max = -1.f;
-  if (softcap > 0.f) {
-    bool normal = true;
-    double cs_pow = (double)p.cap_scale;
-    for (int i = 0; i < kTanhPolyTerms; ++i) {
-      const double b = (double)kTanhPoly[i] * (double)p.cap_log2 * cs_pow;
-      p.cap_poly[i] = (float)b;
-      normal = normal && std::isnormal(p.cap_poly[i]);
-      cs_pow *= (double)p.cap_scale * (double)p.cap_scale;
-    }
-    // The polynomial's leading coefficient is positive, so a masked score (-inf) comes out
-    // of it as -inf: the kernels need no other mask on the polynomial path.
-    static_assert(kTanhPoly[kTanhPolyTerms - 1] > 0.f, "leading coefficient");
-    if (normal)
-      p.cap_fast_max = kTanhPolyMaxY / p.cap_scale;
-  }
+  soft_cap_poly(p.cap_scale, p.cap_log2, p.cap_poly, p.cap_fast_max);
   p.mask = mask_params(mask_kind, window, doc_offsets, num_docs, Nq, Nk);
   p.alibi = alibi_slopes;
   if ((long long)p.num_pairs * B * Hq > (1LL << 31) - 1) return ATTN_ERR_UNSUPPORTED;
@@ -505,6 +508,7 @@ extern "C" int attn_bwd_alibi(const void* q, const void* k, const void* v, const
   p.alibi = alibi_slopes;
   p.cap_scale = softcap > 0.f ? scale / softcap : 0.f;
   p.cap_log2 = softcap > 0.f ? softcap * kLog2e : 0.f;
+  soft_cap_poly(p.cap_scale, p.cap_log2, p.cap_poly, p.cap_fast_max);
   p.err = error_word_ptr(dev);
   if (p.err == nullptr) return ATTN_ERR_CUDA;
   if (Nq > 0 && launch_bwd_rowdot(o, dout, lse, const_cast<float*>(p.dvec),

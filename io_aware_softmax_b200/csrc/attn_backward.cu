@@ -102,10 +102,50 @@ __device__ __forceinline__ float bf(uint32_t u) { return __uint_as_float(u); }
 //   grads: ds = p (dp - Dv) and bf16 pairs of ds (and of p, optionally) for the 32 columns
 //          [OFF, OFF + 32).
 // l2(j) and dv(j) give the four columns' values, vis(j) a 4-bit mask of visible pairs.
-// kCap: the score is soft-capped, x = cap_log2 tanh(s cap_scale) - l2 (base 2).
+// kCap: the score is soft-capped, x = cap_log2 tanh(s cap_scale) - l2 (base 2).  When every
+// raw score of the run, in every lane of the warp, lies in the polynomial's range
+// (|s| <= cap_fast_max), x is the polynomial of cap_poly with the subtraction folded into
+// its last step -- square, four Horner multiply-adds and one more, in paired f32x2
+// instructions, no MUFU work besides the exponential; otherwise tanh(y) = 1 - 2/(e^(2y)+1)
+// on ex2 and rcp.  The choice is per warp and per call, so the loop that runs is one
+// straight block of code.
 template <int N, bool kCap = false, typename L2, typename Vis>
 __device__ __forceinline__ void probs(uint32_t (&s)[N], float ks, L2 l2, Vis vis,
-                                      float cap_scale = 0.f, float cap_log2 = 0.f) {
+                                      const BwdParams& bp) {
+  if constexpr (kCap) {
+    float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+    for (int c = 0; c < N; c += 4) {
+      a0 = max3f(a0, fabsf(bf(s[c])), fabsf(bf(s[c + 1])));
+      a1 = max3f(a1, fabsf(bf(s[c + 2])), fabsf(bf(s[c + 3])));
+    }
+    if (__all_sync(0xffffffffu, fmaxf(a0, a1) <= bp.cap_fast_max)) {
+      const float b0 = bp.cap_poly[0], b1 = bp.cap_poly[1], b2 = bp.cap_poly[2],
+                  b3 = bp.cap_poly[3], b4 = bp.cap_poly[4];
+#pragma unroll
+      for (int j = 0; j < N / 4; ++j) {
+        const float4 l = l2(j);
+        const unsigned m = vis(j);
+        const int c = 4 * j;
+        float x[4];
+#pragma unroll
+        for (int h = 0; h < 4; h += 2) {
+          const float s0 = bf(s[c + h]), s1 = bf(s[c + h + 1]);
+          float w0, w1, t0, t1;
+          fmul2(w0, w1, s0, s1, s0, s1);
+          ffma2(t0, t1, w0, w1, b4, b4, b3, b3);
+          ffma2(t0, t1, t0, t1, w0, w1, b2, b2);
+          ffma2(t0, t1, t0, t1, w0, w1, b1, b1);
+          ffma2(t0, t1, t0, t1, w0, w1, b0, b0);
+          ffma2(x[h], x[h + 1], t0, t1, s0, s1, h ? -l.z : -l.x, h ? -l.w : -l.y);
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+          s[c + i] = __float_as_uint(((m >> i) & 1u) ? ex2_approx(x[i]) : 0.f);
+      }
+      return;
+    }
+  }
 #pragma unroll
   for (int j = 0; j < N / 4; ++j) {
     const float4 l = l2(j);
@@ -113,10 +153,10 @@ __device__ __forceinline__ void probs(uint32_t (&s)[N], float ks, L2 l2, Vis vis
     const int c = 4 * j;
     float x0, x1, x2, x3;
     if constexpr (kCap) {
-      x0 = fmaf(cap_log2, tanh_via_ex2(bf(s[c]) * cap_scale), -l.x);
-      x1 = fmaf(cap_log2, tanh_via_ex2(bf(s[c + 1]) * cap_scale), -l.y);
-      x2 = fmaf(cap_log2, tanh_via_ex2(bf(s[c + 2]) * cap_scale), -l.z);
-      x3 = fmaf(cap_log2, tanh_via_ex2(bf(s[c + 3]) * cap_scale), -l.w);
+      x0 = fmaf(bp.cap_log2, tanh_via_ex2(bf(s[c]) * bp.cap_scale), -l.x);
+      x1 = fmaf(bp.cap_log2, tanh_via_ex2(bf(s[c + 1]) * bp.cap_scale), -l.y);
+      x2 = fmaf(bp.cap_log2, tanh_via_ex2(bf(s[c + 2]) * bp.cap_scale), -l.z);
+      x3 = fmaf(bp.cap_log2, tanh_via_ex2(bf(s[c + 3]) * bp.cap_scale), -l.w);
     } else {
       ffma2(x0, x1, bf(s[c]), bf(s[c + 1]), ks, ks, -l.x, -l.y);
       ffma2(x2, x3, bf(s[c + 2]), bf(s[c + 3]), ks, ks, -l.z, -l.w);
@@ -511,10 +551,10 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
           const float c = (float)(4 * j);
           return make_float4(fmaf(slope2, fabsf(drow - c), l2r), fmaf(slope2, fabsf(drow - c - 1.f), l2r),
                              fmaf(slope2, fabsf(drow - c - 2.f), l2r), fmaf(slope2, fabsf(drow - c - 3.f), l2r));
-        }, [&](int j) { return vis(4 * j); });
+        }, [&](int j) { return vis(4 * j); }, p);
       } else {
         probs<64, kCap>(s, p.kscale, [&](int) { return l2r4; }, [&](int j) { return vis(4 * j); },
-                        p.cap_scale, p.cap_log2);
+                        p);
       }
       ok = __all_sync(0xffffffffu, mbar_wait(bar(BAR_DP), t & 1, abort_flag, p.err, kSiteBwdS));
       if (!ok) break;
@@ -811,13 +851,13 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmQ,
         tmem_ld_x32_async(tl + kTmemX + col, pr0);
         tmem_ld_wait_x32(pr0);
         probs<32, kCap>(pr0, p.kscale, [&](int j) { return l2f(4 * j); },
-                        [&](int j) { return vis(4 * j); }, p.cap_scale, p.cap_log2);
+                        [&](int j) { return vis(4 * j); }, p);
         pack_pairs(pr0, pk);
         tmem_st_x16(tl + kTmemX + col, pk);
         tmem_ld_x32_async(tl + kTmemX + col + 32u, pr1);
         tmem_ld_wait_x32(pr1);
         probs<32, kCap>(pr1, p.kscale, [&](int j) { return l2f(32 + 4 * j); },
-                        [&](int j) { return vis(32 + 4 * j); }, p.cap_scale, p.cap_log2);
+                        [&](int j) { return vis(32 + 4 * j); }, p);
         pack_pairs(pr1, pk);
         tmem_st_x16(tl + kTmemX + col + 16u, pk);
       }

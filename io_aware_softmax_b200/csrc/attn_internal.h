@@ -72,6 +72,8 @@ struct BwdParams {
   const float* alibi;  // fp32 [Hq] ALiBi slopes (natural-log units), or nullptr
   float cap_scale;    // soft-cap c > 0: scale / c (0: no cap)
   float cap_log2;     // c * log2(e)
+  float cap_poly[5];  // the polynomial tanh, as FwdParams::cap_poly
+  float cap_fast_max; // as FwdParams::cap_fast_max
   uint32_t* err;      // device error word of the library (bits, first site)
 };
 
