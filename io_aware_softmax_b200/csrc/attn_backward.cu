@@ -109,9 +109,12 @@ __device__ __forceinline__ float bf(uint32_t u) { return __uint_as_float(u); }
 // instructions, no MUFU work besides the exponential; otherwise tanh(y) = 1 - 2/(e^(2y)+1)
 // on ex2 and rcp.  The choice is per warp and per call, so the loop that runs is one
 // straight block of code.
-template <int N, bool kCap = false, typename L2, typename Vis>
+// kKeepX (with kCap): s keeps the base-2 exponent x itself (-inf where not visible) instead
+// of p = 2^x, for a caller whose grads step takes kFromX.
+template <int N, bool kCap = false, bool kKeepX = false, typename L2, typename Vis>
 __device__ __forceinline__ void probs(uint32_t (&s)[N], float ks, L2 l2, Vis vis,
                                       const BwdParams& bp) {
+  static_assert(!kKeepX || kCap, "the exponent is kept on the soft-cap path only");
   if constexpr (kCap) {
     float a0 = 0.f, a1 = 0.f;
 #pragma unroll
@@ -141,7 +144,8 @@ __device__ __forceinline__ void probs(uint32_t (&s)[N], float ks, L2 l2, Vis vis
         }
 #pragma unroll
         for (int i = 0; i < 4; ++i)
-          s[c + i] = __float_as_uint(((m >> i) & 1u) ? ex2_approx(x[i]) : 0.f);
+          s[c + i] = __float_as_uint(((m >> i) & 1u) ? (kKeepX ? x[i] : ex2_approx(x[i]))
+                                                     : (kKeepX ? -INFINITY : 0.f));
       }
       return;
     }
@@ -161,10 +165,17 @@ __device__ __forceinline__ void probs(uint32_t (&s)[N], float ks, L2 l2, Vis vis
       ffma2(x0, x1, bf(s[c]), bf(s[c + 1]), ks, ks, -l.x, -l.y);
       ffma2(x2, x3, bf(s[c + 2]), bf(s[c + 3]), ks, ks, -l.z, -l.w);
     }
-    s[c] = __float_as_uint((m & 1u) ? ex2_approx(x0) : 0.f);
-    s[c + 1] = __float_as_uint((m & 2u) ? ex2_approx(x1) : 0.f);
-    s[c + 2] = __float_as_uint((m & 4u) ? ex2_approx(x2) : 0.f);
-    s[c + 3] = __float_as_uint((m & 8u) ? ex2_approx(x3) : 0.f);
+    if constexpr (kKeepX) {
+      s[c] = __float_as_uint((m & 1u) ? x0 : -INFINITY);
+      s[c + 1] = __float_as_uint((m & 2u) ? x1 : -INFINITY);
+      s[c + 2] = __float_as_uint((m & 4u) ? x2 : -INFINITY);
+      s[c + 3] = __float_as_uint((m & 8u) ? x3 : -INFINITY);
+    } else {
+      s[c] = __float_as_uint((m & 1u) ? ex2_approx(x0) : 0.f);
+      s[c + 1] = __float_as_uint((m & 2u) ? ex2_approx(x1) : 0.f);
+      s[c + 2] = __float_as_uint((m & 4u) ? ex2_approx(x2) : 0.f);
+      s[c + 3] = __float_as_uint((m & 8u) ? ex2_approx(x3) : 0.f);
+    }
   }
 }
 
@@ -176,23 +187,49 @@ __device__ __forceinline__ float cap_factor(float p, float l, float inv_cap_log2
   return fmaf(-t, t, 1.f);
 }
 
-template <bool kWantP, int OFF, int N, int ND, bool kCap = false, typename DV,
-          typename L2 = float4 (*)(int)>
+// kFromX (with kCap): pr holds the base-2 exponents x of probs<..., kKeepX>; p = 2^x here,
+// and tanh = (x + l2) / cap_log2 comes from x directly, so the pair of steps takes one MUFU
+// operation per score (the exponential) instead of an exponential and a logarithm.
+__device__ __forceinline__ float cap_factor_x(float x, float l, float inv_cap_log2) {
+  const float t = (x + l) * inv_cap_log2;
+  return (x != -INFINITY) ? fmaf(-t, t, 1.f) : 0.f;
+}
+
+template <bool kWantP, int OFF, int N, int ND, bool kCap = false, bool kFromX = false,
+          typename DV, typename L2 = float4 (*)(int)>
 __device__ __forceinline__ void grads(const uint32_t (&pr)[N], const uint32_t (&dp)[ND], DV dv,
                                       uint32_t (&pk)[16], uint32_t (&dsk)[16], L2 l2 = nullptr,
                                       float inv_cap_log2 = 0.f) {
   static_assert(ND == 32 || ND == N, "dp holds these 32 columns or all N");
+  static_assert(!kFromX || kCap, "exponents are kept on the soft-cap path only");
   constexpr int DOFF = (ND == 32) ? 0 : OFF;
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
     const float4 d = dv(j);
     const int c = OFF + 4 * j, e = DOFF + 4 * j;
-    const float p0 = bf(pr[c]), p1 = bf(pr[c + 1]), p2 = bf(pr[c + 2]), p3 = bf(pr[c + 3]);
+    float p0, p1, p2, p3;
+    if constexpr (kFromX) {
+      p0 = ex2_approx(bf(pr[c]));
+      p1 = ex2_approx(bf(pr[c + 1]));
+      p2 = ex2_approx(bf(pr[c + 2]));
+      p3 = ex2_approx(bf(pr[c + 3]));
+    } else {
+      p0 = bf(pr[c]);
+      p1 = bf(pr[c + 1]);
+      p2 = bf(pr[c + 2]);
+      p3 = bf(pr[c + 3]);
+    }
     float d0 = p0 * (bf(dp[e]) - d.x);
     float d1 = p1 * (bf(dp[e + 1]) - d.y);
     float d2 = p2 * (bf(dp[e + 2]) - d.z);
     float d3 = p3 * (bf(dp[e + 3]) - d.w);
-    if constexpr (kCap) {
+    if constexpr (kCap && kFromX) {
+      const float4 l = l2(j);
+      d0 *= cap_factor_x(bf(pr[c]), l.x, inv_cap_log2);
+      d1 *= cap_factor_x(bf(pr[c + 1]), l.y, inv_cap_log2);
+      d2 *= cap_factor_x(bf(pr[c + 2]), l.z, inv_cap_log2);
+      d3 *= cap_factor_x(bf(pr[c + 3]), l.w, inv_cap_log2);
+    } else if constexpr (kCap) {
       const float4 l = l2(j);
       d0 *= cap_factor(p0, l.x, inv_cap_log2);
       d1 *= cap_factor(p1, l.y, inv_cap_log2);
@@ -553,8 +590,9 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                              fmaf(slope2, fabsf(drow - c - 2.f), l2r), fmaf(slope2, fabsf(drow - c - 3.f), l2r));
         }, [&](int j) { return vis(4 * j); }, p);
       } else {
-        probs<64, kCap>(s, p.kscale, [&](int) { return l2r4; }, [&](int j) { return vis(4 * j); },
-                        p);
+        // with the cap, s keeps the exponents: nothing reads P before the grads step
+        probs<64, kCap, kCap>(s, p.kscale, [&](int) { return l2r4; },
+                              [&](int j) { return vis(4 * j); }, p);
       }
       ok = __all_sync(0xffffffffu, mbar_wait(bar(BAR_DP), t & 1, abort_flag, p.err, kSiteBwdS));
       if (!ok) break;
@@ -564,14 +602,14 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       tmem_ld_wait_x64(dp);
       {
         uint32_t pk[16], dsk[16];
-        grads<false, 0, 64, 64, kCap>(s, dp, [&](int) { return dr4; }, pk, dsk,
-                                      [&](int) { return l2r4; }, inv_cap);
+        grads<false, 0, 64, 64, kCap, kCap>(s, dp, [&](int) { return dr4; }, pk, dsk,
+                                            [&](int) { return l2r4; }, inv_cap);
         tmem_st_x16(tl + kTmemY + col, dsk);
       }
       {
         uint32_t pk[16], dsk[16];
-        grads<false, 32, 64, 64, kCap>(s, dp, [&](int) { return dr4; }, pk, dsk,
-                                       [&](int) { return l2r4; }, inv_cap);
+        grads<false, 32, 64, 64, kCap, kCap>(s, dp, [&](int) { return dr4; }, pk, dsk,
+                                             [&](int) { return l2r4; }, inv_cap);
         tmem_st_x16(tl + kTmemY + col + 16u, dsk);
       }
       tmem_wait_st();
