@@ -230,6 +230,7 @@ extern "C" int attn_fwd_alibi(const void* q, const void* k, const void* v, void*
   soft_cap_poly(p.cap_scale, p.cap_log2, p.cap_poly, p.cap_fast_max);
   p.mask = mask_params(mask_kind, window, doc_offsets, num_docs, Nq, Nk);
   p.alibi = alibi_slopes;
+  p.kv_reverse = alibi_slopes != nullptr ? 1 : 0;
   if ((long long)p.num_pairs * B * Hq > (1LL << 31) - 1) return ATTN_ERR_UNSUPPORTED;
   p.err = error_word_ptr(current_device());
   if (p.err == nullptr) return ATTN_ERR_CUDA;

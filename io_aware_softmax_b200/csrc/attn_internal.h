@@ -33,6 +33,10 @@ struct FwdParams {
   // for raw scores |s| <= cap_fast_max (|s cap_scale| <= 1/2); cap_fast_max < 0 disables it
   float cap_poly[5];
   float cap_fast_max;
+  // Units visit their K/V tiles last to first (ALiBi: the tiles nearest the diagonal hold
+  // the row maxima, so O is hardly ever rescaled; other calls keep the ascending order,
+  // which measured faster under a plain causal mask).
+  int kv_reverse;
   MaskParams mask;
   const float* alibi; // fp32 [Hq] ALiBi slopes (natural-log units per key of distance) or null
   // FP8 (E4M3) inputs, null otherwise: per 128-row block scales of Q and K, per head of V

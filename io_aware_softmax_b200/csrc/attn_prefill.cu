@@ -252,8 +252,9 @@ __device__ __forceinline__ float tile_row_exp_half(const uint32_t (&s)[128], int
   return ((a0 + a1) + (b0 + b1)) + ((c0 + c1) + (d0 + d1));
 }
 
-// K/V tiles [a, b] (relative to the CTA's first tile) that query tile t must visit; n = 0
-// when the tile has no valid row.
+// K/V tiles [a, b] (relative to the unit's first tile jt0) that query tile t must visit; n = 0
+// when the tile has no valid row.  make_pair_work turns them into the unit's steps that
+// visit them (the same numbers, or mirrored when the steps run last tile first).
 struct TileRange {
   int a, b, n;
 };
@@ -316,7 +317,23 @@ __device__ __forceinline__ PairWork make_pair_work(const FwdParams& p, int bh, i
   }
   w.rng[0] = tile_range(p, w.q0[0], w.jt0, w.n_tiles);
   w.rng[1] = tile_range(p, w.q0[1], w.jt0, w.n_tiles);
+  // p.kv_reverse: steps run from the last K/V tile to the first (step j takes tile
+  // jt0 + n_tiles - 1 - j, kv_tile_of_step), and each range becomes the steps that visit it.
+  // The tiles nearest the diagonal come first: under ALiBi they hold the row maxima, so the
+  // running max is set at once and O is hardly ever rescaled.
+  if (p.kv_reverse)
+    for (int t = 0; t < 2; ++t)
+      if (w.rng[t].n > 0) {
+        const int a = w.rng[t].a, b = w.rng[t].b;
+        w.rng[t].a = w.n_tiles - 1 - b;
+        w.rng[t].b = w.n_tiles - 1 - a;
+      }
   return w;
+}
+
+// Absolute index of the K/V tile that step j of unit w visits.
+__device__ __forceinline__ int kv_tile_of_step(const FwdParams& p, const PairWork& w, int j) {
+  return p.kv_reverse ? w.jt0 + w.n_tiles - 1 - j : w.jt0 + j;
 }
 
 // The CTA's sequence of query pairs (the grid is persistent: one CTA per SM).  Unit u of a
@@ -476,7 +493,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
               !mbar_wait(bar(BAR_EMPTY + s), (round - 1) & 1, abort_flag, p.err, kSiteEmpty))
             return false;
           mbar_arrive_expect_tx(bar(BAR_FULL + s), C::kTileBytes);
-          const int row = (w.jt0 + (i >> 1)) * kBN;
+          const int row = kv_tile_of_step(p, w, i >> 1) * kBN;
           const CUtensorMap* m = (i & 1) ? &tmV : &tmK;
           if (kFp8 && (i & 1)) {
             // FP8 V is stored transposed ([d][keys] per head): one box of d rows x 128 keys
@@ -708,7 +725,7 @@ attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmQ,
         tc_fence_after();
         uint32_t s[128];
         tmem_ld_x128(tS, s);
-        const int k0 = (w.jt0 + rng.a + i) * kBN;
+        const int k0 = kv_tile_of_step(p, w, rng.a + i) * kBN;
         const bool masked =
             !(lo_last <= k0 && k0 + kBN - 1 <= hi_first && k0 + kBN <= p.Nk);
         float mx;
