@@ -371,7 +371,8 @@ __device__ __forceinline__ void for_each_pair(const FwdParams& p, const int* sch
 // 2 G - 1 - c of every 2 G, G the grid -- which gives each CTA one of the heaviest and one of
 // the lightest of each round (within 2 % of the longest-first greedy deal on the packed-
 // document workload, against 20 % above the mean for dealing in index order).  keys is
-// scratch shared memory for the sort; the CTA's list goes to sched[0] (count), sched[1..].
+// scratch shared memory for the sort; the CTA's list goes to sched[0] (count), sched[1..],
+// in index order.
 __device__ __forceinline__ void build_schedule(const FwdParams& p, uint32_t* keys, int* sched) {
   const int P = p.num_pairs;
   const int U = p.B * (p.head_pairs ? p.Hq / 2 : p.Hq) * P;
@@ -406,9 +407,24 @@ __device__ __forceinline__ void build_schedule(const FwdParams& p, uint32_t* key
     const int m = r % G2;
     if (m == c || m == G2 - 1 - c) sched[1 + 2 * (r / G2) + (m >= G ? 1 : 0)] = (int)(keys[r] & 0xffffu);
   }
+  __syncthreads();
+  // The CTA runs its units in index order (head-major, query rows ascending), not in cost
+  // order: every CTA then moves through the heads at about the same pace, and a document's
+  // K/V tiles are read by its query tiles while they are still in L2 (in cost order the
+  // query tiles of one document run at scattered times and their K/V comes from DRAM again).
   if (threadIdx.x == 0) {
     const int rem = U % G2;
-    sched[0] = 2 * (U / G2) + (rem > c ? 1 : 0) + (rem > G2 - 1 - c ? 1 : 0);
+    const int n = 2 * (U / G2) + (rem > c ? 1 : 0) + (rem > G2 - 1 - c ? 1 : 0);
+    sched[0] = n;
+    for (int i = 2; i <= n; ++i) {           // insertion sort of sched[1..n], n <= kSchedMax
+      const int v = sched[i];
+      int j = i - 1;
+      while (j >= 1 && sched[j] > v) {
+        sched[j + 1] = sched[j];
+        --j;
+      }
+      sched[j + 1] = v;
+    }
   }
   // the K/V ring's copies will overwrite the keys through the async proxy
   fence_proxy_async_smem();
