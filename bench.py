@@ -754,7 +754,9 @@ def bench_fp8(w, args, world, local, peaks, peak_src):
                         "frac_of_hbm": round(quant_bytes / (qt * 1e-3) / 1e9 /
                                              float(peaks.get("hbm_gbs",
                                                              FALLBACK_PEAKS["hbm_gbs"])), 4),
-                        "launches": "Q, K, V: 1 each (V transposed, one scale per head, a cluster of 8 CTAs per head)"},
+                        "launches": "Q, K, V: 1 each (V transposed, one scale per head, a cluster of 8 CTAs per head)",
+                        "traffic": {"quant_rows (Q or K)": recorded_traffic("quant_rows"),
+                                    "quant_vt (V)": recorded_traffic("quant_vt")}},
            "accuracy": fp8_accuracy(w),
            "value": round(whole_job_rate(flops, world, ms) / 1e12, 2), "unit": "TFLOP/s",
            "ms_per_step": round(ms, 4), "steps": steps,
