@@ -12,7 +12,8 @@
 // the cache is read once per group, never replicated -- "3.7 어텐션 II", section 3.7.5),
 // a persistent grid of (SM count x resident CTAs) walks the (batch, kv-head, split) items,
 // and a producer warp keeps a 3-stage ring of 64-token K/V tiles in flight with TMA loads
-// (128B-swizzled, no multicast).  The four consumer warps each take 16 tokens of a stage.
+// (128B-swizzled, each CTA loading only into its own shared memory).  The four consumer
+// warps each take 16 tokens of a stage.
 // The two small products per 16 tokens (scores = q K^T with the G rows padded to 16, and
 // O += P V) use warp-level mma.sync so that the SM's issue slots stay free for the memory
 // pipeline; the tensor work is a few percent of what the tensor cores could do in the time

@@ -1,6 +1,7 @@
 // Thin inline-PTX wrappers for the sm_100a features the attention kernels use:
-// mbarriers, TMA tensor loads (no multicast anywhere), tcgen05 tensor-core MMAs with TMEM
-// accumulators, TMEM loads/stores, and bounded waits that report instead of hanging.
+// mbarriers, TMA tensor loads (each into the issuing CTA's own shared memory), tcgen05
+// tensor-core MMAs with TMEM accumulators, TMEM loads/stores, and bounded waits that report
+// instead of hanging.
 #pragma once
 
 #include <cstdint>
